@@ -1,0 +1,397 @@
+"""Benchmark of the key-only GLA forward pass (libgtr.so) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 640|1024|2048|stack|tiny] [--path auto|split|fused]
+                    [--no-sweep] [--no-cpu-baseline]
+
+One step = one gtr_gla_fwd call over one batch of synthetic input of the
+named workload (default: the 640^2 image, 40x40 grid, 1.6K tokens, 6 heads,
+fp16).  Directions rotate over the workload's direction list.  Inputs and
+outputs rotate over enough buffer sets that the working set exceeds the 126 MB
+L2 several times, so every step streams from HBM.  The K timed steps are
+captured in one CUDA graph (the pages time the operator under CUDA Graph) and
+timed with CUDA events on the capture stream, bracketed by a barrier and a
+device synchronise; under torchrun every rank runs its own replica and the
+slowest rank's time counts.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gtr_inputs import DTYPES, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "GLA fwd tokens/s and % of HBM roofline at 1.6K/4.1K/16.4K tokens, 1×B200"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FLOPS_PER_TOKEN_HEAD = 24704  # chunkwise, causal: 4*dk*dv + (C+1)(dk+dv)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def n_sets_for(w) -> int:
+    per = w.algorithmic_bytes()
+    return max(3, min(64, math.ceil(3 * L2_BYTES / per)))
+
+
+def make_sets(w, n, device, rank):
+    sets = []
+    for i in range(n):
+        d = w.direction_of_call(i)
+        q, k, v, lg = make_inputs(w, w.seed(d, i) + 100000 * rank, device=device)
+        out = torch.empty((w.B, w.L, w.heads, w.d_v), dtype=DTYPES[w.out_dtype], device=device)
+        sets.append((d, q, k, v, lg, out))
+    return sets
+
+
+def time_graph(gtr, w, sets, steps, warmup, path, stream, dist, device, per_call_events=True):
+    """Capture `steps` calls (rotating sets) in one graph; return (total_ms, per-call ms list)."""
+    ws = torch.empty(max(256, gtr.workspace_bytes(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
+                                                  {"f32": 0, "f16": 1, "bf16": 2}[w.dtype], path)),
+                     dtype=torch.uint8, device=device)
+
+    def call(i):
+        d, q, k, v, lg, out = sets[i % len(sets)]
+        gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=d, out=out, path=path, workspace=ws,
+                    stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 1)):
+            call(i)
+    torch.cuda.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)] if per_call_events else []
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            if per_call_events:
+                evs[i].record(stream)
+            call(i)
+        if per_call_events:
+            evs[steps].record(stream)
+    # warm the graph itself (W replays of one step's worth are not needed: one full replay)
+    g.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    start.record(stream)
+    g.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist)
+    total = start.elapsed_time(end)
+    per = []
+    if per_call_events:
+        try:
+            per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+        except RuntimeError:  # event nodes not timeable: fall back to the replay average
+            per = [total / steps] * steps
+    del g
+    return total, per
+
+
+def cpu_oracle_sample(w, seconds=10.0):
+    """Time the fp64 oracle on whole (batch, head) slices of the workload for ~`seconds`."""
+    import oracle
+    d = w.directions[0]
+    q, k, v, lg = make_inputs(w, w.seed(d))
+    sl = (slice(0, 1), slice(None), slice(0, 1), slice(None))
+    qs, ks, vs, gs = (t[sl].contiguous() for t in (q, k, v, lg))
+    oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)  # build + warm
+    threads = oracle.max_threads()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 1000:
+            break
+    tokens = n * w.L  # one head of one image per call
+    return {"value": tokens / el / w.heads, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} oracle calls on one (batch, head) slice of the {w.name} workload "
+                      f"(L={w.L}, d_k=d_v={w.d_k}, fp64), {el:.1f} s; token-heads/s divided by "
+                      f"{w.heads} heads to give image tokens/s"}
+
+
+def sweep(gtr, names, path, device, stream, hbm):
+    res = {}
+    for name in names:
+        w = WORKLOADS[name]
+        sets = make_sets(w, n_sets_for(w), device, 0)
+        steps = 2 * len(sets)
+        total, per = time_graph(gtr, w, sets, steps, 3, path, stream, None, device)
+        mean = sum(per) / len(per)
+        gbs = w.algorithmic_bytes() / (mean * 1e-3) / 1e9
+        res[name] = {"L": w.L, "tokens_per_s": w.B * w.L / (mean * 1e-3),
+                     "us_per_call": mean * 1e3, "GBps": gbs, "hbm_frac": gbs / hbm,
+                     "path": gtr.plan(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
+                                      {"f32": 0, "f16": 1, "bf16": 2}[w.dtype])[0]}
+        del sets
+        torch.cuda.empty_cache()
+    return res
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    import oracle
+    d = w.directions[0]
+    q, k, v, lg = make_inputs(w, w.seed(d))
+    sl = (slice(0, 1), slice(None), slice(0, 1), slice(None))
+    qs, ks, vs, gs = (t[sl].contiguous() for t in (q, k, v, lg))
+    for _ in range(args.warmup):
+        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+    el = time.perf_counter() - t0
+    value = args.steps * w.L / el / w.heads
+    sample = (f"each step: the fp64 oracle on one (batch, head) slice of the {w.name} workload "
+              f"(L={w.L}), token-heads/s divided by {w.heads} heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "grid": [w.H, w.W], "heads": w.heads,
+                       "d_k": w.d_k, "d_v": w.d_v, "seq_len": w.L, "in_dtype": w.dtype},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    world, rank, local = dist_env()
+    dist = init_dist(world, local)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import gated_token_recurrence_b200 as gtr
+
+    w = WORKLOADS[args.workload]
+    hbm, tc, peak_kind = peaks()
+    path_name, launches = gtr.plan(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
+                                   {"f32": 0, "f16": 1, "bf16": 2}[w.dtype])
+    if args.path != "auto":
+        path_name = args.path
+    stream = torch.cuda.Stream(device)
+    sets = make_sets(w, n_sets_for(w), device, rank)
+
+    uuid = str(getattr(torch.cuda.get_device_properties(device), "uuid", ""))
+    clocks = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or local))
+    clocks.start()
+    # soak ~1 s so the clock record covers a busy GPU, then the K timed steps
+    soak_steps = 4 * len(sets)
+    time_graph(gtr, w, sets, soak_steps, args.warmup, args.path, stream, None, device,
+               per_call_events=False)
+    total_ms, per = time_graph(gtr, w, sets, args.steps, args.warmup, args.path, stream, dist,
+                               device)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(dist, total_ms, device)
+    tokens_per_step = w.B * w.L
+    value = world * args.steps * tokens_per_step / (total_ms * 1e-3)
+    mean_call = sum(per) / len(per)
+    achieved = w.algorithmic_bytes() / (mean_call * 1e-3) / 1e9
+
+    # end to end through the host-buffer entry (pinned host memory, copies inside)
+    d0, q, k, v, lg, out = sets[0]
+    hq, hk, hv, hg = (t.cpu().pin_memory() for t in (q, k, v, lg))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        gtr.gla_fwd_host(hq, hk, hv, hg, hout, grid=(w.H, w.W), direction=d0, stream=stream)
+    barrier(dist)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        gtr.gla_fwd_host(hq, hk, hv, hg, hout, grid=(w.H, w.W), direction=d0, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1), device)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg))
+    d2h = hout.numel() * hout.element_size()
+
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_sweep:
+        extra["sweep"] = sweep(gtr, [n for n in ("640", "1024", "2048", "stack") if n != w.name],
+                               args.path, device, stream, hbm)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(w, seconds=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "grid": [w.H, w.W], "heads": w.heads,
+                       "d_k": w.d_k, "d_v": w.d_v, "seq_len": w.L, "global_batch": w.B * world,
+                       "in_dtype": w.dtype, "out_dtype": w.out_dtype,
+                       "directions": list(w.directions), "path": path_name,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "timing": "K steps in one CUDA graph, CUDA events on the capture stream",
+                       "l2": f"inputs and outputs rotate over {len(sets)} buffer sets "
+                             f"({len(sets) * w.algorithmic_bytes() / 2**20:.0f} MiB > L2)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": f"gtr_gla_fwd call ({launches} launch"
+                                   f"{'es' if launches != 1 else ''}, {path_name} path)",
+                         "bytes_per_call": w.algorithmic_bytes(),
+                         "us_per_call": mean_call * 1e3,
+                         "tensor_frac": (w.token_heads * FLOPS_PER_TOKEN_HEAD / (mean_call * 1e-3)
+                                         / 1e12) / tc},
+            "e2e": {"value": world * e2e_steps * tokens_per_step / (e2e_ms * 1e-3),
+                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * launches,
+            "clocks": clk,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="640", choices=sorted(WORKLOADS))
+    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

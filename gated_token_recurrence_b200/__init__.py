@@ -1,0 +1,179 @@
+"""Python binding of libgtr.so (key-only gated linear attention forward, sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libgtr.so``.  PyTorch supplies device memory and streams.  There
+is no CPU fallback: importing this package fails if the library is missing.
+
+    import gated_token_recurrence_b200 as gtr
+    out = gtr.gla_fwd(q, k, v, log_gamma, grid=(H, W), direction=gtr.L2R)
+
+Tensors are [B, L, heads, d] (log_gamma fp32 [B, L, heads, d_k]), contiguous,
+on the current CUDA device.  See include/gtr.h for the full contract.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgtr.so")
+
+L2R, R2L, T2B, B2T = 0, 1, 2, 3
+F32, F16, BF16 = 0, 1, 2
+PATH_AUTO, PATH_SPLIT, PATH_FUSED = 0, 1, 2
+PATHS = {"auto": PATH_AUTO, "split": PATH_SPLIT, "fused": PATH_FUSED}
+STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "GTR_ERR_CUDA",
+          4: "GTR_ERR_TIMEOUT", 5: "GTR_ERR_WORKSPACE"}
+
+# every symbol include/gtr.h declares
+EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
+            "gtr_gla_workspace_bytes", "gtr_gla_fwd_ex", "gtr_gla_fwd_host",
+            "gtr_gla_read_error", "gtr_gla_plan", "gtr_status_string", "gtr_version")
+
+
+class GTRError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}" if what else STATUS.get(status, str(status)))
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libgtr.so not found at {LIB_PATH}; build it with "
+            "`python gated_token_recurrence_b200/build.py` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    fwd_args = [vp] * 5 + [i] * 7
+    lib.gtr_gla_fwd.argtypes = fwd_args + [i, i, vp]
+    for name in ("gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32"):
+        getattr(lib, name).argtypes = fwd_args + [vp]
+    lib.gtr_gla_fwd_ex.argtypes = fwd_args + [i, i, i, vp, sz, vp]
+    lib.gtr_gla_fwd_host.argtypes = fwd_args + [i, i, vp]
+    lib.gtr_gla_workspace_bytes.argtypes = [i] * 8
+    lib.gtr_gla_workspace_bytes.restype = sz
+    lib.gtr_gla_read_error.argtypes = [vp, vp]
+    lib.gtr_gla_plan.argtypes = [i] * 7 + [ctypes.POINTER(i), ctypes.POINTER(i)]
+    lib.gtr_status_string.argtypes = [i]
+    lib.gtr_status_string.restype = ctypes.c_char_p
+    lib.gtr_version.argtypes = []
+    for name in ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
+                 "gtr_gla_fwd_ex", "gtr_gla_fwd_host", "gtr_gla_read_error", "gtr_gla_plan",
+                 "gtr_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}[t.dtype]
+
+
+def default_out_dtype(in_dtype):
+    """fp16 -> fp16, bf16 -> fp32, fp32 -> fp32."""
+    import torch
+    return torch.float16 if in_dtype == torch.float16 else torch.float32
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise GTRError(st, what)
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _shape(q, v, grid):
+    B, L, heads, d_k = q.shape
+    H, W = grid
+    if H * W != L:
+        raise ValueError(f"grid {H}x{W} does not match L={L}")
+    return B, heads, H, W, d_k, v.shape[-1]
+
+
+def workspace_bytes(B: int, heads: int, H: int, W: int, d_k: int = 64, d_v: int = 64,
+                    in_dtype: int = F16, path: str = "auto") -> int:
+    return int(lib.gtr_gla_workspace_bytes(B, heads, H, W, d_k, d_v, in_dtype, PATHS[path]))
+
+
+def gla_fwd(q, k, v, log_gamma, grid: Tuple[int, int], direction: int = L2R, out=None,
+            path: str = "auto", workspace=None, stream=None):
+    """Forward pass on CUDA tensors; returns ``out`` ([B, L, heads, d_v]).
+
+    ``workspace`` (a uint8 CUDA tensor of at least :func:`workspace_bytes`)
+    selects the caller-managed-workspace entry (no allocation, capturable);
+    without it the library's cached per-device workspace is used, and ``path``
+    must then be "auto".
+    """
+    import torch
+    B, heads, H, W, d_k, d_v = _shape(q, v, grid)
+    if out is None:
+        out = torch.empty((B, H * W, heads, d_v), dtype=default_out_dtype(q.dtype), device=q.device)
+    for t in (q, k, v, log_gamma, out):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("gla_fwd takes contiguous CUDA tensors")
+    if log_gamma.dtype != torch.float32:
+        raise ValueError("log_gamma must be float32")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share a dtype")
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), log_gamma.data_ptr(), out.data_ptr(),
+            B, heads, H, W, d_k, d_v, int(direction), _dtype_code(q), _dtype_code(out))
+    s = _stream_handle(stream)
+    if workspace is None and path == "auto":
+        _check(lib.gtr_gla_fwd(*args, s), "gtr_gla_fwd")
+    else:
+        if workspace is None:
+            nbytes = workspace_bytes(B, heads, H, W, d_k, d_v, _dtype_code(q), path)
+            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+        _check(lib.gtr_gla_fwd_ex(*args, PATHS[path], workspace.data_ptr(), workspace.numel(), s),
+               "gtr_gla_fwd_ex")
+    return out
+
+
+def gla_fwd_host(q, k, v, log_gamma, out, grid: Tuple[int, int], direction: int = L2R,
+                 stream=None):
+    """Forward pass on HOST (CPU, ideally pinned) tensors through ``gtr_gla_fwd_host``.
+
+    The library copies the inputs in, runs, copies ``out`` back and synchronises.
+    """
+    B, heads, H, W, d_k, d_v = _shape(q, v, grid)
+    for t in (q, k, v, log_gamma, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("gla_fwd_host takes contiguous CPU tensors")
+    st = lib.gtr_gla_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), log_gamma.data_ptr(),
+                              out.data_ptr(), B, heads, H, W, d_k, d_v, int(direction),
+                              _dtype_code(q), _dtype_code(out), _stream_handle(stream))
+    _check(st, "gtr_gla_fwd_host")
+    return out
+
+
+def plan(B: int, heads: int, H: int, W: int, d_k: int = 64, d_v: int = 64,
+         in_dtype: int = F16) -> Tuple[str, int]:
+    """(path name, kernel launches per call) that the dispatcher picks for this problem."""
+    path, launches = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.gtr_gla_plan(B, heads, H, W, d_k, d_v, in_dtype, ctypes.byref(path),
+                            ctypes.byref(launches)), "gtr_gla_plan")
+    name = {v: k for k, v in PATHS.items()}[path.value]
+    return name, launches.value
+
+
+def read_error(workspace=None, stream=None) -> int:
+    """Synchronise and return (and clear) the device error word; 0 = none."""
+    ptr = None if workspace is None else workspace.data_ptr()
+    return int(lib.gtr_gla_read_error(ptr, _stream_handle(stream)))
+
+
+def status_string(st: int) -> str:
+    return lib.gtr_status_string(int(st)).decode()
+
+
+def version() -> int:
+    return int(lib.gtr_version())

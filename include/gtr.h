@@ -1,0 +1,176 @@
+/*
+ * gtr.h - C ABI of libgtr.so: forward pass of key-only gated linear attention
+ * (GLA) over an H x W patch-token grid, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (GTR: Gated Token Recurrence for Efficient Dense Prediction;
+ * digest page paper.rainbus.top/paper/2609.26590, prerequisite "Gated linear
+ * attention (GLA)" and section "Core method"; page 0539edu.com, section 3.1):
+ *
+ *     S_t = Diag(gamma_t) S_{t-1} + k_t^T v_t,      S_{-1} = 0
+ *     o_t = d_k^{-1/2} q_t S_t
+ *
+ * per (batch, head), S_t in R^{d_k x d_v}, gamma_t in (0,1]^{d_k} a per-key-
+ * channel gate given as log_gamma = log(gamma) (the value side is not decayed),
+ * zero initial state, forward only (the operator specialisation in step 5 of
+ * that page's "Method details").  The L = grid_H * grid_W tokens are visited
+ * in one of four scan orders (section "Core method": left->right,
+ * right->left, top->bottom, bottom->top), read as:
+ *
+ *   GTR_L2R: rows top to bottom, each row x = 0 .. W-1
+ *   GTR_R2L: rows top to bottom, each row x = W-1 .. 0
+ *   GTR_T2B: columns left to right, each column y = 0 .. H-1
+ *   GTR_B2T: columns left to right, each column y = H-1 .. 0
+ *
+ * as one sequence: the state carries across line ends.  The work is done
+ * chunkwise (chunk C = 64): per-chunk summaries, a boundary-state scan and
+ * per-chunk outputs (first page, prerequisite "Chunkwise parallel"; page
+ * 0539edu.com section 3.3 "Hardware-aware chunked inference"), which reaches
+ * the sequential result up to rounding.
+ *
+ * LAYOUT.  q, k: [B, L, heads, d_k]; v: [B, L, heads, d_v]; log_gamma (always
+ * fp32): [B, L, heads, d_k]; out: [B, L, heads, d_v].  All row-major and
+ * contiguous; token index m = y * grid_W + x.  out[b, m, h, :] is the output
+ * of the token at grid cell m whatever the direction.
+ *
+ * OWNERSHIP.  The caller owns every buffer.  Device pointers must be 16-byte
+ * aligned and `out` must not overlap any input.  Nothing is retained after a
+ * call returns except the library's own cached workspace (below).
+ *
+ * ASYNCHRONY.  Device entry points enqueue work on `stream` (a cudaStream_t;
+ * NULL = legacy default stream) and return without synchronising.  Numerical
+ * preconditions, not checked on the device: log_gamma finite and <= 0.
+ *
+ * ERRORS.  Every entry point returns a gtr_status_t.  Argument problems are
+ * caught on the host before anything is enqueued (GTR_ERR_INVALID_ARG,
+ * GTR_ERR_UNSUPPORTED); launch failures return GTR_ERR_CUDA.  Failures found
+ * on the device (a bounded wait that ran out) are recorded in an error word
+ * inside the workspace and returned by gtr_gla_read_error().
+ */
+#ifndef GTR_H_
+#define GTR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t == struct CUstream_st* */
+typedef struct CUstream_st *gtr_stream_t;
+
+typedef enum { GTR_L2R = 0, GTR_R2L = 1, GTR_T2B = 2, GTR_B2T = 3 } gtr_direction_t;
+
+/* Element types.  log_gamma is always GTR_F32. */
+typedef enum { GTR_F32 = 0, GTR_F16 = 1, GTR_BF16 = 2 } gtr_dtype_t;
+
+typedef enum {
+    GTR_OK = 0,
+    GTR_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, bad enum */
+    GTR_ERR_UNSUPPORTED = 2, /* valid but not implemented (d_k, d_v, dtype pairing) */
+    GTR_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    GTR_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out (see gtr_gla_read_error) */
+    GTR_ERR_WORKSPACE = 5    /* workspace too small, or would have to grow during stream capture */
+} gtr_status_t;
+
+/* Execution paths.  GTR_PATH_AUTO lets the length-aware dispatcher choose. */
+typedef enum {
+    GTR_PATH_AUTO = 0,
+    GTR_PATH_SPLIT = 1, /* three launches: chunk summaries -> state scan -> chunk outputs (any dtype) */
+    GTR_PATH_FUSED = 2  /* single tensor-core launch (fp16/bf16 inputs) */
+} gtr_path_t;
+
+/*
+ * Supported shapes: d_k = d_v = 64.  dtype pairings (in -> out):
+ * F32 -> F32;  F16 -> F16 or F32;  BF16 -> F32 or BF16.
+ * Limits: B*heads <= 65535 * 64, L <= 2^28, B*L*heads*64 < 2^40 elements.
+ */
+
+/*
+ * Generic entry.  Uses a workspace owned by the library, cached per device
+ * and grown on demand with cudaMalloc (never while `stream` is being
+ * captured: that returns GTR_ERR_WORKSPACE - make one uncaptured call of the
+ * same or a larger size first).  Calls sharing the cached workspace must be
+ * ordered on the device (one stream, or synchronised streams); concurrent
+ * calls on independent streams need their own workspaces (gtr_gla_fwd_ws).
+ */
+gtr_status_t gtr_gla_fwd(const void *q, const void *k, const void *v,
+                         const float *log_gamma, void *out,
+                         int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                         int direction, int in_dtype, int out_dtype,
+                         gtr_stream_t stream);
+
+/* Typed forms with the problem's own argument list; the output dtype is
+ * F16 for F16 inputs and F32 for BF16 and F32 inputs. */
+gtr_status_t gtr_gla_fwd_f16(const void *q, const void *k, const void *v,
+                             const float *log_gamma, void *out, int B, int heads,
+                             int grid_H, int grid_W, int d_k, int d_v, int direction,
+                             gtr_stream_t stream);
+gtr_status_t gtr_gla_fwd_bf16(const void *q, const void *k, const void *v,
+                              const float *log_gamma, void *out, int B, int heads,
+                              int grid_H, int grid_W, int d_k, int d_v, int direction,
+                              gtr_stream_t stream);
+gtr_status_t gtr_gla_fwd_f32(const void *q, const void *k, const void *v,
+                             const float *log_gamma, void *out, int B, int heads,
+                             int grid_H, int grid_W, int d_k, int d_v, int direction,
+                             gtr_stream_t stream);
+
+/* Bytes of device workspace a gtr_gla_fwd_ex call with these arguments needs
+ * (for every path the dispatcher may choose).  0 for invalid arguments. */
+size_t gtr_gla_workspace_bytes(int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                               int in_dtype, int path);
+
+/*
+ * Caller-managed workspace (the persistent workspace of page 0539edu.com,
+ * appendix E.3.1): `workspace` is a device buffer of `ws_bytes` >=
+ * gtr_gla_workspace_bytes(...), 256-byte aligned.  The library allocates
+ * nothing and never synchronises, so the call can be captured in a CUDA
+ * graph.  The workspace's contents need no initialisation and may be reused
+ * by the next call once this one has finished on the device.  `path` is a
+ * gtr_path_t.
+ */
+gtr_status_t gtr_gla_fwd_ex(const void *q, const void *k, const void *v,
+                            const float *log_gamma, void *out,
+                            int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                            int direction, int in_dtype, int out_dtype, int path,
+                            void *workspace, size_t ws_bytes, gtr_stream_t stream);
+
+/*
+ * Host-buffer entry: q, k, v, log_gamma and out are HOST pointers (pinned
+ * memory gives full copy speed; pageable works).  The library copies the
+ * inputs to device buffers it caches per device, runs the forward pass on
+ * `stream`, copies the result back and synchronises `stream` before
+ * returning.  Not capturable.
+ */
+gtr_status_t gtr_gla_fwd_host(const void *q, const void *k, const void *v,
+                              const float *log_gamma, void *out,
+                              int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                              int direction, int in_dtype, int out_dtype,
+                              gtr_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of
+ * `workspace` (NULL = the library's cached workspace of the current device).
+ * GTR_OK when no device-side failure was recorded.
+ */
+gtr_status_t gtr_gla_read_error(void *workspace, gtr_stream_t stream);
+
+/*
+ * The length-aware dispatcher's decision for a problem: writes the path
+ * GTR_PATH_AUTO would take to *path and the number of kernel launches one
+ * call enqueues to *launches (either pointer may be NULL).  Host-only.
+ */
+gtr_status_t gtr_gla_plan(int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                          int in_dtype, int *path, int *launches);
+
+/* Human-readable name of a status code (static storage). */
+const char *gtr_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int gtr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTR_H_ */

@@ -1,0 +1,78 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, and rejects bad arguments on the host before anything reaches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_token_recurrence_b200 as gtr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*[\w\s\*]+?\b(gtr_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert "gtr_gla_fwd" in names and "gtr_gla_fwd_ex" in names
+    assert set(gtr.EXPORTED) <= set(names)
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(gtr.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_status_strings_and_version():
+    assert gtr.status_string(0) == "GTR_OK"
+    assert gtr.status_string(4) == "GTR_ERR_TIMEOUT"
+    assert gtr.status_string(99) == "GTR_ERR_UNKNOWN"
+    assert gtr.version() >= 100
+
+
+def _fwd_ex(**kw):
+    a = dict(q=16, k=16, v=16, g=16, out=16, B=1, heads=2, H=4, W=4, dk=64, dv=64, direction=0,
+             din=gtr.F16, dout=gtr.F16, path=0, ws=None, ws_bytes=0)
+    a.update(kw)
+    return gtr.lib.gtr_gla_fwd_ex(a["q"], a["k"], a["v"], a["g"], a["out"], a["B"], a["heads"],
+                                  a["H"], a["W"], a["dk"], a["dv"], a["direction"], a["din"],
+                                  a["dout"], a["path"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(g=8), 1),          # null / misaligned
+    (dict(B=0), 1), (dict(heads=-1), 1), (dict(H=0), 1), (dict(W=-3), 1),
+    (dict(direction=4), 1), (dict(direction=-1), 1), (dict(din=7), 1), (dict(path=9), 1),
+    (dict(dk=32), 2), (dict(dv=128), 2),                              # valid but unsupported
+    (dict(din=gtr.F32, dout=gtr.F16), 2), (dict(din=gtr.BF16, dout=gtr.F16), 2),
+    (dict(ws=None, ws_bytes=0), 5),                                   # workspace missing
+])
+def test_bad_arguments_rejected_on_host(kw, code):
+    assert _fwd_ex(**kw) == code
+
+
+def test_workspace_query():
+    n = gtr.workspace_bytes(1, 6, 40, 40, 64, 64, gtr.F16, "split")
+    units = 6 * 25
+    assert n == 256 + units * (2 * 64 * 64 + 64) * 4
+    assert gtr.workspace_bytes(1, 6, 40, 40, 64, 64, gtr.F16, "auto") >= n
+    assert gtr.workspace_bytes(0, 6, 40, 40) == 0
+    assert gtr.workspace_bytes(1, 6, 40, 40, 32, 64) == 0
+
+
+def test_typed_entries_validate_too():
+    f = gtr.lib.gtr_gla_fwd_f16
+    assert f(None, 16, 16, 16, 16, 1, 1, 8, 8, 64, 64, 0, None) == 1
+    assert gtr.lib.gtr_gla_fwd_f32(16, 16, 16, 16, 16, 1, 1, 8, 8, 64, 64, 9, None) == 1
+    assert gtr.lib.gtr_gla_fwd_bf16(16, 16, 16, 16, 16, 1, 1, 8, 8, 48, 64, 0, None) == 2

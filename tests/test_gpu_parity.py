@@ -1,0 +1,193 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Criterion (per output tensor): max |o - o_ref| <= tol * rms(o_ref), with
+tol = 1e-2 for fp16/bf16 inputs (fp32 accumulation) and 1e-5 for fp32 inputs.
+Every case draws its inputs from the seeded generators in gtr_inputs; the
+oracle sees exactly the bytes the GPU sees.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_token_recurrence_b200 as gtr
+import oracle
+from gtr_inputs import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "f16": 1e-2, "bf16": 1e-2}
+PATHS = ["split"]
+
+
+def rel_err(out: torch.Tensor, ref: np.ndarray) -> float:
+    o = out.detach().to("cpu", torch.float64).numpy()
+    assert np.isfinite(o).all(), "non-finite output"
+    return float(np.abs(o - ref).max() / np.sqrt(np.mean(ref ** 2)))
+
+
+def run_gpu(w: Workload, q, k, v, lg, direction, path="auto", out_dtype=None):
+    dev = torch.device("cuda:0")
+    out = None
+    if out_dtype is not None:
+        out = torch.empty((w.B, w.L, w.heads, w.d_v), dtype=out_dtype, device=dev)
+    o = gtr.gla_fwd(q.to(dev), k.to(dev), v.to(dev), lg.to(dev), grid=(w.H, w.W),
+                    direction=direction, out=out, path=path)
+    torch.cuda.synchronize()
+    return o
+
+
+def check(w: Workload, direction: int, seed: int, path="auto", out_dtype=None, tol=None):
+    q, k, v, lg = make_inputs(w, seed)
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, direction)
+    out = run_gpu(w, q, k, v, lg, direction, path, out_dtype)
+    err = rel_err(out, ref)
+    bound = TOL[w.dtype] if tol is None else tol
+    assert err <= bound, f"{w.name} dir={direction} path={path}: max err / rms = {err:.3e} > {bound}"
+    return err
+
+
+# ------------------------------------------------------------------ the five workloads
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+@pytest.mark.parametrize("name", ["tiny", "640", "1024", "2048"])
+def test_workload_all_directions(name, path):
+    w = WORKLOADS[name]
+    for d in w.directions:
+        check(w, d, w.seed(d), path)
+
+
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+def test_stack_workload_twelve_calls(path):
+    w = WORKLOADS["stack"]
+    for call in range(w.calls):
+        d = w.direction_of_call(call)
+        check(w, d, w.seed(d, call), path)
+
+
+def test_stack_workload_transposed_orientation():
+    w = WORKLOADS["stack"].with_(H=80, W=48, B=2)
+    for d in range(4):
+        check(w, d, 4700 + d)
+
+
+# ------------------------------------------------------------------ shapes and edge cases
+ODD = [
+    (1, 1, 1, 1), (1, 1, 1, 64), (1, 1, 64, 1), (1, 3, 7, 9), (2, 2, 5, 13), (1, 2, 33, 31),
+    (3, 1, 16, 20), (1, 4, 8, 200), (1, 2, 130, 3), (2, 3, 65, 1),
+]
+
+
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("shape", ODD)
+def test_ragged_and_degenerate_shapes(shape, dtype, path):
+    B, heads, H, W = shape
+    w = Workload("odd", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=1.0, index=9)
+    for d in range(4):
+        check(w, d, 9000 + 100 * H + W + d, path)
+
+
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+def test_strong_decay_gates(dtype, path):
+    """log gamma = logsigmoid(g - 2)/2: about -1 per token, a chunk decays by ~e^-70."""
+    w = Workload("strong", B=1, heads=2, H=24, W=24, dtype=dtype, gate_offset=-2.0, index=9)
+    q, k, v, g = make_inputs(w, 77)
+    lg = torch.nn.functional.logsigmoid(torch.logit(torch.exp(g * 16.0)) - 0.0) / 2.0
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 1)
+    out = run_gpu(w, q, k, v, lg, 1, path)
+    assert rel_err(out, ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+def test_no_decay_gates(path):
+    """log gamma = 0 exactly (causal linear attention); states grow with the sequence."""
+    w = Workload("nodecay", B=1, heads=2, H=32, W=40, dtype="bf16", index=9)
+    q, k, v, _ = make_inputs(w, 78)
+    lg = torch.zeros((w.B, w.L, w.heads, w.d_k), dtype=torch.float32)
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 2)
+    out = run_gpu(w, q, k, v, lg, 2, path)
+    assert rel_err(out, ref) <= 1e-2
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.float16])
+def test_fp16_inputs_either_output_dtype(out_dtype):
+    w = WORKLOADS["640"].with_(heads=2)
+    check(w, 3, 555, out_dtype=out_dtype)
+
+
+def test_bf16_inputs_bf16_output_runs():
+    """bf16 output is allowed; its own rounding costs ~2^-9 * max|o|, so the bound is looser."""
+    w = WORKLOADS["1024"].with_(heads=2, H=32)
+    check(w, 0, 556, out_dtype=torch.bfloat16, tol=3e-2)
+
+
+# ------------------------------------------------------------------ entry points agree
+def test_entry_points_agree_bitwise():
+    w = WORKLOADS["640"].with_(heads=3)
+    q, k, v, lg = make_inputs(w, 4242)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, lg))
+    a = gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), direction=1)
+    ws = torch.empty(gtr.workspace_bytes(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16), dtype=torch.uint8,
+                     device=dev)
+    b = gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), direction=1, workspace=ws)
+    c = torch.empty_like(a)
+    st = gtr.lib.gtr_gla_fwd_f16(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), gd.data_ptr(),
+                                 c.data_ptr(), w.B, w.heads, w.H, w.W, 64, 64, 1,
+                                 torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    host_out = torch.empty(a.shape, dtype=a.dtype).pin_memory()
+    gtr.gla_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), lg.pin_memory(), host_out,
+                     grid=(w.H, w.W), direction=1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(a, c)
+    assert torch.equal(a.cpu(), host_out)
+    assert gtr.read_error() == 0
+    assert gtr.read_error(ws) == 0
+
+
+def test_repeated_calls_are_deterministic():
+    w = WORKLOADS["1024"].with_(heads=4)
+    q, k, v, lg = (t.cuda() for t in make_inputs(w, 31))
+    a = gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=2)
+    b = gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=2)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_typed_bf16_and_f32_entries():
+    for name, fn, od in (("1024", gtr.lib.gtr_gla_fwd_bf16, torch.float32),
+                         ("tiny", gtr.lib.gtr_gla_fwd_f32, torch.float32)):
+        w = WORKLOADS[name].with_(heads=2)
+        q, k, v, lg = make_inputs(w, 99)
+        ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 3)
+        qd, kd, vd, gd = (t.cuda() for t in (q, k, v, lg))
+        out = torch.empty((w.B, w.L, w.heads, 64), dtype=od, device="cuda")
+        st = fn(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), gd.data_ptr(), out.data_ptr(), w.B,
+                w.heads, w.H, w.W, 64, 64, 3, torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        assert st == 0
+        assert rel_err(out, ref) <= TOL[w.dtype]
+
+
+def test_graph_capture_with_caller_workspace():
+    """gtr_gla_fwd_ex allocates nothing and can be captured in a CUDA graph."""
+    w = WORKLOADS["640"].with_(heads=2)
+    q, k, v, lg = make_inputs(w, 1234)
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 0)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, lg))
+    ws = torch.empty(gtr.workspace_bytes(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((w.B, w.L, w.heads, 64), dtype=torch.float16, device=dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), out=out, workspace=ws)  # warm-up outside capture
+    torch.cuda.synchronize()
+    out.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), out=out, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert rel_err(out, ref) <= 1e-2
