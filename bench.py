@@ -156,11 +156,11 @@ def make_sets(w, n, device, rank):
     return sets
 
 
-def time_graph(gtr, w, sets, steps, warmup, path, stream, dist, device, per_call_events=True):
+def time_graph(gtr, w, sets, steps, warmup, path, stream, dist, device, per_call_events=True,
+               check=True):
     """Capture `steps` calls (rotating sets) in one graph; return (total_ms, per-call ms list)."""
-    ws = torch.empty(max(256, gtr.workspace_bytes(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
-                                                  {"f32": 0, "f16": 1, "bf16": 2}[w.dtype], path)),
-                     dtype=torch.uint8, device=device)
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
+                           {"f32": 0, "f16": 1, "bf16": 2}[w.dtype], path, device)
 
     def call(i):
         d, q, k, v, lg, out = sets[i % len(sets)]
@@ -180,15 +180,26 @@ def time_graph(gtr, w, sets, steps, warmup, path, stream, dist, device, per_call
             call(i)
         if per_call_events:
             evs[steps].record(stream)
-    # warm the graph itself (W replays of one step's worth are not needed: one full replay)
-    g.replay()
+    # torch replays a graph on the CURRENT stream: make that the timed stream
+    with torch.cuda.stream(stream):
+        g.replay()  # warm replay
     torch.cuda.synchronize()
+    if check:
+        # the graph really did the work: its last output equals an eager call's, bit for bit
+        i = steps - 1
+        d, q, k, v, lg, out = sets[i % len(sets)]
+        ref = gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=d, path=path, workspace=ws,
+                          stream=stream)
+        torch.cuda.synchronize()
+        if not torch.equal(ref, out):
+            raise RuntimeError("graph replay output differs from an eager call")
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dist)
     torch.cuda.synchronize()
-    start.record(stream)
-    g.replay()
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        g.replay()
+        end.record(stream)
     torch.cuda.synchronize()
     barrier(dist)
     total = start.elapsed_time(end)
@@ -374,6 +385,22 @@ def run_ours(args):
     return 0
 
 
+def run_profile(args):
+    """Eager calls only (no graph, sweep, e2e or CPU leg): the command ncu captures."""
+    import gated_token_recurrence_b200 as gtr
+    device = torch.device("cuda", 0)
+    w = WORKLOADS[args.workload]
+    sets = make_sets(w, min(n_sets_for(w), 8), device, 0)
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
+                           {"f32": 0, "f16": 1, "bf16": 2}[w.dtype], args.path, device)
+    for i in range(args.warmup + args.steps):
+        d, q, k, v, lg, out = sets[i % len(sets)]
+        gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=d, out=out, path=args.path, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": w.name, "calls": args.warmup + args.steps, "path": args.path}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -385,11 +412,15 @@ def main(argv=None):
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="eager calls only, for ncu captures (prints no bench line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile(args)
     return run_ours(args)
 
 

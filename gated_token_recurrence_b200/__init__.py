@@ -29,7 +29,8 @@ STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "G
 # every symbol include/gtr.h declares
 EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
             "gtr_gla_workspace_bytes", "gtr_gla_fwd_ex", "gtr_gla_fwd_host",
-            "gtr_gla_read_error", "gtr_gla_plan", "gtr_status_string", "gtr_version")
+            "gtr_gla_read_error", "gtr_gla_plan", "gtr_gla_workspace_init", "gtr_status_string",
+            "gtr_version")
 
 
 class GTRError(RuntimeError):
@@ -54,13 +55,14 @@ def _load() -> ctypes.CDLL:
     lib.gtr_gla_workspace_bytes.argtypes = [i] * 8
     lib.gtr_gla_workspace_bytes.restype = sz
     lib.gtr_gla_read_error.argtypes = [vp, vp]
+    lib.gtr_gla_workspace_init.argtypes = [vp, sz, vp]
     lib.gtr_gla_plan.argtypes = [i] * 7 + [ctypes.POINTER(i), ctypes.POINTER(i)]
     lib.gtr_status_string.argtypes = [i]
     lib.gtr_status_string.restype = ctypes.c_char_p
     lib.gtr_version.argtypes = []
     for name in ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
                  "gtr_gla_fwd_ex", "gtr_gla_fwd_host", "gtr_gla_read_error", "gtr_gla_plan",
-                 "gtr_version"):
+                 "gtr_gla_workspace_init", "gtr_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -104,12 +106,21 @@ def workspace_bytes(B: int, heads: int, H: int, W: int, d_k: int = 64, d_v: int 
     return int(lib.gtr_gla_workspace_bytes(B, heads, H, W, d_k, d_v, in_dtype, PATHS[path]))
 
 
+def new_workspace(B: int, heads: int, H: int, W: int, d_k: int = 64, d_v: int = 64,
+                  in_dtype: int = F16, path: str = "auto", device=None):
+    """A zeroed uint8 CUDA tensor sized for :func:`gla_fwd` with ``workspace=``."""
+    import torch
+    n = max(256, workspace_bytes(B, heads, H, W, d_k, d_v, in_dtype, path))
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
 def gla_fwd(q, k, v, log_gamma, grid: Tuple[int, int], direction: int = L2R, out=None,
             path: str = "auto", workspace=None, stream=None):
     """Forward pass on CUDA tensors; returns ``out`` ([B, L, heads, d_v]).
 
-    ``workspace`` (a uint8 CUDA tensor of at least :func:`workspace_bytes`)
-    selects the caller-managed-workspace entry (no allocation, capturable);
+    ``workspace`` (a uint8 CUDA tensor of at least :func:`workspace_bytes`,
+    zeroed before its first use - see :func:`new_workspace`) selects the
+    caller-managed-workspace entry (no allocation, capturable);
     without it the library's cached per-device workspace is used, and ``path``
     must then be "auto".
     """
@@ -131,8 +142,7 @@ def gla_fwd(q, k, v, log_gamma, grid: Tuple[int, int], direction: int = L2R, out
         _check(lib.gtr_gla_fwd(*args, s), "gtr_gla_fwd")
     else:
         if workspace is None:
-            nbytes = workspace_bytes(B, heads, H, W, d_k, d_v, _dtype_code(q), path)
-            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+            workspace = new_workspace(B, heads, H, W, d_k, d_v, _dtype_code(q), path, q.device)
         _check(lib.gtr_gla_fwd_ex(*args, PATHS[path], workspace.data_ptr(), workspace.numel(), s),
                "gtr_gla_fwd_ex")
     return out

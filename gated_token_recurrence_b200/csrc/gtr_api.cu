@@ -118,9 +118,8 @@ gtr_status_t ensure(DeviceBuffer& buf, size_t bytes, cudaStream_t stream) {
     cudaGetLastError();
     return GTR_ERR_CUDA;
   }
-  // a zero header: the device error word starts clear
-  if (cudaMemsetAsync(buf.ptr, 0, sizeof(WsHeader) < want ? sizeof(WsHeader) : want, stream) != cudaSuccess)
-    return GTR_ERR_CUDA;
+  // a zeroed workspace is a ready one (clear error word, counters and flags)
+  if (cudaMemsetAsync(buf.ptr, 0, want, stream) != cudaSuccess) return GTR_ERR_CUDA;
   buf.bytes = want;
   return GTR_OK;
 }
@@ -218,6 +217,12 @@ gtr_status_t gtr_gla_fwd_ex(const void* q, const void* k, const void* v, const f
   const Problem p = make_problem(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v,
                                  direction, in_dtype, out_dtype);
   return run(p, path, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+gtr_status_t gtr_gla_workspace_init(void* workspace, size_t ws_bytes, gtr_stream_t stream) {
+  if (!workspace || !is_aligned(workspace, 256) || ws_bytes < sizeof(WsHeader)) return GTR_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? GTR_OK : GTR_ERR_CUDA;
 }
 
 gtr_status_t gtr_gla_fwd_host(const void* q, const void* k, const void* v, const float* log_gamma,

@@ -9,7 +9,8 @@ and the oracle's tests draw from here, so the two sides see identical bytes.
 Recipe (the same for every workload): a CPU ``torch.Generator`` seeded with
 ``seed`` draws q, k, v, g in that order, each fp32 N(0, 1) of shape
 [B, L, heads, d]; q, k, v are multiplied by ``scale`` and rounded to the
-storage dtype (round-to-nearest-even); ``log_gamma = logsigmoid(g + offset) / 16``
+storage dtype (round-to-nearest-even); ``log_gamma = logsigmoid(g + offset) / tau`` (tau = 16 unless a test asks for
+stronger gates)
 stays fp32.  The grids are the stride-16 patch grids of the images the GTR
 pages evaluate (640^2 -> 40x40, 1024^2 -> 64x64, 2048^2 -> 128x128,
 1280x768 -> 80 wide by 48 high).  No public dataset is involved.
@@ -41,6 +42,7 @@ class Workload:
     dtype: str = "f16"
     scale: float = 1.0
     gate_offset: float = 0.0
+    gate_tau: float = 16.0
     directions: tuple = (0,)
     calls: int = 1
     index: int = 0
@@ -110,7 +112,7 @@ def make_inputs(w: Workload, seed: int, device: Optional[str] = None):
     q = (q * w.scale).to(dt)
     k = (k * w.scale).to(dt)
     v = (v * w.scale).to(dt)
-    log_gamma = F.logsigmoid(g + w.gate_offset) / 16.0
+    log_gamma = F.logsigmoid(g + w.gate_offset) / w.gate_tau
     if device is not None:
         q, k, v, log_gamma = (t.to(device) for t in (q, k, v, log_gamma))
     return q, k, v, log_gamma

@@ -125,15 +125,19 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_H, int grid_W, int d_k
  * appendix E.3.1): `workspace` is a device buffer of `ws_bytes` >=
  * gtr_gla_workspace_bytes(...), 256-byte aligned.  The library allocates
  * nothing and never synchronises, so the call can be captured in a CUDA
- * graph.  The workspace's contents need no initialisation and may be reused
- * by the next call once this one has finished on the device.  `path` is a
- * gtr_path_t.
+ * graph.  A fresh workspace must be zeroed once before its first use
+ * (gtr_gla_workspace_init, or any memset to 0); after that every call leaves
+ * it ready for the next, so it may be reused by the next call once this one
+ * has finished on the device.  `path` is a gtr_path_t.
  */
 gtr_status_t gtr_gla_fwd_ex(const void *q, const void *k, const void *v,
                             const float *log_gamma, void *out,
                             int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
                             int direction, int in_dtype, int out_dtype, int path,
                             void *workspace, size_t ws_bytes, gtr_stream_t stream);
+
+/* Zero `ws_bytes` of a caller workspace on `stream` (asynchronous; capturable). */
+gtr_status_t gtr_gla_workspace_init(void *workspace, size_t ws_bytes, gtr_stream_t stream);
 
 /*
  * Host-buffer entry: q, k, v, log_gamma and out are HOST pointers (pinned

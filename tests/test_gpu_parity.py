@@ -90,9 +90,9 @@ def test_ragged_and_degenerate_shapes(shape, dtype, path):
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 def test_strong_decay_gates(dtype, path):
     """log gamma = logsigmoid(g - 2)/2: about -1 per token, a chunk decays by ~e^-70."""
-    w = Workload("strong", B=1, heads=2, H=24, W=24, dtype=dtype, gate_offset=-2.0, index=9)
-    q, k, v, g = make_inputs(w, 77)
-    lg = torch.nn.functional.logsigmoid(torch.logit(torch.exp(g * 16.0)) - 0.0) / 2.0
+    w = Workload("strong", B=1, heads=2, H=24, W=24, dtype=dtype, gate_offset=-2.0, gate_tau=2.0,
+                 index=9)
+    q, k, v, lg = make_inputs(w, 77)
     ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 1)
     out = run_gpu(w, q, k, v, lg, 1, path)
     assert rel_err(out, ref) <= TOL[dtype]
@@ -128,8 +128,7 @@ def test_entry_points_agree_bitwise():
     dev = torch.device("cuda:0")
     qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, lg))
     a = gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), direction=1)
-    ws = torch.empty(gtr.workspace_bytes(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16), dtype=torch.uint8,
-                     device=dev)
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16, device=dev)
     b = gtr.gla_fwd(qd, kd, vd, gd, grid=(w.H, w.W), direction=1, workspace=ws)
     c = torch.empty_like(a)
     st = gtr.lib.gtr_gla_fwd_f16(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), gd.data_ptr(),
@@ -179,6 +178,8 @@ def test_graph_capture_with_caller_workspace():
     qd, kd, vd, gd = (t.to(dev) for t in (q, k, v, lg))
     ws = torch.empty(gtr.workspace_bytes(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16), dtype=torch.uint8,
                      device=dev)
+    assert gtr.lib.gtr_gla_workspace_init(ws.data_ptr(), ws.numel(),
+                                          torch.cuda.current_stream().cuda_stream) == 0
     out = torch.empty((w.B, w.L, w.heads, 64), dtype=torch.float16, device=dev)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
