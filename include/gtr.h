@@ -153,6 +153,35 @@ gtr_status_t gtr_gla_fwd_host(const void *q, const void *k, const void *v,
                               gtr_stream_t stream);
 
 /*
+ * Allocation-free form of gtr_gla_fwd, for callers that may not call
+ * cudaMalloc (for instance a plugin inside an inference engine that allows
+ * device allocation only at build time, or a real-time loop that must not take
+ * cudaMalloc's implicit device synchronisation after start-up).  The paper has
+ * no counterpart: it is an interface convenience of this library.
+ *
+ * It runs the split path (GTR_PATH_SPLIT) with its scratch in a fixed
+ * 20 MiB array compiled into the library; every GPU that loads libgtr.so
+ * holds that array until the process exits.  Problems whose scratch,
+ * gtr_gla_workspace_bytes(..., GTR_PATH_SPLIT), exceeds 20 MiB - more than
+ * 636 chunk units B * heads * ceil(L / 64) - are refused on the host with
+ * GTR_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress while that device is current, and caches it; make that
+ * first call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents: calls that overlap on the GPU (different
+ * streams or threads without ordering) race and must be serialised by the
+ * caller.  Arguments, layouts and return codes are otherwise those of
+ * gtr_gla_fwd.
+ */
+gtr_status_t gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 const float *log_gamma, void *out,
+                                 int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                                 int direction, int in_dtype, int out_dtype,
+                                 gtr_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of
  * `workspace` (NULL = the library's cached workspace of the current device).
  * GTR_OK when no device-side failure was recorded.
