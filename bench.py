@@ -408,7 +408,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="640", choices=sorted(WORKLOADS))
-    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused"])
+    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused", "fused_sequential"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

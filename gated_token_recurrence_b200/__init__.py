@@ -21,10 +21,11 @@ LIB_PATH = os.path.join(_HERE, "libgtr.so")
 
 L2R, R2L, T2B, B2T = 0, 1, 2, 3
 F32, F16, BF16 = 0, 1, 2
-PATH_AUTO, PATH_SPLIT, PATH_FUSED = 0, 1, 2
-PATHS = {"auto": PATH_AUTO, "split": PATH_SPLIT, "fused": PATH_FUSED}
+PATH_AUTO, PATH_SPLIT, PATH_FUSED, PATH_FUSED_SEQUENTIAL = 0, 1, 2, 3
+PATHS = {"auto": PATH_AUTO, "split": PATH_SPLIT, "fused": PATH_FUSED,
+         "fused_sequential": PATH_FUSED_SEQUENTIAL}
 STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "GTR_ERR_CUDA",
-          4: "GTR_ERR_TIMEOUT", 5: "GTR_ERR_WORKSPACE"}
+          4: "GTR_ERR_TIMEOUT", 5: "GTR_ERR_WORKSPACE", 6: "GTR_ERR_RANGE"}
 
 # every symbol include/gtr.h declares
 EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",

@@ -58,23 +58,34 @@ Problem make_problem(const void* q, const void* k, const void* v, const float* g
 }
 
 // Length-aware dispatch.  The fused tensor-core path takes fp16/bf16 inputs;
-// fp32 inputs (exact FFMA arithmetic) take the split path.
+// fp32 inputs (exact FFMA arithmetic) and sequences shorter than one chunk take the
+// split path.  For a single partial chunk the fp16 rounding of the gate-scaled
+// operands is no longer averaged over many tokens (a cancelling dot product can
+// dominate the output), and the split path is just as fast there.
 int choose_path(const Problem& p, int requested) {
   if (requested != GTR_PATH_AUTO) return requested;
-  return GTR_PATH_SPLIT;
+  if (p.in_dtype == GTR_F32 || p.L() < kChunk) return GTR_PATH_SPLIT;
+  return GTR_PATH_FUSED;
+}
+
+bool fused_ok(const Problem& p) {
+  return p.in_dtype != GTR_F32 && (long long)p.B * p.L() < (1ll << 31);
 }
 
 size_t path_workspace_bytes(const Problem& p, int path) {
   switch (path) {
     case GTR_PATH_SPLIT: return split_workspace_bytes(p);
+    case GTR_PATH_FUSED:
+    case GTR_PATH_FUSED_SEQUENTIAL: return fused_ok(p) ? fused_workspace_bytes(p) : 0;
     default: return 0;
   }
 }
 
 int path_launches(const Problem& p, int path) {
-  (void)p;
   switch (path) {
     case GTR_PATH_SPLIT: return 3;
+    case GTR_PATH_FUSED:
+    case GTR_PATH_FUSED_SEQUENTIAL: return fused_launches(p);
     default: return 0;
   }
 }
@@ -131,6 +142,8 @@ gtr_status_t run(const Problem& p, int path, void* ws, size_t ws_bytes, cudaStre
   if (!ws || ws_bytes < need || !is_aligned(ws, 256)) return GTR_ERR_WORKSPACE;
   switch (chosen) {
     case GTR_PATH_SPLIT: return launch_split(p, ws, stream);
+    case GTR_PATH_FUSED: return launch_fused(p, ws, stream, -1);
+    case GTR_PATH_FUSED_SEQUENTIAL: return launch_fused(p, ws, stream, 0);
     default: return GTR_ERR_UNSUPPORTED;
   }
 }
@@ -193,12 +206,12 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_H, int grid_W, int d_k
                                int in_dtype, int path) {
   const int out_dtype = in_dtype == GTR_F16 ? GTR_F16 : GTR_F32;
   if (check_shape(B, heads, grid_H, grid_W, d_k, d_v, GTR_L2R, in_dtype, out_dtype) != GTR_OK) return 0;
-  if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED) return 0;
+  if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED_SEQUENTIAL) return 0;
   const Problem p = make_problem(nullptr, nullptr, nullptr, nullptr, nullptr, B, heads, grid_H,
                                  grid_W, d_k, d_v, GTR_L2R, in_dtype, out_dtype);
   if (path != GTR_PATH_AUTO) return path_workspace_bytes(p, path);
   size_t m = 0;
-  for (int pth = GTR_PATH_SPLIT; pth <= GTR_PATH_FUSED; ++pth) {
+  for (int pth = GTR_PATH_SPLIT; pth <= GTR_PATH_FUSED_SEQUENTIAL; ++pth) {
     const size_t b = path_workspace_bytes(p, pth);
     if (b > m) m = b;
   }
@@ -213,7 +226,7 @@ gtr_status_t gtr_gla_fwd_ex(const void* q, const void* k, const void* v, const f
   if (st != GTR_OK) return st;
   st = check_ptrs(q, k, v, log_gamma, out);
   if (st != GTR_OK) return st;
-  if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED) return GTR_ERR_INVALID_ARG;
+  if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED_SEQUENTIAL) return GTR_ERR_INVALID_ARG;
   const Problem p = make_problem(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v,
                                  direction, in_dtype, out_dtype);
   return run(p, path, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
@@ -290,6 +303,8 @@ gtr_status_t gtr_gla_read_error(void* workspace, gtr_stream_t stream_) {
   if (h.error) {
     const unsigned int zero[2] = {0u, 0u};
     if (cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return GTR_ERR_CUDA;
+    // a call that gave up on a wait may have left its arrival counters behind: clear them
+    if (h.error == GTR_ERR_TIMEOUT && cudaMemset(ws, 0, fused_reset_bytes()) != cudaSuccess) return GTR_ERR_CUDA;
   }
   return static_cast<gtr_status_t>(h.error);
 }
@@ -315,6 +330,7 @@ const char* gtr_status_string(int status) {
     case GTR_ERR_CUDA: return "GTR_ERR_CUDA";
     case GTR_ERR_TIMEOUT: return "GTR_ERR_TIMEOUT";
     case GTR_ERR_WORKSPACE: return "GTR_ERR_WORKSPACE";
+    case GTR_ERR_RANGE: return "GTR_ERR_RANGE";
     default: return "GTR_ERR_UNKNOWN";
   }
 }

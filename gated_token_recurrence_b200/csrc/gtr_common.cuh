@@ -23,6 +23,12 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must stay 256 bytes");
 
+// Every workspace starts with the header and a fixed 2 KB region of per-sequence
+// arrival counters (used by the fused path, kept zero between calls); each path's own
+// arrays start after this prefix, so calls of different paths can share a workspace.
+constexpr size_t kWsCounterBytes = 2048;
+constexpr size_t kWsPrefixBytes = sizeof(WsHeader) + kWsCounterBytes;
+
 struct Problem {
   const void* q;
   const void* k;

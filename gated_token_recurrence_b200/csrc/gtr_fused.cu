@@ -1,0 +1,1030 @@
+// Fused path: one launch, tcgen05 tensor cores, fp16/bf16 inputs.
+//
+// The chunkwise operator of page 0539edu.com, section 3.3 (chunk summaries ->
+// light boundary-state scan -> per-chunk outputs; intra-chunk causal scores
+// consumed on chip) and of the first GTR page, prerequisite "Chunkwise
+// parallel", built as one persistent, warp-specialised sm_100a kernel.
+//
+// Per chunk of C = 64 scan positions of one (batch, head), with A the in-chunk
+// inclusive cumsum of log2-gates and a = A[last] (per key channel):
+//   Qh = Q * 2^A   (<= |q|)     Kh = K * 2^-A   (>= |k|, bounded by the chunk's decay)
+//   P  = mask_{j<=i}(Qh Kh^T)   = sum_k q_ik k_jk 2^(A_ik - A_jk)
+//   O  = Qh S + P V             (S = state at the chunk start)
+//   U' = Kh^T V,  S <- 2^a * (S + U')     (= Diag(d) S + K~^T V with K~ = K * 2^(a - A))
+// All MMA operands are fp16 (bf16 inputs convert exactly inside the fp16 range);
+// accumulation and the state are fp32.  A chunk whose gates decay too fast for
+// the factorisation to stay inside fp16 gets its scores from the CUDA cores
+// (2^(A_i - A_j) per pair).  Values beyond the fp16 operand range are reported
+// as GTR_ERR_RANGE.
+//
+// Two modes.  STREAM: one CTA walks a whole sequence, carrying the exact fp32
+// state.  HOLD: the n_s CTAs of a sequence each take a segment of every round;
+// a CTA computes its chunks from a zero segment-start state and keeps the outputs
+// in tensor memory, the n_s CTAs scan the segment summaries (each owns a slice of
+// the 64x64 state entries), and each CTA adds (Q * 2^(A from its segment start))
+// times its segment-start state to the held outputs.  Round r's scan and
+// epilogue overlap round r+1's chunks (two held sets).
+//
+// Warp roles (480 threads):
+//   warps 0-3   WG_A  load-side math: cumulative gates, Qh / Kh tiles, held tiles
+//   warps 4-7   WG_B  score masking, fp32 state update, STREAM epilogue
+//   warps 8-11  WG_C  HOLD round end: summary scan, correction, epilogue
+//   warps 12-13 producer: cp.async of one token row per thread (direction remap,
+//               128-byte-swizzled placement, zero fill past the sequence end)
+//   warp 14     tcgen05 MMA issuer and tensor-memory owner
+#include <atomic>
+#include <mutex>
+#include <type_traits>
+
+#include "gtr_common.cuh"
+#include "gtr_internal.h"
+#include "gtr_sm100.cuh"
+
+namespace gtr {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 2;          // TMA staging depth (chunks in flight)
+constexpr int kHeldPerSet = 3;      // chunks held per CTA per round (HOLD)
+constexpr int kThreads = 480;
+constexpr int kProducerThreads = 64;
+constexpr int kMmaWarp = 14;
+constexpr int kWG = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kF16Safe = 60000.f;  // largest magnitude an fp16 operand may carry
+
+// shared memory (bytes); every 16-bit tile is [64][64], 128 B rows, 128 B swizzle
+constexpr int kTile = 8192;
+constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
+constexpr int kStageBytes = 3 * kTile + kGTile;      // Q, K, V, G
+constexpr int kOffStage = 0;
+constexpr int kOffOp = kOffStage + kStages * kStageBytes;  // [2] x (Qh, Kh)
+constexpr int kOffP = kOffOp + 2 * 2 * kTile;              // [2]
+constexpr int kOffS = kOffP + 2 * kTile;                   // [2]
+constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
+constexpr int kOffHeld = kOffSst + kTile;                  // [2 sets][kHeldPerSet]
+constexpr int kOffOut = kOffHeld + 2 * kHeldPerSet * kTile;  // 64 rows x 256 B staging
+constexpr int kOffMisc = kOffOut + 16384;
+constexpr int kMiscBytes = 3072;
+constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+
+// tensor memory columns
+constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0) and U' (lane tile 1)
+constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 outputs; HOLD: [2 sets] x 128 held outputs
+constexpr uint32_t kLaneTile1 = 16u << 16;
+
+// HOLD-mode counters sit at a fixed place right after the workspace header, whatever
+// the problem size, so that a workspace kept zero between calls stays valid across shapes.
+constexpr size_t kMaxHoldSegments = 256;  // CTAs of one launch in HOLD mode (>= the SM count)
+constexpr size_t kCounterBytes = 2 * kMaxHoldSegments * sizeof(unsigned int);
+static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
+constexpr int kMaxOwn = 16;               // state entries per WG_C thread (n_s >= 2)
+
+struct FusedParams {
+  Problem p;
+  WsHeader* hdr;
+  unsigned int* counters;  // [n_seq][2], monotonic within a call, zero between calls
+  float* agg;              // [n_seq][2 round parities][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
+  uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
+  int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD
+  int grid;
+  float scale;
+  float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
+};
+
+struct Misc {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t opready[2], opfree[2], su_full[2], su_free[2], sready[2], pready[2], o_full[2], o_free[2];
+  uint64_t agg_pub[2], corr_ready[2], corr_done[2], set_free[2];
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  int abort;
+  int go[3][2];          // per-warpgroup wait decisions, alternating slots
+  int fb[2];             // chunk parity -> scores from the CUDA cores
+  alignas(16) float red[4][64];  // WG_A cumsum: per-warp channel totals
+  float a2last[2][64];   // chunk parity -> in-chunk log2 decay per channel
+};
+static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// 2^x on the special-function unit.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Bounded mbarrier wait: the thread sleeps in hardware until the phase completes; only
+// after about a second without completion does the CTA record a timeout and abort.
+__device__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+  if (mbar_wait_sleep(bar, parity, 1000000u)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (*(volatile int*)&ms->abort) return false;
+    if (mbar_wait_sleep(bar, parity, 1000000u)) return true;
+    if (globaltimer() - t0 > 1000000000ull) {
+      record_error(hdr, GTR_ERR_TIMEOUT, where);
+      *(volatile int*)&ms->abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait until a global counter reaches `target`.
+__device__ bool wait_counter(const unsigned int* ctr, unsigned int target, Misc* ms, WsHeader* hdr,
+                             uint32_t where) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (*(volatile int*)&ms->abort) return false;
+    if (globaltimer() - t0 > 1000000000ull) {
+      record_error(hdr, GTR_ERR_TIMEOUT, where);
+      *(volatile int*)&ms->abort = 1;
+      return false;
+    }
+    __nanosleep(128);
+  }
+}
+
+__device__ __forceinline__ void red_release_add(unsigned int* ctr, unsigned int v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(v) : "memory");
+}
+
+// Named barrier of one 128-thread warpgroup (ids 1..3).
+__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory"); }
+
+// Warpgroup wait: its first thread does the bounded wait, then every thread of the
+// group takes the same decision (no thread is left alone at a named barrier) and
+// observes the completed phase itself.
+__device__ bool wg_wait(int wg, int wtid, uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr,
+                        uint32_t where, int& slot) {
+  if (wtid == 0) {
+    const bool ok = wait_bar(bar, parity, ms, hdr, where);
+    ms->go[wg][slot] = ok && !*(volatile int*)&ms->abort;
+  }
+  wg_sync(wg);
+  const bool go = *(volatile int*)&ms->go[wg][slot] != 0;
+  slot ^= 1;
+  if (go) (void)mbar_try_wait(bar, parity);
+  return go;
+}
+
+__device__ bool wg_agree(int wg, int wtid, bool ok0, Misc* ms, int& slot) {
+  if (wtid == 0) ms->go[wg][slot] = ok0 && !*(volatile int*)&ms->abort;
+  wg_sync(wg);
+  const bool go = *(volatile int*)&ms->go[wg][slot] != 0;
+  slot ^= 1;
+  return go;
+}
+
+template <typename T> struct Pack2;
+template <> struct Pack2<__half> {
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack(uint32_t u) {
+    return __half22float2(*reinterpret_cast<__half2*>(&u));
+  }
+};
+template <> struct Pack2<__nv_bfloat16> {
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ float2 unpack(uint32_t u) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+  }
+};
+
+__device__ __forceinline__ bool f16_ok(float x) { return fabsf(x) <= kF16Safe; }
+
+// Scale 16 output values (columns cb..cb+15 of one row) and stage them, in the
+// output dtype, in a linear shared-memory row for a bulk store.
+template <typename Tout>
+__device__ __forceinline__ void stage_out16(uint8_t* orow, int cb, float* v, float scale) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] *= scale;
+  if constexpr (sizeof(Tout) == 4) {
+#pragma unroll
+    for (int e = 0; e < 16; e += 4)
+      *reinterpret_cast<float4*>(orow + (cb + e) * 4) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+  } else {
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pk[e] = Pack2<Tout>::pack(v[2 * e], v[2 * e + 1]);
+    *reinterpret_cast<uint4*>(orow + cb * 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(orow + cb * 2 + 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  }
+}
+
+// Store one staged 64-value output row (a token-head) at its grid cell.
+template <typename Tout>
+__device__ __forceinline__ void store_row(const Problem& p, int b, int h, long long s, const uint8_t* orow) {
+  const long long L = p.L();
+  const long long m = scan_to_token(s, p.direction, p.H, p.W);
+  uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + (((long long)b * L + m) * p.heads + h) * 64 * sizeof(Tout);
+  fence_proxy_async_smem();
+  bulk_store(dst, orow, 64 * sizeof(Tout));
+  bulk_commit();
+}
+
+// TMEM row (lane tile 0 or 1 of this warp's lane quarter) of a 64-column region ->
+// scaled output row, stored.  All 32 lanes take part in the loads; `mine` lanes store.
+template <typename Tout>
+__device__ __forceinline__ void epilogue_rows(const Problem& p, int b, int h, uint32_t taddr, bool mine,
+                                              long long s_row, uint8_t* orow, float scale) {
+#pragma unroll
+  for (int cb = 0; cb < 64; cb += 16) {
+    float v[16];
+    tmem_ld16(taddr + cb, v);
+    tmem_wait_ld();
+    if (mine) stage_out16<Tout>(orow, cb, v, scale);
+  }
+  if (mine && s_row < p.L()) store_row<Tout>(p, b, h, s_row, orow);
+}
+
+struct Span {
+  int c0, c1;
+};
+
+// Chunk range of segment s in round r: every segment of every round holds Gr chunks
+// (Gr = ceil(Nc / (n_s * rounds)) <= kHeldPerSet) except at the sequence end.
+__device__ __forceinline__ Span round_span(const FusedParams& fp, int r, int s) {
+  if (fp.mode == 0) return Span{0, fp.Nc};
+  const int gr = (fp.Nc + fp.n_s * fp.rounds - 1) / (fp.n_s * fp.rounds);
+  Span sp;
+  sp.c0 = min(fp.Nc, (r * fp.n_s + s) * gr);
+  sp.c1 = min(fp.Nc, (r * fp.n_s + s + 1) * gr);
+  return sp;
+}
+
+// Phase parity for the n-th use of a double-buffered barrier, and for waiting on its
+// release by use n-2 (passes at once for n < 2 on a fresh barrier).
+__device__ __forceinline__ uint32_t ph_of(int n) { return (uint32_t)(n >> 1) & 1u; }
+__device__ __forceinline__ uint32_t ph_free(int n) { return ((uint32_t)(n >> 1) & 1u) ^ 1u; }
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_gla_kernel(const __grid_constant__ FusedParams fp) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Misc* ms = reinterpret_cast<Misc*>(smem + kOffMisc);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const Problem& p = fp.p;
+  WsHeader* hdr = fp.hdr;
+
+  const bool hold = fp.mode == 1;
+  const int seq = hold ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
+  const int seg = hold ? (int)blockIdx.x % fp.n_s : 0;
+  const int b = seq / p.heads, h = seq % p.heads;
+  const long long L = p.L();
+  const int rounds = hold ? fp.rounds : 1;
+  bool range_bad = false;
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&ms->full[i], kProducerThreads);
+      mbar_init(&ms->empty[i], 2);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms->opready[i], 1);
+      mbar_init(&ms->opfree[i], 1);
+      mbar_init(&ms->su_full[i], 1);
+      mbar_init(&ms->su_free[i], 1);
+      mbar_init(&ms->sready[i], 1);
+      mbar_init(&ms->pready[i], 1);
+      mbar_init(&ms->o_full[i], 1);
+      mbar_init(&ms->o_free[i], 1);
+      mbar_init(&ms->agg_pub[i], 1);
+      mbar_init(&ms->corr_ready[i], 1);
+      mbar_init(&ms->corr_done[i], 1);
+      mbar_init(&ms->set_free[i], 1);
+    }
+    mbar_init(&ms->mma_final, 1);
+    ms->abort = 0;
+    for (int i = 0; i < 3; ++i) ms->go[i][0] = ms->go[i][1] = 0;
+    ms->fb[0] = ms->fb[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&ms->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 12 || warp == 13) {
+    // ===================================================================== producer (cp.async)
+    // Thread t loads row t (scan position c*64 + t) of Q, K, V (128 B each, placed in
+    // the 128-byte-swizzle layout) and of the log-gates (256 B, plain).  Rows past the
+    // sequence end are zero-filled (source size 0).
+    const int pt = tid - 12 * 32;  // 0..63 = chunk row
+    int n = 0;
+    bool stop = false;
+    const uint8_t* gq = reinterpret_cast<const uint8_t*>(p.q);
+    const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.k);
+    const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.v);
+    const uint8_t* gg = reinterpret_cast<const uint8_t*>(p.log_gamma);
+    for (int r = 0; r < rounds && !stop; ++r) {
+      const Span sp = round_span(fp, r, seg);
+      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
+        const int st = n % kStages;
+        int ok = 0;
+        if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
+        uint8_t* sb = smem + kOffStage + st * kStageBytes;
+        const long long s = (long long)c * kChunk + pt;
+        const bool valid = s < L;
+        const long long row = valid ? token_head_row(p, b, h, s) : 0;
+        const uint32_t nb = valid ? 16u : 0u;
+        const uint8_t* q16 = gq + row * 128;
+        const uint8_t* k16 = gk + row * 128;
+        const uint8_t* v16 = gv + row * 128;
+        const uint8_t* g32 = gg + row * 256;
+        const uint32_t d0 = smem_u32(sb) + pt * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t sw = (uint32_t)((j ^ (pt & 7)) << 4);
+          cp_async16(d0 + sw, q16 + 16 * j, nb);
+          cp_async16(d0 + kTile + sw, k16 + 16 * j, nb);
+          cp_async16(d0 + 2 * kTile + sw, v16 + 16 * j, nb);
+        }
+        const uint32_t dg = smem_u32(sb) + 3 * kTile + pt * 256;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cp_async16(dg + 16 * j, g32 + 16 * j, nb);
+        cp_async_arrive_noinc(&ms->full[st]);
+      }
+    }
+    if (stop) {
+      // copies already issued must land before this CTA's shared memory is released
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+  } else if (warp == kMmaWarp) {
+    // ===================================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_f16(0, 64, 64, 0, 0);  // A K-major, B K-major
+      const uint32_t id_kv = idesc_f16(0, 64, 64, 1, 1);  // A MN-major, B MN-major
+      const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);  // A K-major, B MN-major
+      const uint32_t s_base = smem_u32(smem);
+      int n = 0;
+      int next_corr = 0;  // oldest round whose correction is not issued yet (HOLD)
+      bool ok = true;
+      // held outputs of round rc += (Q 2^(A_seg)) S_segment_start
+      auto issue_corr = [&](int rc, bool block) -> bool {
+        const int sig = rc & 1;
+        if (block) {
+          if (!wait_bar(&ms->corr_ready[sig], ph_of(rc), ms, hdr, 0x205)) return false;
+        } else if (!mbar_try_wait(&ms->corr_ready[sig], ph_of(rc))) {
+          return false;
+        }
+        tc_fence_after();
+        const Span spc = round_span(fp, rc, seg);
+        const int G = spc.c1 - spc.c0;
+        for (int g = 0; g < G; ++g) {
+          const uint32_t d_o = tmem + kColO + 128u * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+          const uint32_t a_h = s_base + kOffHeld + (sig * kHeldPerSet + g) * kTile;
+          for (int k = 0; k < 4; ++k)
+            mma_f16(d_o, sw128_desc(a_h + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
+        }
+        mma_commit(&ms->corr_done[sig]);
+        return true;
+      };
+      for (int r = 0; r < rounds && ok; ++r) {
+        const Span sp = round_span(fp, r, seg);
+        const int sig = r & 1;
+        if (hold && r >= 2) {
+          // this set's held slots are reused: round r-2's correction must be issued and its
+          // epilogue finished first
+          while (ok && next_corr <= r - 2) ok = issue_corr(next_corr++, true);
+          if (!ok || !wait_bar(&ms->set_free[sig], ph_free(r), ms, hdr, 0x206)) { ok = false; break; }
+        }
+        for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
+          const int bb = n & 1, st = n % kStages;
+          const uint32_t op = s_base + kOffOp + bb * 2 * kTile;  // Qh, then Kh
+          const uint32_t a_v = s_base + kOffStage + st * kStageBytes + 2 * kTile;
+          if (!wait_bar(&ms->opready[bb], ph_of(n), ms, hdr, 0x200) ||
+              !wait_bar(&ms->su_free[bb], ph_free(n), ms, hdr, 0x201)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t su = tmem + kColSU + 64u * bb;
+          for (int k = 0; k < 4; ++k)  // scores = Qh Kh^T
+            mma_f16(su, sw128_desc(op + 32 * k), sw128_desc(op + kTile + 32 * k), id_qk, k > 0);
+          for (int k = 0; k < 4; ++k)  // U' = Kh^T V
+            mma_f16(su + kLaneTile1, sw128_desc(op + kTile + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
+          mma_commit(&ms->su_full[bb]);
+          uint32_t d_o;
+          if (hold) {
+            d_o = tmem + kColO + 128u * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+          } else {
+            d_o = tmem + kColO + 64u * bb;
+            if (!wait_bar(&ms->o_free[bb], ph_free(n), ms, hdr, 0x202)) { ok = false; break; }
+          }
+          if (!wait_bar(&ms->sready[bb], ph_of(n), ms, hdr, 0x203)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_s = s_base + kOffS + bb * kTile;
+          for (int k = 0; k < 4; ++k)  // O = Qh S
+            mma_f16(d_o, sw128_desc(op + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
+          if (!wait_bar(&ms->pready[bb], ph_of(n), ms, hdr, 0x204)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_p = s_base + kOffP + bb * kTile;
+          for (int k = 0; k < 4; ++k)  // O += P V
+            mma_f16(d_o, sw128_desc(a_p + 32 * k), sw128_desc(a_v + 2048 * k), id_qs, 1);
+          mma_commit(&ms->o_full[bb]);
+          mma_commit(&ms->opfree[bb]);
+          mma_commit(&ms->empty[st]);
+          if (hold && next_corr < r && issue_corr(next_corr, false)) ++next_corr;
+        }
+      }
+      while (ok && hold && next_corr < rounds) ok = issue_corr(next_corr++, true);
+      // every MMA issued here has completed before tensor memory is freed
+      mma_commit(&ms->mma_final);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&ms->mma_final, 0) && globaltimer() - t0 < 1000000000ull) {
+      }
+    }
+  } else if (warp < 4) {
+    // ===================================================================== WG_A: operand tiles
+    const int wg = 0, wtid = tid;
+    const int cc = wtid & 7;   // channels 8cc .. 8cc+7
+    const int rb = wtid >> 3;  // rows 4rb .. 4rb+3
+    float a2seg[8];            // log2 decay from the segment start, per channel (HOLD)
+    int slot = 0, n = 0;
+    bool alive = true;
+    for (int r = 0; r < rounds && alive; ++r) {
+      const Span sp = round_span(fp, r, seg);
+      const int sig = r & 1;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a2seg[e] = 0.f;
+      if (hold && r >= 2 && sp.c1 > sp.c0 &&
+          !wg_wait(wg, wtid, &ms->set_free[sig], ph_free(r), ms, hdr, 0x300, slot)) { alive = false; break; }
+      for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
+        const int bb = n & 1, st = n % kStages;
+        if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot) ||
+            !wg_wait(wg, wtid, &ms->opfree[bb], ph_free(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+        uint8_t* sb = smem + kOffStage + st * kStageBytes;
+        float* G = reinterpret_cast<float*>(sb + 3 * kTile);
+        // ---- in-chunk cumulative log2-gates: my 4 rows, then a scan over the 16 row blocks
+        float A[4][8];
+        float run[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) run[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4* gp = reinterpret_cast<const float4*>(G + (4 * rb + i) * 64 + 8 * cc);
+          const float4 g0 = gp[0], g1 = gp[1];
+          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            run[e] = fmaf(gv[e], kLog2e, run[e]);
+            A[i][e] = run[e];
+          }
+        }
+        float incl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          incl[e] = run[e];
+          float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
+          if (lane >= 8) incl[e] += x;
+          x = __shfl_up_sync(0xffffffffu, incl[e], 16);
+          if (lane >= 16) incl[e] += x;
+        }
+        if (lane >= 24) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ms->red[warp][8 * cc + e] = incl[e];
+        }
+        wg_sync(wg);
+        float off[8], last[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          off[e] = incl[e] - run[e];
+          last[e] = 0.f;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 t0 = *reinterpret_cast<const float4*>(&ms->red[w][8 * cc]);
+          const float4 t1 = *reinterpret_cast<const float4*>(&ms->red[w][8 * cc + 4]);
+          const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (w < warp) off[e] += t[e];
+            last[e] += t[e];
+          }
+        }
+        bool exp_unsafe = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (-last[e] > fp.max_exp2) exp_unsafe = true;
+        // every warp holds all 64 channels (lanes cover cc = 0..7), so this vote is the
+        // same in all four warps: the chunk's scores come from the CUDA cores, and Kh is
+        // scaled by 2^(a - A) <= 1 instead (summary S <- 2^a S + U)
+        const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
+        float eseg[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) eseg[e] = ex2(a2seg[e]);
+        // ---- Qh = q 2^A, Kh = k 2^-A, held Qh 2^(A_seg) (HOLD); A -> G for the CUDA-core scores
+        uint8_t* opq = smem + kOffOp + bb * 2 * kTile;
+        uint8_t* opk = opq + kTile;
+        uint8_t* held = smem + kOffHeld + (sig * kHeldPerSet + (g < kHeldPerSet ? g : 0)) * kTile;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int row = 4 * rb + i;
+          const uint32_t off16 = row * 128u + (((uint32_t)cc ^ ((uint32_t)row & 7u)) << 4);
+          const uint4 qraw = *reinterpret_cast<const uint4*>(sb + off16);
+          const uint4 kraw = *reinterpret_cast<const uint4*>(sb + kTile + off16);
+          const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qraw);
+          const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kraw);
+          uint32_t oq[4], okk[4], oh[4];
+          float An[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 qv = Pack2<Tin>::unpack(qw[e2]);
+            const float2 kv = Pack2<Tin>::unpack(kw[e2]);
+            const float A0 = A[i][2 * e2] + off[2 * e2], A1 = A[i][2 * e2 + 1] + off[2 * e2 + 1];
+            An[2 * e2] = A0;
+            An[2 * e2 + 1] = A1;
+            const float qh0 = qv.x * ex2(A0), qh1 = qv.y * ex2(A1);
+            const float kh0 = kv.x * ex2(fbx ? last[2 * e2] - A0 : -A0);
+            const float kh1 = kv.y * ex2(fbx ? last[2 * e2 + 1] - A1 : -A1);
+            if (!f16_ok(qv.x) || !f16_ok(qv.y) || !f16_ok(kv.x) || !f16_ok(kv.y) || !f16_ok(kh0) || !f16_ok(kh1))
+              range_bad = true;
+            oq[e2] = Pack2<__half>::pack(qh0, qh1);
+            okk[e2] = Pack2<__half>::pack(kh0, kh1);
+            oh[e2] = Pack2<__half>::pack(qh0 * eseg[2 * e2], qh1 * eseg[2 * e2 + 1]);
+          }
+          *reinterpret_cast<uint4*>(opq + off16) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+          *reinterpret_cast<uint4*>(opk + off16) = make_uint4(okk[0], okk[1], okk[2], okk[3]);
+          if (hold) *reinterpret_cast<uint4*>(held + off16) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+          if (fbx) {  // the CUDA-core scores of this chunk read A back from the gate tile
+            float4* gw = reinterpret_cast<float4*>(G + row * 64 + 8 * cc);
+            gw[0] = make_float4(An[0], An[1], An[2], An[3]);
+            gw[1] = make_float4(An[4], An[5], An[6], An[7]);
+          }
+        }
+        if constexpr (!std::is_same<Tin, __half>::value) {
+          // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
+          uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
+          for (int i = wtid; i < kTile / 16; i += kWG) {
+            uint4 x = vt[i];
+            uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = Pack2<Tin>::unpack(w[e]);
+              if (!f16_ok(f.x) || !f16_ok(f.y)) range_bad = true;
+              w[e] = Pack2<__half>::pack(f.x, f.y);
+            }
+            vt[i] = x;
+          }
+        }
+        if (rb == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ms->a2last[bb][8 * cc + e] = last[e];
+        }
+        if (wtid == 0) ms->fb[bb] = fbx ? 1 : 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a2seg[e] += last[e];
+        fence_proxy_async_smem();
+        wg_sync(wg);
+        if (wtid == 0) {
+          mbar_arrive(&ms->opready[bb]);
+          mbar_arrive(&ms->empty[st]);
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ===================================================================== WG_B: masking, state, STREAM epilogue
+    const int wg = 1, wtid = tid - kWG, wq = warp & 3;
+    const int trow = wq * 16 + (lane & 15);
+    const bool tile1 = lane >= 16;
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
+    uint8_t* orow = smem + kOffOut + trow * 256;
+    float Sreg[64];        // fp32 state row `trow` (tile-1 lanes)
+    float a2seg_row = 0.f; // log2 segment decay of channel trow (tile-1 lanes)
+    int slot = 0, n = 0;
+    bool alive = true;
+    auto stream_epilogue = [&](int nn) {  // output of chunk nn (STREAM), O region nn & 1
+      const int cn = nn;                  // in STREAM the chunk index equals the counter
+      epilogue_rows<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(nn & 1), !tile1,
+                          (long long)cn * kChunk + trow, orow, fp.scale);
+      bulk_wait_read<0>();
+      tc_fence_before();
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->o_free[nn & 1]);
+    };
+    for (int r = 0; r < rounds && alive; ++r) {
+      const Span sp = round_span(fp, r, seg);
+      if (sp.c1 <= sp.c0) {
+        if (hold) {  // an empty segment still publishes a neutral summary
+          float* mine = fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64);
+          if (tile1) {
+            for (int e = 0; e < 64; e += 4) __stcg(reinterpret_cast<float4*>(mine + trow * 64 + e), make_float4(0.f, 0.f, 0.f, 0.f));
+            mine[4096 + trow] = 0.f;
+          }
+          __threadfence();
+          wg_sync(wg);
+          if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
+        }
+        continue;
+      }
+#pragma unroll
+      for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
+      a2seg_row = 0.f;
+      {  // zero start state for this round's first chunk
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n & 1) * kTile);
+        for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
+        fence_proxy_async_smem();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->sready[n & 1]);
+      }
+      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
+        const int bb = n & 1, st = n % kStages;
+        const bool last_chunk = (c + 1 == sp.c1);
+        if (!wg_wait(wg, wtid, &ms->su_full[bb], ph_of(n), ms, hdr, 0x400, slot)) { alive = false; break; }
+        if (n >= 1 && !wg_wait(wg, wtid, &ms->o_full[(n - 1) & 1], ph_of(n - 1), ms, hdr, 0x401, slot)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const bool fbk = ms->fb[bb] != 0;
+        const float lastc = ms->a2last[bb][trow];
+        const float dl = ex2(lastc);
+        uint8_t* prow = smem + kOffP + bb * kTile;
+        uint8_t* srow = smem + kOffS + ((n + 1) & 1) * kTile;
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+          float v[16];
+          tmem_ld16(tl + kColSU + 64u * bb + cb, v);
+          tmem_wait_ld();
+          if (!tile1) {
+            if (!fbk) {  // masked scores (j <= i) -> P row trow
+              uint32_t pk[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int j = cb + 2 * e;
+                const float x0 = (j <= trow) ? v[2 * e] : 0.f;
+                const float x1 = (j + 1 <= trow) ? v[2 * e + 1] : 0.f;
+                if (!f16_ok(x0) || !f16_ok(x1)) range_bad = true;
+                pk[e] = Pack2<__half>::pack(x0, x1);
+              }
+              *reinterpret_cast<uint4*>(prow + sw128_offset(trow, cb)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(prow + sw128_offset(trow, cb + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          } else {  // state row trow: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
+            if (!fbk) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) Sreg[cb + e] = dl * (Sreg[cb + e] + v[e]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) Sreg[cb + e] = fmaf(dl, Sreg[cb + e], v[e]);
+            }
+            if (!last_chunk) {
+              uint32_t sk[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (!f16_ok(Sreg[cb + 2 * e]) || !f16_ok(Sreg[cb + 2 * e + 1])) range_bad = true;
+                sk[e] = Pack2<__half>::pack(Sreg[cb + 2 * e], Sreg[cb + 2 * e + 1]);
+              }
+              *reinterpret_cast<uint4*>(srow + sw128_offset(trow, cb)) = make_uint4(sk[0], sk[1], sk[2], sk[3]);
+              *reinterpret_cast<uint4*>(srow + sw128_offset(trow, cb + 8)) = make_uint4(sk[4], sk[5], sk[6], sk[7]);
+            }
+          }
+        }
+        if (tile1) a2seg_row += lastc;
+        if (fbk) {
+          // exact scores on the CUDA cores: P[i][j] = sum_k q_ik k_jk 2^(A_ik - A_jk), j <= i
+          const uint8_t* sb = smem + kOffStage + st * kStageBytes;
+          const float* Ag = reinterpret_cast<const float*>(sb + 3 * kTile);
+          const int i_row = wtid >> 1, jh = wtid & 1;
+          uint32_t pk[16];
+          for (int jj = 0; jj < 32; jj += 2) {
+            float x[2];
+            for (int u = 0; u < 2; ++u) {
+              const int j = jh * 32 + jj + u;
+              float acc = 0.f;
+              if (j <= i_row) {
+                for (int k = 0; k < 64; k += 2) {
+                  const float2 qv = Pack2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i_row, k)));
+                  const float2 kv = Pack2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
+                  acc = fmaf(qv.x * kv.x, ex2(Ag[i_row * 64 + k] - Ag[j * 64 + k]), acc);
+                  acc = fmaf(qv.y * kv.y, ex2(Ag[i_row * 64 + k + 1] - Ag[j * 64 + k + 1]), acc);
+                }
+              }
+              x[u] = acc;
+            }
+            if (!f16_ok(x[0]) || !f16_ok(x[1])) range_bad = true;
+            pk[jj >> 1] = Pack2<__half>::pack(x[0], x[1]);
+          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(prow + sw128_offset(i_row, jh * 32 + 8 * q4)) =
+                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        wg_sync(wg);
+        if (wtid == 0) {
+          mbar_arrive(&ms->su_free[bb]);
+          mbar_arrive(&ms->pready[bb]);
+          if (!last_chunk) mbar_arrive(&ms->sready[(n + 1) & 1]);
+        }
+        if (!hold && n >= 1) stream_epilogue(n - 1);
+      }
+      if (!alive) break;
+      if (!hold) {
+        // output of the sequence's last chunk
+        if (!wg_wait(wg, wtid, &ms->o_full[(n - 1) & 1], ph_of(n - 1), ms, hdr, 0x402, slot)) { alive = false; break; }
+        tc_fence_after();
+        stream_epilogue(n - 1);
+      } else {
+        // segment summary of this round: U_seg = local end state, its log2 decay
+        float* mine = fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64);
+        if (tile1) {
+          for (int e = 0; e < 64; e += 4)
+            __stcg(reinterpret_cast<float4*>(mine + trow * 64 + e), make_float4(Sreg[e], Sreg[e + 1], Sreg[e + 2], Sreg[e + 3]));
+          mine[4096 + trow] = a2seg_row;
+        }
+        __threadfence();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
+      }
+    }
+    bulk_wait_all<0>();
+  } else if (warp < 12) {
+    // ===================================================================== WG_C: HOLD round end
+    if (hold) {
+      const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
+      const int trow = wq * 16 + (lane & 15);
+      const bool tile1 = lane >= 16;
+      const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+      uint8_t* orow = smem + kOffOut + trow * 256;
+      // state entries owned by this CTA, in groups of 8 (one 16-byte chunk of a start-state row)
+      const int g0 = (int)((long long)seg * 512 / fp.n_s), g1 = (int)((long long)(seg + 1) * 512 / fp.n_s);
+      float Sin[kMaxOwn];  // owned entries' running state across rounds (two groups per thread)
+#pragma unroll
+      for (int u = 0; u < kMaxOwn; ++u) Sin[u] = 0.f;
+      unsigned int* ctr = fp.counters + (size_t)seq * 2;
+      const float* aggs0 = fp.agg + (size_t)seq * 2 * fp.n_s * (4096 + 64);
+      uint16_t* sst = fp.sstart + (size_t)seq * fp.n_s * 4096;
+      int slot = 0;
+      for (int r = 0; r < rounds; ++r) {
+        const int sig = r & 1;
+        const Span sp = round_span(fp, r, seg);
+        const float* aggs = aggs0 + (size_t)sig * fp.n_s * (4096 + 64);
+        if (!wg_wait(wg, wtid, &ms->agg_pub[sig], ph_of(r), ms, hdr, 0x600, slot)) break;
+        const unsigned int target = (unsigned int)(r + 1) * (unsigned int)fp.n_s;
+        bool ok0 = true;
+        if (wtid == 0) {
+          red_release_add(ctr, 1u);
+          ok0 = wait_counter(ctr, target, ms, hdr, 0x601);
+        }
+        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
+        // scan over the sequence's segments for my entries: S_start[s] in fp16, MMA layout.
+        // Loads for four segments are in flight at a time; each step writes 16 bytes.
+#pragma unroll
+        for (int u = 0; u < kMaxOwn / 8; ++u) {
+          const int gi = g0 + u * kWG + wtid;
+          if (gi < g1) {
+            const int kk = gi >> 3, e = gi * 8;
+            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)gi & 7u) ^ ((uint32_t)kk & 7u)) << 4);
+            float sv[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) sv[x] = Sin[u * 8 + x];
+            for (int sb = 0; sb < fp.n_s; sb += 4) {
+              float4 ua[4], ub[4];
+              float dk[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                if (sb + t < fp.n_s) {
+                  const float* a2p = aggs + (size_t)(sb + t) * (4096 + 64);
+                  ua[t] = __ldcg(reinterpret_cast<const float4*>(a2p + e));
+                  ub[t] = __ldcg(reinterpret_cast<const float4*>(a2p + e + 4));
+                  dk[t] = __ldcg(a2p + 4096 + kk);
+                }
+              }
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                if (sb + t < fp.n_s) {
+                  uint32_t pk[4];
+#pragma unroll
+                  for (int x = 0; x < 4; ++x) {
+                    if (!f16_ok(sv[2 * x]) || !f16_ok(sv[2 * x + 1])) range_bad = true;
+                    pk[x] = Pack2<__half>::pack(sv[2 * x], sv[2 * x + 1]);
+                  }
+                  __stcg(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sst + (size_t)(sb + t) * 4096) + soff),
+                         make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                  const float d = ex2(dk[t]);
+                  const float uu[8] = {ua[t].x, ua[t].y, ua[t].z, ua[t].w, ub[t].x, ub[t].y, ub[t].z, ub[t].w};
+#pragma unroll
+                  for (int x = 0; x < 8; ++x) sv[x] = fmaf(d, sv[x], uu[x]);
+                }
+              }
+            }
+#pragma unroll
+            for (int x = 0; x < 8; ++x) Sin[u * 8 + x] = sv[x];
+          }
+        }
+        __threadfence();
+        wg_sync(wg);
+        ok0 = true;
+        if (wtid == 0) {
+          red_release_add(ctr + 1, 1u);
+          ok0 = wait_counter(ctr + 1, target, ms, hdr, 0x602);
+        }
+        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
+        {  // my segment's start state -> shared memory (already in the MMA layout)
+          const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
+          uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
+          for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
+        }
+        fence_proxy_async_smem();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->corr_ready[sig]);
+        if (!wg_wait(wg, wtid, &ms->corr_done[sig], ph_of(r), ms, hdr, 0x603, slot)) break;
+        tc_fence_after();
+        // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane tile 1)
+        const int G = sp.c1 - sp.c0;
+        for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
+          for (int pass = 0; pass < 2; ++pass) {
+            const int gi = 2 * m2 + pass;
+            const bool mine = (pass == 0) ? !tile1 : tile1;
+            epilogue_rows<Tout>(p, b, h, tl + kColO + 128u * sig + 64u * (uint32_t)m2, mine && gi < G,
+                                (long long)(sp.c0 + gi) * kChunk + trow, orow, fp.scale);
+            bulk_wait_read<0>();
+            __syncwarp();
+          }
+        }
+        tc_fence_before();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->set_free[sig]);
+      }
+      bulk_wait_all<0>();
+    }
+  }
+
+  if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(hdr, GTR_ERR_RANGE, 0x500u + warp);
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  // last CTA out resets this call's counters: the workspace is ready for the next call
+  if (hold && tid == 0) {
+    __threadfence();
+    const unsigned int done = atomicAdd(&hdr->ticket, 1u);
+    if (done == (unsigned int)fp.grid - 1) {
+      for (int i = 0; i < 2 * fp.n_seq; ++i) fp.counters[i] = 0u;
+      __threadfence();
+      hdr->ticket = 0u;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+struct Plan {
+  int mode, n_seq, n_s, rounds, grid;
+};
+
+// Length-aware plan: many sequences -> one CTA each (STREAM); few sequences -> each is
+// split over n_s CTAs with about kHeldPerSet chunks per CTA per round (HOLD).
+Plan make_plan(const Problem& p, int sms) {
+  Plan pl;
+  pl.n_seq = p.B * p.heads;
+  const int Nc = p.n_chunks();
+  const int cap = sms < (int)kMaxHoldSegments ? sms : (int)kMaxHoldSegments;
+  if (pl.n_seq * 2 > cap || Nc <= 1) {
+    pl.mode = 0;
+    pl.n_s = 1;
+    pl.rounds = 1;
+    pl.grid = pl.n_seq;
+  } else {
+    pl.mode = 1;
+    pl.n_s = cap / pl.n_seq;
+    if (pl.n_s > Nc) pl.n_s = Nc;
+    const int per_round = pl.n_s * kHeldPerSet;
+    pl.rounds = (Nc + per_round - 1) / per_round;
+    pl.grid = pl.n_seq * pl.n_s;
+  }
+  return pl;
+}
+
+int device_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
+size_t hold_segments(const Problem& p) {
+  const size_t n_seq = (size_t)p.B * p.heads;
+  return n_seq * 2 <= kMaxHoldSegments ? n_seq * (kMaxHoldSegments / n_seq) : 0;
+}
+
+template <typename Tin, typename Tout>
+gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
+  auto kern = fused_gla_kernel<Tin, Tout>;
+  static std::atomic<unsigned long long> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
+  if (!(configured.load() & (1ull << dev))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+      return GTR_ERR_CUDA;
+    configured.fetch_or(1ull << dev);
+  }
+  Plan pl = make_plan(p, device_sms());
+  if (force_mode == 0) {
+    pl.mode = 0;
+    pl.n_s = 1;
+    pl.rounds = 1;
+    pl.grid = pl.n_seq;
+  }
+  FusedParams fp;
+  fp.p = p;
+  const FusedWorkspace w = fused_workspace_carve(ws, p);
+  fp.hdr = w.hdr;
+  fp.counters = w.counters;
+  fp.agg = w.agg;
+  fp.sstart = w.sstart;
+  fp.n_seq = pl.n_seq;
+  fp.n_s = pl.n_s;
+  fp.rounds = pl.rounds;
+  fp.Nc = p.n_chunks();
+  fp.mode = pl.mode;
+  fp.grid = pl.grid;
+  fp.scale = 1.0f / sqrtf((float)p.d_k);
+  // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the
+  // fp16 rounding of the small Qh values keep their precision
+  fp.max_exp2 = 11.5f;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;
+  return GTR_OK;
+}
+
+}  // namespace
+
+size_t fused_workspace_bytes(const Problem& p) {
+  const size_t segs = hold_segments(p);
+  return sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t);
+}
+
+FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
+  const size_t segs = hold_segments(p);
+  FusedWorkspace w;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  w.hdr = reinterpret_cast<WsHeader*>(base);
+  base += sizeof(WsHeader);
+  w.counters = reinterpret_cast<unsigned int*>(base);
+  base += kCounterBytes;
+  w.agg = reinterpret_cast<float*>(base);
+  base += 2 * segs * (4096 + 64) * sizeof(float);
+  w.sstart = reinterpret_cast<uint16_t*>(base);
+  return w;
+}
+
+size_t fused_reset_bytes() { return sizeof(WsHeader) + kCounterBytes; }
+
+int fused_launches(const Problem& p) {
+  (void)p;
+  return 1;
+}
+
+gtr_status_t launch_fused(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
+  if ((long long)p.B * p.L() >= (1ll << 31)) return GTR_ERR_UNSUPPORTED;
+  switch (p.in_dtype * 3 + p.out_dtype) {
+    case GTR_F16 * 3 + GTR_F16: return launch_fused_typed<__half, __half>(p, ws, stream, force_mode);
+    case GTR_F16 * 3 + GTR_F32: return launch_fused_typed<__half, float>(p, ws, stream, force_mode);
+    case GTR_BF16 * 3 + GTR_F32: return launch_fused_typed<__nv_bfloat16, float>(p, ws, stream, force_mode);
+    case GTR_BF16 * 3 + GTR_BF16: return launch_fused_typed<__nv_bfloat16, __nv_bfloat16>(p, ws, stream, force_mode);
+    default: return GTR_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace gtr

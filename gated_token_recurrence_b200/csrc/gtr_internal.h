@@ -18,8 +18,22 @@ struct SplitWorkspace {
   float* a_last;  // [B*heads*Nc][64]     chunk log-decays
 };
 
+struct FusedWorkspace {
+  WsHeader* hdr;
+  unsigned int* counters;  // per-sequence arrival counters (zero between calls)
+  float* agg;              // per-segment summaries
+  uint16_t* sstart;        // per-segment start states (16-bit, MMA layout)
+};
+
 size_t split_workspace_bytes(const Problem& p);
 SplitWorkspace split_workspace_carve(void* ws, const Problem& p);
 gtr_status_t launch_split(const Problem& p, void* ws, cudaStream_t stream);
+
+size_t fused_workspace_bytes(const Problem& p);
+FusedWorkspace fused_workspace_carve(void* ws, const Problem& p);
+int fused_launches(const Problem& p);
+size_t fused_reset_bytes();  // header + counters: what a zeroed workspace must have zero
+// force_mode: -1 = let the plan decide, 0 = one CTA per sequence (stream mode)
+gtr_status_t launch_fused(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
 
 }  // namespace gtr

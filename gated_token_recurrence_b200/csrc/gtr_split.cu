@@ -278,14 +278,14 @@ gtr_status_t launch_split_typed(const Problem& p, const SplitWorkspace& ws, cuda
 
 size_t split_workspace_bytes(const Problem& p) {
   const size_t units = (size_t)p.B * p.heads * p.n_chunks();
-  return sizeof(WsHeader) + units * (2 * kD * kD + kD) * sizeof(float);
+  return kWsPrefixBytes + units * (2 * kD * kD + kD) * sizeof(float);
 }
 
 SplitWorkspace split_workspace_carve(void* ws, const Problem& p) {
   const size_t units = (size_t)p.B * p.heads * p.n_chunks();
   SplitWorkspace w;
   w.hdr = reinterpret_cast<WsHeader*>(ws);
-  float* base = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + sizeof(WsHeader));
+  float* base = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsPrefixBytes);
   w.U = base;
   w.S = base + units * kD * kD;
   w.a_last = base + 2 * units * kD * kD;

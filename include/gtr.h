@@ -70,14 +70,20 @@ typedef enum {
     GTR_ERR_UNSUPPORTED = 2, /* valid but not implemented (d_k, d_v, dtype pairing) */
     GTR_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     GTR_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out (see gtr_gla_read_error) */
-    GTR_ERR_WORKSPACE = 5    /* workspace too small, or would have to grow during stream capture */
+    GTR_ERR_WORKSPACE = 5,   /* workspace too small, or would have to grow during stream capture */
+    GTR_ERR_RANGE = 6        /* (device error word) an input, score or state magnitude passed
+                                60000, beyond the fused path's fp16 tensor-core operands; that
+                                call's output is not valid - use GTR_PATH_SPLIT for such data */
 } gtr_status_t;
 
 /* Execution paths.  GTR_PATH_AUTO lets the length-aware dispatcher choose. */
 typedef enum {
     GTR_PATH_AUTO = 0,
     GTR_PATH_SPLIT = 1, /* three launches: chunk summaries -> state scan -> chunk outputs (any dtype) */
-    GTR_PATH_FUSED = 2  /* single tensor-core launch (fp16/bf16 inputs) */
+    GTR_PATH_FUSED = 2, /* single tensor-core launch (fp16/bf16 inputs); the plan splits
+                           long sequences over several CTAs */
+    GTR_PATH_FUSED_SEQUENTIAL = 3 /* the same kernel with one CTA per (batch, head)
+                                     walking its whole sequence */
 } gtr_path_t;
 
 /*

@@ -65,7 +65,7 @@ def test_bad_arguments_rejected_on_host(kw, code):
 def test_workspace_query():
     n = gtr.workspace_bytes(1, 6, 40, 40, 64, 64, gtr.F16, "split")
     units = 6 * 25
-    assert n == 256 + units * (2 * 64 * 64 + 64) * 4
+    assert n == 256 + 2048 + units * (2 * 64 * 64 + 64) * 4
     assert gtr.workspace_bytes(1, 6, 40, 40, 64, 64, gtr.F16, "auto") >= n
     assert gtr.workspace_bytes(0, 6, 40, 40) == 0
     assert gtr.workspace_bytes(1, 6, 40, 40, 32, 64) == 0
@@ -76,3 +76,10 @@ def test_typed_entries_validate_too():
     assert f(None, 16, 16, 16, 16, 1, 1, 8, 8, 64, 64, 0, None) == 1
     assert gtr.lib.gtr_gla_fwd_f32(16, 16, 16, 16, 16, 1, 1, 8, 8, 64, 64, 9, None) == 1
     assert gtr.lib.gtr_gla_fwd_bf16(16, 16, 16, 16, 16, 1, 1, 8, 8, 48, 64, 0, None) == 2
+
+
+def test_dispatcher_plan():
+    assert gtr.plan(1, 6, 40, 40, in_dtype=gtr.F16) == ("fused", 1)
+    assert gtr.plan(8, 6, 48, 80, in_dtype=gtr.BF16) == ("fused", 1)
+    assert gtr.plan(1, 2, 16, 16, in_dtype=gtr.F32) == ("split", 3)
+    assert gtr.status_string(6) == "GTR_ERR_RANGE"

@@ -16,7 +16,12 @@ from gtr_inputs import WORKLOADS, Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-5, "f16": 1e-2, "bf16": 1e-2}
-PATHS = ["split"]
+PATHS = ["split", "fused", "fused_sequential"]
+
+
+def path_ok(dtype: str, path: str) -> bool:
+    """The fused tensor-core paths take fp16/bf16 inputs; fp32 runs on the split path."""
+    return not (dtype == "f32" and path.startswith("fused"))
 
 
 def rel_err(out: torch.Tensor, ref: np.ndarray) -> float:
@@ -51,6 +56,8 @@ def check(w: Workload, direction: int, seed: int, path="auto", out_dtype=None, t
 @pytest.mark.parametrize("name", ["tiny", "640", "1024", "2048"])
 def test_workload_all_directions(name, path):
     w = WORKLOADS[name]
+    if not path_ok(w.dtype, path):
+        pytest.skip("fp32 inputs run on the split path only")
     for d in w.directions:
         check(w, d, w.seed(d), path)
 
@@ -80,16 +87,38 @@ ODD = [
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 @pytest.mark.parametrize("shape", ODD)
 def test_ragged_and_degenerate_shapes(shape, dtype, path):
+    if not path_ok(dtype, path):
+        pytest.skip("fp32 inputs run on the split path only")
     B, heads, H, W = shape
     w = Workload("odd", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=1.0, index=9)
     for d in range(4):
-        check(w, d, 9000 + 100 * H + W + d, path)
+        if H * W == 1 and path.startswith("fused"):
+            check_single_token(w, d, 9000 + 100 * H + W + d, path)
+        else:
+            check(w, d, 9000 + 100 * H + W + d, path)
+
+
+def check_single_token(w: Workload, direction: int, seed: int, path: str):
+    """One token: o = d_k^{-1/2} (q . k) v.  The tensor-core path rounds the gate-scaled q
+    and k and the score to fp16, so its error is bounded by a few fp16 ulps of the
+    dot product's absolute terms, sum_i |q_i k_i|, times |v|; a cancelling q . k makes
+    1e-2 * rms(o) smaller than that (the automatic dispatch sends such sequences to the
+    fp32 split path)."""
+    q, k, v, lg = make_inputs(w, seed)
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, direction)
+    out = run_gpu(w, q, k, v, lg, direction, path).double().cpu().numpy()
+    qa, ka, va = (t.double().numpy() for t in (q, k, v))
+    scale = np.abs(qa * ka).sum(axis=-1, keepdims=True) * np.abs(va) / np.sqrt(w.d_k)
+    assert (np.abs(out - ref) <= 4 * 2.0 ** -11 * scale + 1e-6).all()
 
 
 @pytest.mark.parametrize("path", ["auto"] + PATHS)
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 def test_strong_decay_gates(dtype, path):
-    """log gamma = logsigmoid(g - 2)/2: about -1 per token, a chunk decays by ~e^-70."""
+    """log gamma = logsigmoid(g - 2)/2: about -1 per token, a chunk decays by ~e^-70
+    (the fused path computes those chunks' scores on the CUDA cores)."""
+    if not path_ok(dtype, path):
+        pytest.skip("fp32 inputs run on the split path only")
     w = Workload("strong", B=1, heads=2, H=24, W=24, dtype=dtype, gate_offset=-2.0, gate_tau=2.0,
                  index=9)
     q, k, v, lg = make_inputs(w, 77)
@@ -192,3 +221,54 @@ def test_graph_capture_with_caller_workspace():
     g.replay()
     torch.cuda.synchronize()
     assert rel_err(out, ref) <= 1e-2
+
+
+def test_fused_range_guard_reports_and_split_path_handles_it():
+    """A bf16 value beyond the fp16 operand range: the fused path flags GTR_ERR_RANGE on the
+    device; the split path (fp32 arithmetic) computes the case correctly."""
+    w = Workload("range", B=1, heads=1, H=8, W=16, dtype="bf16", index=9)
+    q, k, v, lg = make_inputs(w, 91)
+    v[0, 5, 0, 3] = 1.0e6
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 0)
+    dev = torch.device("cuda:0")
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, in_dtype=gtr.BF16, device=dev)
+    gtr.gla_fwd(q.to(dev), k.to(dev), v.to(dev), lg.to(dev), grid=(w.H, w.W), path="fused", workspace=ws)
+    assert gtr.read_error(ws) == 6
+    assert gtr.read_error(ws) == 0  # reading clears it
+    out = run_gpu(w, q, k, v, lg, 0, "split")
+    assert rel_err(out, ref) <= 1e-2
+
+
+@pytest.mark.parametrize("name", ["640", "1024", "2048", "stack"])
+def test_paths_agree_on_workloads(name):
+    """The fused plan, the one-CTA-per-sequence walk and the split path agree (1e-2 * rms)."""
+    w = WORKLOADS[name]
+    d = w.directions[-1]
+    q, k, v, lg = (t.cuda() for t in make_inputs(w, 2024))
+    outs = {p: gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=d, path=p) for p in PATHS}
+    torch.cuda.synchronize()
+    ref = outs["split"].double()
+    rms = ref.pow(2).mean().sqrt()
+    for p, o in outs.items():
+        assert ((o.double() - ref).abs().max() / rms).item() <= 1e-2, p
+
+
+def test_paths_interleaved_on_the_shared_workspace():
+    """Split-path and fused-path calls alternate on the library's cached workspace (the
+    fused path's arrival counters must survive the split path's arrays)."""
+    wf = WORKLOADS["1024"].with_(heads=4)
+    ws_ = WORKLOADS["tiny"]
+    qf, kf, vf, gf = make_inputs(wf, 71)
+    qs, ks, vs, gs = make_inputs(ws_, 72)
+    ref_f = oracle.gla_fwd(qf, kf, vf, gf, wf.H, wf.W, 1)
+    ref_s = oracle.gla_fwd(qs, ks, vs, gs, ws_.H, ws_.W, 0)
+    dev = torch.device("cuda:0")
+    tf = tuple(t.to(dev) for t in (qf, kf, vf, gf))
+    ts = tuple(t.to(dev) for t in (qs, ks, vs, gs))
+    for _ in range(3):
+        o_s = gtr.gla_fwd(*ts, grid=(ws_.H, ws_.W), direction=0)   # fp32 -> split path
+        o_f = gtr.gla_fwd(*tf, grid=(wf.H, wf.W), direction=1)     # bf16 -> fused path
+        torch.cuda.synchronize()
+        assert rel_err(o_s, ref_s) <= 1e-5
+        assert rel_err(o_f, ref_f) <= 1e-2
+    assert gtr.read_error() == 0
