@@ -7,15 +7,18 @@
 //
 // Per chunk of C = 64 scan positions of one (batch, head), with A the in-chunk
 // inclusive cumsum of log2-gates and a = A[last] (per key channel):
-//   Qh = Q * 2^A   (<= |q|)     Kh = K * 2^-A   (>= |k|, bounded by the chunk's decay)
-//   P  = mask_{j<=i}(Qh Kh^T)   = sum_k q_ik k_jk 2^(A_ik - A_jk)
-//   O  = Qh S + P V             (S = state at the chunk start)
+//   Qh = Q * 2^A   (<= |q|)     Kh = K * 2^-A / sqrt(d_k)   (bounded by the chunk's decay)
+//   P  = mask_{j<=i}(Qh Kh^T)   = d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk)
+//   O  = Qh S + P V             (S = state at the chunk start, kept scaled by d_k^-1/2)
 //   U' = Kh^T V,  S <- 2^a * (S + U')     (= Diag(d) S + K~^T V with K~ = K * 2^(a - A))
-// All MMA operands are fp16 (bf16 inputs convert exactly inside the fp16 range);
-// accumulation and the state are fp32.  A chunk whose gates decay too fast for
-// the factorisation to stay inside fp16 gets its scores from the CUDA cores
-// (2^(A_i - A_j) per pair).  Values beyond the fp16 operand range are reported
-// as GTR_ERR_RANGE.
+// The power-of-two factor d_k^-1/2 = 1/8 rides on Kh, so every product below
+// already carries it and the outputs leave tensor memory final.  All MMA operands
+// are fp16 (bf16 inputs convert exactly inside the fp16 range); accumulation and
+// the state are fp32.  Qh and Kh overwrite the Q and K tiles they are built from.
+// A chunk whose gates decay too fast for the factorisation to stay inside fp16
+// gets its scores from the CUDA cores (2^(A_i - A_j) per pair), written straight
+// into tensor memory.  Outputs that come out non-finite (an operand beyond the
+// fp16 range) are reported as GTR_ERR_RANGE.
 //
 // Two modes.  STREAM: one CTA walks a whole sequence, carrying the exact fp32
 // state.  HOLD: the n_s CTAs of a sequence each take a segment of every round;
@@ -26,9 +29,10 @@
 // epilogue overlap round r+1's chunks (two held sets).
 //
 // Warp roles (480 threads):
-//   warps 0-3   WG_A  load-side math: cumulative gates, Qh / Kh tiles, held tiles
-//   warps 4-7   WG_B  score masking, fp32 state update, STREAM epilogue
-//   warps 8-11  WG_C  HOLD round end: summary scan, correction, epilogue
+//   warps 0-3   WG_A  cumulative gates, Qh / Kh in place, held tiles, CUDA-core scores
+//   warps 4-7   WG_B  score masking and fp32 state update (16-lane tensor-memory loads,
+//               so every lane of a warp does the same work)
+//   warps 8-11  WG_C  epilogue (both modes); HOLD round end: summary scan, correction
 //   warps 12-13 producer: cp.async of one token row per thread (direction remap,
 //               128-byte-swizzled placement, zero fill past the sequence end)
 //   warp 14     tcgen05 MMA issuer and tensor-memory owner
@@ -45,35 +49,35 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 2;          // TMA staging depth (chunks in flight)
-constexpr int kHeldPerSet = 3;      // chunks held per CTA per round (HOLD)
+constexpr int kStages = 3;          // staging depth (chunks in flight)
+constexpr int kHeldPerSet = 4;      // chunks held per CTA per round (HOLD)
 constexpr int kThreads = 480;
 constexpr int kProducerThreads = 64;
 constexpr int kMmaWarp = 14;
 constexpr int kWG = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kF16Safe = 60000.f;  // largest magnitude an fp16 operand may carry
 
 // shared memory (bytes); every 16-bit tile is [64][64], 128 B rows, 128 B swizzle
 constexpr int kTile = 8192;
 constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
-constexpr int kStageBytes = 3 * kTile + kGTile;      // Q, K, V, G
+constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V, G
 constexpr int kOffStage = 0;
-constexpr int kOffOp = kOffStage + kStages * kStageBytes;  // [2] x (Qh, Kh)
-constexpr int kOffP = kOffOp + 2 * 2 * kTile;              // [2]
-constexpr int kOffS = kOffP + 2 * kTile;                   // [2]
+constexpr int kOffP = kOffStage + kStages * kStageBytes;   // masked scores
+constexpr int kOffS = kOffP + kTile;                       // [2] chunk-start states
 constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
 constexpr int kOffHeld = kOffSst + kTile;                  // [2 sets][kHeldPerSet]
-constexpr int kOffOut = kOffHeld + 2 * kHeldPerSet * kTile;  // 64 rows x 256 B staging
-constexpr int kOffMisc = kOffOut + 16384;
+constexpr int kOffMisc = kOffHeld + 2 * kHeldPerSet * kTile;
 constexpr int kMiscBytes = 3072;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 
 // tensor memory columns
 constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0) and U' (lane tile 1)
-constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 outputs; HOLD: [2 sets] x 128 held outputs
+constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 output pairs; HOLD: [2 sets] x kSetCols
 constexpr uint32_t kLaneTile1 = 16u << 16;
+constexpr uint32_t kSetCols = 64u * (kHeldPerSet / 2);
+static_assert(kHeldPerSet % 2 == 0, "held chunks come in lane-tile pairs");
+static_assert(kColO + 2 * kSetCols <= kTmemCols, "tensor memory budget");
 
 // HOLD-mode counters sit at a fixed place right after the workspace header, whatever
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
@@ -90,21 +94,21 @@ struct FusedParams {
   uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
   int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD
   int grid;
-  float scale;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
 };
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
-  uint64_t opready[2], opfree[2], su_full[2], su_free[2], sready[2], pready[2], o_full[2], o_free[2];
+  uint64_t opready[2], su_full[2], su_free[2], sready[2], pready, pv_done;
+  uint64_t o_full[2], o_free[2];
   uint64_t agg_pub[2], corr_ready[2], corr_done[2], set_free[2];
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
   int go[3][2];          // per-warpgroup wait decisions, alternating slots
-  int fb[2];             // chunk parity -> scores from the CUDA cores
-  alignas(16) float red[4][64];  // WG_A cumsum: per-warp channel totals
-  float a2last[2][64];   // chunk parity -> in-chunk log2 decay per channel
+  int fb[kStages];       // stage -> scores from the CUDA cores
+  alignas(16) float red[4][64];   // WG_A cumsum: per-warp channel totals
+  float a2last[kStages][64];      // stage -> in-chunk log2 decay per channel
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -152,7 +156,7 @@ __device__ bool wait_counter(const unsigned int* ctr, unsigned int target, Misc*
       *(volatile int*)&ms->abort = 1;
       return false;
     }
-    __nanosleep(128);
+    __nanosleep(64);
   }
 }
 
@@ -187,71 +191,79 @@ __device__ bool wg_agree(int wg, int wtid, bool ok0, Misc* ms, int& slot) {
   return go;
 }
 
-template <typename T> struct Pack2;
-template <> struct Pack2<__half> {
-  static __device__ __forceinline__ uint32_t pack(float a, float b) {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-  static __device__ __forceinline__ float2 unpack(uint32_t u) {
-    return __half22float2(*reinterpret_cast<__half2*>(&u));
-  }
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) { return h2_bits(__floats2half2_rn(a, b)); }
+
+// Two 16-bit input values -> fp32.
+template <typename T> struct In2;
+template <> struct In2<__half> {
+  static __device__ __forceinline__ float2 unpack(uint32_t u) { return __half22float2(bits_h2(u)); }
 };
-template <> struct Pack2<__nv_bfloat16> {
-  static __device__ __forceinline__ uint32_t pack(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
+template <> struct In2<__nv_bfloat16> {
   static __device__ __forceinline__ float2 unpack(uint32_t u) {
-    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
   }
 };
 
-__device__ __forceinline__ bool f16_ok(float x) { return fabsf(x) <= kF16Safe; }
+__device__ __forceinline__ void sts32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
 
-// Scale 16 output values (columns cb..cb+15 of one row) and stage them, in the
-// output dtype, in a linear shared-memory row for a bulk store.
+// Half an output row (32 values of a token-head starting at column col0, in registers)
+// -> its grid cell.  `nf` collects x * 0 over the stored values: it turns NaN once any
+// of them is not finite.
 template <typename Tout>
-__device__ __forceinline__ void stage_out16(uint8_t* orow, int cb, float* v, float scale) {
-#pragma unroll
-  for (int e = 0; e < 16; ++e) v[e] *= scale;
+__device__ __forceinline__ void store_out_half(const Problem& p, int b, int h, long long s, int col0,
+                                               const float* v, float& nf) {
+  const long long m = scan_to_token(s, p.direction, p.H, p.W);
+  Tout* dst = reinterpret_cast<Tout*>(p.out) + (((long long)b * p.L() + m) * p.heads + h) * 64 + col0;
   if constexpr (sizeof(Tout) == 4) {
 #pragma unroll
-    for (int e = 0; e < 16; e += 4)
-      *reinterpret_cast<float4*>(orow + (cb + e) * 4) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+    for (int e = 0; e < 32; e += 4) {
+      nf = fmaf(v[e], 0.f, nf);
+      nf = fmaf(v[e + 1], 0.f, nf);
+      nf = fmaf(v[e + 2], 0.f, nf);
+      nf = fmaf(v[e + 3], 0.f, nf);
+      __stcs(reinterpret_cast<float4*>(dst + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
+    }
   } else {
-    uint32_t pk[8];
+    __half2 acc = __float2half2_rn(0.f);
+    const __half2 zero = __float2half2_rn(0.f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) pk[e] = Pack2<Tout>::pack(v[2 * e], v[2 * e + 1]);
-    *reinterpret_cast<uint4*>(orow + cb * 2) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<uint4*>(orow + cb * 2 + 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    for (int e = 0; e < 32; e += 8) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if constexpr (std::is_same<Tout, __half>::value) {
+          pk[u] = pack_h2(v[e + 2 * u], v[e + 2 * u + 1]);
+          acc = __hfma2(bits_h2(pk[u]), zero, acc);
+        } else {
+          __nv_bfloat162 hb = __floats2bfloat162_rn(v[e + 2 * u], v[e + 2 * u + 1]);
+          pk[u] = *reinterpret_cast<uint32_t*>(&hb);
+          nf = fmaf(v[e + 2 * u], 0.f, nf);
+          nf = fmaf(v[e + 2 * u + 1], 0.f, nf);
+        }
+      }
+      __stcs(reinterpret_cast<uint4*>(dst + e), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+    }
+    if constexpr (std::is_same<Tout, __half>::value) {
+      const float2 a = __half22float2(acc);
+      nf += a.x + a.y;
+    }
   }
 }
 
-// Store one staged 64-value output row (a token-head) at its grid cell.
+// One output row of a lane-tile pair region in tensor memory (this thread's lane),
+// 32 columns at a time, -> its grid cell when `valid`.
 template <typename Tout>
-__device__ __forceinline__ void store_row(const Problem& p, int b, int h, long long s, const uint8_t* orow) {
-  const long long L = p.L();
-  const long long m = scan_to_token(s, p.direction, p.H, p.W);
-  uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + (((long long)b * L + m) * p.heads + h) * 64 * sizeof(Tout);
-  fence_proxy_async_smem();
-  bulk_store(dst, orow, 64 * sizeof(Tout));
-  bulk_commit();
-}
-
-// TMEM row (lane tile 0 or 1 of this warp's lane quarter) of a 64-column region ->
-// scaled output row, stored.  All 32 lanes take part in the loads; `mine` lanes store.
-template <typename Tout>
-__device__ __forceinline__ void epilogue_rows(const Problem& p, int b, int h, uint32_t taddr, bool mine,
-                                              long long s_row, uint8_t* orow, float scale) {
+__device__ __forceinline__ void epilogue_row(const Problem& p, int b, int h, uint32_t taddr, bool valid,
+                                             long long s, float& nf) {
 #pragma unroll
-  for (int cb = 0; cb < 64; cb += 16) {
-    float v[16];
-    tmem_ld16(taddr + cb, v);
+  for (int half = 0; half < 2; ++half) {
+    float v[32];
+    tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
-    if (mine) stage_out16<Tout>(orow, cb, v, scale);
+    if (valid) store_out_half<Tout>(p, b, h, s, 32 * half, v, nf);
   }
-  if (mine && s_row < p.L()) store_row<Tout>(p, b, h, s_row, orow);
 }
 
 struct Span {
@@ -291,20 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
   const int rounds = hold ? fp.rounds : 1;
-  bool range_bad = false;
+  float nonfinite = 0.f;
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&ms->full[i], kProducerThreads);
-      mbar_init(&ms->empty[i], 2);
+      mbar_init(&ms->empty[i], 1);
+      ms->fb[i] = 0;
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms->opready[i], 1);
-      mbar_init(&ms->opfree[i], 1);
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
       mbar_init(&ms->sready[i], 1);
-      mbar_init(&ms->pready[i], 1);
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
       mbar_init(&ms->agg_pub[i], 1);
@@ -312,15 +323,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->corr_done[i], 1);
       mbar_init(&ms->set_free[i], 1);
     }
+    mbar_init(&ms->pready, 1);
+    mbar_init(&ms->pv_done, 1);
     mbar_init(&ms->mma_final, 1);
     ms->abort = 0;
     for (int i = 0; i < 3; ++i) ms->go[i][0] = ms->go[i][1] = 0;
-    ms->fb[0] = ms->fb[1] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&ms->tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  if (warp >= 4 && warp < 8) {
+    // the masked-score tile: entries above the diagonal blocks stay zero for good
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4* pz = reinterpret_cast<uint4*>(smem + kOffP);
+    for (int i = tid - kWG; i < kTile / 16; i += kWG) pz[i] = z;
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -369,10 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_arrive_noinc(&ms->full[st]);
       }
     }
-    if (stop) {
-      // copies already issued must land before this CTA's shared memory is released
-      asm volatile("cp.async.wait_all;" ::: "memory");
-    }
+    // copies already issued must land before this CTA's shared memory is released
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ===================================================================== MMA issuer
     if (lane == 0) {
@@ -395,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Span spc = round_span(fp, rc, seg);
         const int G = spc.c1 - spc.c0;
         for (int g = 0; g < G; ++g) {
-          const uint32_t d_o = tmem + kColO + 128u * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+          const uint32_t d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
           const uint32_t a_h = s_base + kOffHeld + (sig * kHeldPerSet + g) * kTile;
           for (int k = 0; k < 4; ++k)
             mma_f16(d_o, sw128_desc(a_h + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
@@ -414,37 +431,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
           const int bb = n & 1, st = n % kStages;
-          const uint32_t op = s_base + kOffOp + bb * 2 * kTile;  // Qh, then Kh
-          const uint32_t a_v = s_base + kOffStage + st * kStageBytes + 2 * kTile;
+          const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
+          const uint32_t a_k = a_q + kTile;                            // Kh
+          const uint32_t a_v = a_q + 2 * kTile;
           if (!wait_bar(&ms->opready[bb], ph_of(n), ms, hdr, 0x200) ||
               !wait_bar(&ms->su_free[bb], ph_free(n), ms, hdr, 0x201)) { ok = false; break; }
           tc_fence_after();
           const uint32_t su = tmem + kColSU + 64u * bb;
-          for (int k = 0; k < 4; ++k)  // scores = Qh Kh^T
-            mma_f16(su, sw128_desc(op + 32 * k), sw128_desc(op + kTile + 32 * k), id_qk, k > 0);
+          if (!*(volatile int*)&ms->fb[st]) {
+            for (int k = 0; k < 4; ++k)  // scores = Qh Kh^T
+              mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
+          }
           for (int k = 0; k < 4; ++k)  // U' = Kh^T V
-            mma_f16(su + kLaneTile1, sw128_desc(op + kTile + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
+            mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
           mma_commit(&ms->su_full[bb]);
           uint32_t d_o;
           if (hold) {
-            d_o = tmem + kColO + 128u * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+            d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
           } else {
-            d_o = tmem + kColO + 64u * bb;
-            if (!wait_bar(&ms->o_free[bb], ph_free(n), ms, hdr, 0x202)) { ok = false; break; }
+            const int pr = n >> 1;  // output pair: chunks 2pr (lane tile 0) and 2pr+1 (lane tile 1)
+            d_o = tmem + kColO + 64u * (uint32_t)(pr & 1) + ((n & 1) ? kLaneTile1 : 0u);
+            if (!(n & 1) && !wait_bar(&ms->o_free[pr & 1], ph_free(pr), ms, hdr, 0x202)) { ok = false; break; }
           }
           if (!wait_bar(&ms->sready[bb], ph_of(n), ms, hdr, 0x203)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_s = s_base + kOffS + bb * kTile;
           for (int k = 0; k < 4; ++k)  // O = Qh S
-            mma_f16(d_o, sw128_desc(op + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-          if (!wait_bar(&ms->pready[bb], ph_of(n), ms, hdr, 0x204)) { ok = false; break; }
+            mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
+          if (!wait_bar(&ms->pready, (uint32_t)n & 1u, ms, hdr, 0x204)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_p = s_base + kOffP + bb * kTile;
+          const uint32_t a_p = s_base + kOffP;
           for (int k = 0; k < 4; ++k)  // O += P V
             mma_f16(d_o, sw128_desc(a_p + 32 * k), sw128_desc(a_v + 2048 * k), id_qs, 1);
-          mma_commit(&ms->o_full[bb]);
-          mma_commit(&ms->opfree[bb]);
+          mma_commit(&ms->pv_done);
           mma_commit(&ms->empty[st]);
+          if (!hold && ((n & 1) || c + 1 == sp.c1)) mma_commit(&ms->o_full[(n >> 1) & 1]);
           if (hold && next_corr < r && issue_corr(next_corr, false)) ++next_corr;
         }
       }
@@ -472,8 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           !wg_wait(wg, wtid, &ms->set_free[sig], ph_free(r), ms, hdr, 0x300, slot)) { alive = false; break; }
       for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
         const int bb = n & 1, st = n % kStages;
-        if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot) ||
-            !wg_wait(wg, wtid, &ms->opfree[bb], ph_free(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+        if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot)) {
+          alive = false;
+          break;
+        }
         uint8_t* sb = smem + kOffStage + st * kStageBytes;
         float* G = reinterpret_cast<float*>(sb + 3 * kTile);
         // ---- in-chunk cumulative log2-gates: my 4 rows, then a scan over the 16 row blocks
@@ -523,114 +546,141 @@ __global__ void __launch_bounds__(kThreads, 1)
             last[e] += t[e];
           }
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) A[i][e] += off[e];
         bool exp_unsafe = false;
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if (-last[e] > fp.max_exp2) exp_unsafe = true;
         // every warp holds all 64 channels (lanes cover cc = 0..7), so this vote is the
-        // same in all four warps: the chunk's scores come from the CUDA cores, and Kh is
-        // scaled by 2^(a - A) <= 1 instead (summary S <- 2^a S + U)
+        // same in all four warps
         const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
-        float eseg[8];
+        if (fbx) {
+          // ---- CUDA-core scores for this chunk, straight into tensor memory (lane tile 0
+          // of the chunk's score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk), j <= i.
+          // A goes to the gate tile so every thread can read every row.
 #pragma unroll
-        for (int e = 0; e < 8; ++e) eseg[e] = ex2(a2seg[e]);
-        // ---- Qh = q 2^A, Kh = k 2^-A, held Qh 2^(A_seg) (HOLD); A -> G for the CUDA-core scores
-        uint8_t* opq = smem + kOffOp + bb * 2 * kTile;
-        uint8_t* opk = opq + kTile;
+          for (int i = 0; i < 4; ++i) {
+            float4* gw = reinterpret_cast<float4*>(G + (4 * rb + i) * 64 + 8 * cc);
+            gw[0] = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
+            gw[1] = make_float4(A[i][4], A[i][5], A[i][6], A[i][7]);
+          }
+          if (!wg_wait(wg, wtid, &ms->su_free[bb], ph_free(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+          tc_fence_after();
+          const int r0 = 16 * warp + (lane >> 2), cq = 2 * (lane & 3);
+          float sv[32];
+          for (int x = 0; x < 32; ++x) {
+            const int i = r0 + 8 * ((x & 3) >> 1);
+            const int j = 8 * (x >> 2) + cq + (x & 1);
+            float acc = 0.f;
+            if (j <= i) {
+              for (int k = 0; k < 64; k += 2) {
+                const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
+                const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
+                acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
+                acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
+              }
+            }
+            sv[x] = acc * 0.125f;
+          }
+          tmem_st16x256_x8(tmem + ((uint32_t)(32 * warp) << 16) + kColSU + 64u * bb, sv);
+          tmem_wait_st();
+          tc_fence_before();
+          wg_sync(wg);  // every raw q / k read is done before the tiles are overwritten
+        }
+        // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place;
+        // held Qh 2^(A_seg) (HOLD)
+        __half2 eseg[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) eseg[e2] = bits_h2(pack_h2(ex2(a2seg[2 * e2]), ex2(a2seg[2 * e2 + 1])));
+        const __half2 eighth = __float2half2_rn(0.125f);
         uint8_t* held = smem + kOffHeld + (sig * kHeldPerSet + (g < kHeldPerSet ? g : 0)) * kTile;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = 4 * rb + i;
           const uint32_t off16 = row * 128u + (((uint32_t)cc ^ ((uint32_t)row & 7u)) << 4);
-          const uint4 qraw = *reinterpret_cast<const uint4*>(sb + off16);
-          const uint4 kraw = *reinterpret_cast<const uint4*>(sb + kTile + off16);
-          const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qraw);
-          const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kraw);
-          uint32_t oq[4], okk[4], oh[4];
-          float An[8];
+          uint4 qraw = *reinterpret_cast<const uint4*>(sb + off16);
+          uint4 kraw = *reinterpret_cast<const uint4*>(sb + kTile + off16);
+          uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
+          uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
+          uint32_t oh[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 qv = Pack2<Tin>::unpack(qw[e2]);
-            const float2 kv = Pack2<Tin>::unpack(kw[e2]);
-            const float A0 = A[i][2 * e2] + off[2 * e2], A1 = A[i][2 * e2 + 1] + off[2 * e2 + 1];
-            An[2 * e2] = A0;
-            An[2 * e2 + 1] = A1;
-            const float qh0 = qv.x * ex2(A0), qh1 = qv.y * ex2(A1);
-            const float kh0 = kv.x * ex2(fbx ? last[2 * e2] - A0 : -A0);
-            const float kh1 = kv.y * ex2(fbx ? last[2 * e2 + 1] - A1 : -A1);
-            if (!f16_ok(qv.x) || !f16_ok(qv.y) || !f16_ok(kv.x) || !f16_ok(kv.y) || !f16_ok(kh0) || !f16_ok(kh1))
-              range_bad = true;
-            oq[e2] = Pack2<__half>::pack(qh0, qh1);
-            okk[e2] = Pack2<__half>::pack(kh0, kh1);
-            oh[e2] = Pack2<__half>::pack(qh0 * eseg[2 * e2], qh1 * eseg[2 * e2 + 1]);
+            const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
+            const float xk0 = fbx ? last[2 * e2] - A0 : -A0;
+            const float xk1 = fbx ? last[2 * e2 + 1] - A1 : -A1;
+            __half2 qh, kh;
+            if constexpr (std::is_same<Tin, __half>::value) {
+              qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
+              kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
+            } else {
+              const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
+              qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
+              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+            }
+            qw[e2] = h2_bits(qh);
+            kw[e2] = h2_bits(kh);
+            oh[e2] = h2_bits(__hmul2(qh, eseg[e2]));
           }
-          *reinterpret_cast<uint4*>(opq + off16) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
-          *reinterpret_cast<uint4*>(opk + off16) = make_uint4(okk[0], okk[1], okk[2], okk[3]);
+          *reinterpret_cast<uint4*>(sb + off16) = qraw;
+          *reinterpret_cast<uint4*>(sb + kTile + off16) = kraw;
           if (hold) *reinterpret_cast<uint4*>(held + off16) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-          if (fbx) {  // the CUDA-core scores of this chunk read A back from the gate tile
-            float4* gw = reinterpret_cast<float4*>(G + row * 64 + 8 * cc);
-            gw[0] = make_float4(An[0], An[1], An[2], An[3]);
-            gw[1] = make_float4(An[4], An[5], An[6], An[7]);
-          }
         }
         if constexpr (!std::is_same<Tin, __half>::value) {
           // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
           uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
+#pragma unroll
           for (int i = wtid; i < kTile / 16; i += kWG) {
             uint4 x = vt[i];
             uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 f = Pack2<Tin>::unpack(w[e]);
-              if (!f16_ok(f.x) || !f16_ok(f.y)) range_bad = true;
-              w[e] = Pack2<__half>::pack(f.x, f.y);
+              const float2 f = In2<Tin>::unpack(w[e]);
+              w[e] = pack_h2(f.x, f.y);
             }
             vt[i] = x;
           }
         }
         if (rb == 0) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ms->a2last[bb][8 * cc + e] = last[e];
+          for (int e = 0; e < 8; ++e) ms->a2last[st][8 * cc + e] = last[e];
         }
-        if (wtid == 0) ms->fb[bb] = fbx ? 1 : 0;
+        if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) a2seg[e] += last[e];
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) {
-          mbar_arrive(&ms->opready[bb]);
-          mbar_arrive(&ms->empty[st]);
-        }
+        if (wtid == 0) mbar_arrive(&ms->opready[bb]);
       }
     }
   } else if (warp < 8) {
-    // ===================================================================== WG_B: masking, state, STREAM epilogue
+    // ===================================================================== WG_B: masking, state
+    // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
+    // r0 + 8(q>>1), column 8c + cq + (q&1) of the warp's 16-row slice.
     const int wg = 1, wtid = tid - kWG, wq = warp & 3;
-    const int trow = wq * 16 + (lane & 15);
-    const bool tile1 = lane >= 16;
+    const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
-    uint8_t* orow = smem + kOffOut + trow * 256;
-    float Sreg[64];        // fp32 state row `trow` (tile-1 lanes)
-    float a2seg_row = 0.f; // log2 segment decay of channel trow (tile-1 lanes)
+    uint8_t* prow0 = smem + kOffP + r0 * 128;
+    uint8_t* prow1 = smem + kOffP + r1 * 128;
+    float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
+    float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
     int slot = 0, n = 0;
     bool alive = true;
-    auto stream_epilogue = [&](int nn) {  // output of chunk nn (STREAM), O region nn & 1
-      const int cn = nn;                  // in STREAM the chunk index equals the counter
-      epilogue_rows<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(nn & 1), !tile1,
-                          (long long)cn * kChunk + trow, orow, fp.scale);
-      bulk_wait_read<0>();
-      tc_fence_before();
-      wg_sync(wg);
-      if (wtid == 0) mbar_arrive(&ms->o_free[nn & 1]);
-    };
     for (int r = 0; r < rounds && alive; ++r) {
       const Span sp = round_span(fp, r, seg);
+      float* mine = hold ? fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64) : nullptr;
       if (sp.c1 <= sp.c0) {
         if (hold) {  // an empty segment still publishes a neutral summary
-          float* mine = fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64);
-          if (tile1) {
-            for (int e = 0; e < 64; e += 4) __stcg(reinterpret_cast<float4*>(mine + trow * 64 + e), make_float4(0.f, 0.f, 0.f, 0.f));
-            mine[4096 + trow] = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * c + cq), make_float2(0.f, 0.f));
+            __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * c + cq), make_float2(0.f, 0.f));
+          }
+          if ((lane & 3) == 0) {
+            mine[4096 + r0] = 0.f;
+            mine[4096 + r1] = 0.f;
           }
           __threadfence();
           wg_sync(wg);
@@ -639,8 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 #pragma unroll
-      for (int e = 0; e < 64; ++e) Sreg[e] = 0.f;
-      a2seg_row = 0.f;
+      for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
+      a2r0 = a2r1 = 0.f;
       {  // zero start state for this round's first chunk
         const uint4 z = make_uint4(0, 0, 0, 0);
         uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n & 1) * kTile);
@@ -653,122 +703,100 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bb = n & 1, st = n % kStages;
         const bool last_chunk = (c + 1 == sp.c1);
         if (!wg_wait(wg, wtid, &ms->su_full[bb], ph_of(n), ms, hdr, 0x400, slot)) { alive = false; break; }
-        if (n >= 1 && !wg_wait(wg, wtid, &ms->o_full[(n - 1) & 1], ph_of(n - 1), ms, hdr, 0x401, slot)) {
+        // P and the next state tile are free once the previous chunk's P V has completed
+        if (n >= 1 && !wg_wait(wg, wtid, &ms->pv_done, (uint32_t)(n - 1) & 1u, ms, hdr, 0x401, slot)) {
           alive = false;
           break;
         }
         tc_fence_after();
-        const bool fbk = ms->fb[bb] != 0;
-        const float lastc = ms->a2last[bb][trow];
-        const float dl = ex2(lastc);
-        uint8_t* prow = smem + kOffP + bb * kTile;
-        uint8_t* srow = smem + kOffS + ((n + 1) & 1) * kTile;
+        const bool fbk = ms->fb[st] != 0;
+        const float l0 = ms->a2last[st][r0], l1 = ms->a2last[st][r1];
+        const float dl0 = ex2(l0), dl1 = ex2(l1);
+        float sc[32], u[32];
+        tmem_ld16x256_x8(tl + kColSU + 64u * bb, sc);
+        tmem_ld16x256_x8(tl + kColSU + 64u * bb + kLaneTile1, u);
+        tmem_wait_ld();
+        // masked scores -> P (blocks right of the warp's diagonal stay zero)
 #pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
-          float v[16];
-          tmem_ld16(tl + kColSU + 64u * bb + cb, v);
-          tmem_wait_ld();
-          if (!tile1) {
-            if (!fbk) {  // masked scores (j <= i) -> P row trow
-              uint32_t pk[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int j = cb + 2 * e;
-                const float x0 = (j <= trow) ? v[2 * e] : 0.f;
-                const float x1 = (j + 1 <= trow) ? v[2 * e + 1] : 0.f;
-                if (!f16_ok(x0) || !f16_ok(x1)) range_bad = true;
-                pk[e] = Pack2<__half>::pack(x0, x1);
-              }
-              *reinterpret_cast<uint4*>(prow + sw128_offset(trow, cb)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              *reinterpret_cast<uint4*>(prow + sw128_offset(trow, cb + 8)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int cb = 0; cb < 8; ++cb) {
+          if (cb <= 2 * wq + 1) {
+            float x0 = sc[4 * cb], x1 = sc[4 * cb + 1], x2 = sc[4 * cb + 2], x3 = sc[4 * cb + 3];
+            if (cb >= 2 * wq) {
+              const int j = 8 * cb + cq;
+              x0 = (j <= r0) ? x0 : 0.f;
+              x1 = (j + 1 <= r0) ? x1 : 0.f;
+              x2 = (j <= r1) ? x2 : 0.f;
+              x3 = (j + 1 <= r1) ? x3 : 0.f;
             }
-          } else {  // state row trow: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
-            if (!fbk) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) Sreg[cb + e] = dl * (Sreg[cb + e] + v[e]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) Sreg[cb + e] = fmaf(dl, Sreg[cb + e], v[e]);
-            }
-            if (!last_chunk) {
-              uint32_t sk[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (!f16_ok(Sreg[cb + 2 * e]) || !f16_ok(Sreg[cb + 2 * e + 1])) range_bad = true;
-                sk[e] = Pack2<__half>::pack(Sreg[cb + 2 * e], Sreg[cb + 2 * e + 1]);
-              }
-              *reinterpret_cast<uint4*>(srow + sw128_offset(trow, cb)) = make_uint4(sk[0], sk[1], sk[2], sk[3]);
-              *reinterpret_cast<uint4*>(srow + sw128_offset(trow, cb + 8)) = make_uint4(sk[4], sk[5], sk[6], sk[7]);
-            }
+            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
+            sts32(prow0 + o, pack_h2(x0, x1));
+            sts32(prow1 + o, pack_h2(x2, x3));
           }
         }
-        if (tile1) a2seg_row += lastc;
-        if (fbk) {
-          // exact scores on the CUDA cores: P[i][j] = sum_k q_ik k_jk 2^(A_ik - A_jk), j <= i
-          const uint8_t* sb = smem + kOffStage + st * kStageBytes;
-          const float* Ag = reinterpret_cast<const float*>(sb + 3 * kTile);
-          const int i_row = wtid >> 1, jh = wtid & 1;
-          uint32_t pk[16];
-          for (int jj = 0; jj < 32; jj += 2) {
-            float x[2];
-            for (int u = 0; u < 2; ++u) {
-              const int j = jh * 32 + jj + u;
-              float acc = 0.f;
-              if (j <= i_row) {
-                for (int k = 0; k < 64; k += 2) {
-                  const float2 qv = Pack2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i_row, k)));
-                  const float2 kv = Pack2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
-                  acc = fmaf(qv.x * kv.x, ex2(Ag[i_row * 64 + k] - Ag[j * 64 + k]), acc);
-                  acc = fmaf(qv.y * kv.y, ex2(Ag[i_row * 64 + k + 1] - Ag[j * 64 + k + 1]), acc);
-                }
-              }
-              x[u] = acc;
-            }
-            if (!f16_ok(x[0]) || !f16_ok(x[1])) range_bad = true;
-            pk[jj >> 1] = Pack2<__half>::pack(x[0], x[1]);
-          }
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(prow + sw128_offset(i_row, jh * 32 + 8 * q4)) =
-                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float d = (x & 2) ? dl1 : dl0;
+          Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
         }
+        if (!last_chunk) {
+          uint8_t* srow0 = smem + kOffS + ((n + 1) & 1) * kTile + r0 * 128;
+          uint8_t* srow1 = srow0 + 8 * 128;
+#pragma unroll
+          for (int cb = 0; cb < 8; ++cb) {
+            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;
+            sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
+            sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+          }
+        }
+        a2r0 += l0;
+        a2r1 += l1;
         fence_proxy_async_smem();
         tc_fence_before();
         wg_sync(wg);
         if (wtid == 0) {
           mbar_arrive(&ms->su_free[bb]);
-          mbar_arrive(&ms->pready[bb]);
+          mbar_arrive(&ms->pready);
           if (!last_chunk) mbar_arrive(&ms->sready[(n + 1) & 1]);
         }
-        if (!hold && n >= 1) stream_epilogue(n - 1);
       }
       if (!alive) break;
-      if (!hold) {
-        // output of the sequence's last chunk
-        if (!wg_wait(wg, wtid, &ms->o_full[(n - 1) & 1], ph_of(n - 1), ms, hdr, 0x402, slot)) { alive = false; break; }
-        tc_fence_after();
-        stream_epilogue(n - 1);
-      } else {
+      if (hold) {
         // segment summary of this round: U_seg = local end state, its log2 decay
-        float* mine = fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64);
-        if (tile1) {
-          for (int e = 0; e < 64; e += 4)
-            __stcg(reinterpret_cast<float4*>(mine + trow * 64 + e), make_float4(Sreg[e], Sreg[e + 1], Sreg[e + 2], Sreg[e + 3]));
-          mine[4096 + trow] = a2seg_row;
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) {
+          __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb], Ls[4 * cb + 1]));
+          __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+        }
+        if ((lane & 3) == 0) {
+          mine[4096 + r0] = a2r0;
+          mine[4096 + r1] = a2r1;
         }
         __threadfence();
         wg_sync(wg);
         if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
       }
     }
-    bulk_wait_all<0>();
   } else if (warp < 12) {
-    // ===================================================================== WG_C: HOLD round end
-    if (hold) {
-      const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
-      const int trow = wq * 16 + (lane & 15);
-      const bool tile1 = lane >= 16;
-      const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-      uint8_t* orow = smem + kOffOut + trow * 256;
+    // ===================================================================== WG_C: epilogue, HOLD round end
+    const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
+    const int trow = wq * 16 + (lane & 15);
+    const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    int slot = 0;
+    if (!hold) {
+      const int pairs = (fp.Nc + 1) / 2;
+      for (int pr = 0; pr < pairs; ++pr) {
+        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) break;
+        tc_fence_after();
+        const long long s = (long long)(2 * pr + tsel) * kChunk + trow;
+        epilogue_row<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(pr & 1), 2 * pr + tsel < fp.Nc && s < L, s,
+                           nonfinite);
+        tc_fence_before();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->o_free[pr & 1]);
+      }
+    } else {
       // state entries owned by this CTA, in groups of 8 (one 16-byte chunk of a start-state row)
       const int g0 = (int)((long long)seg * 512 / fp.n_s), g1 = (int)((long long)(seg + 1) * 512 / fp.n_s);
       float Sin[kMaxOwn];  // owned entries' running state across rounds (two groups per thread)
@@ -777,7 +805,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       unsigned int* ctr = fp.counters + (size_t)seq * 2;
       const float* aggs0 = fp.agg + (size_t)seq * 2 * fp.n_s * (4096 + 64);
       uint16_t* sst = fp.sstart + (size_t)seq * fp.n_s * 4096;
-      int slot = 0;
       for (int r = 0; r < rounds; ++r) {
         const int sig = r & 1;
         const Span sp = round_span(fp, r, seg);
@@ -818,10 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (sb + t < fp.n_s) {
                   uint32_t pk[4];
 #pragma unroll
-                  for (int x = 0; x < 4; ++x) {
-                    if (!f16_ok(sv[2 * x]) || !f16_ok(sv[2 * x + 1])) range_bad = true;
-                    pk[x] = Pack2<__half>::pack(sv[2 * x], sv[2 * x + 1]);
-                  }
+                  for (int x = 0; x < 4; ++x) pk[x] = pack_h2(sv[2 * x], sv[2 * x + 1]);
                   __stcg(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sst + (size_t)(sb + t) * 4096) + soff),
                          make_uint4(pk[0], pk[1], pk[2], pk[3]));
                   const float d = ex2(dk[t]);
@@ -856,24 +880,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane tile 1)
         const int G = sp.c1 - sp.c0;
         for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
-          for (int pass = 0; pass < 2; ++pass) {
-            const int gi = 2 * m2 + pass;
-            const bool mine = (pass == 0) ? !tile1 : tile1;
-            epilogue_rows<Tout>(p, b, h, tl + kColO + 128u * sig + 64u * (uint32_t)m2, mine && gi < G,
-                                (long long)(sp.c0 + gi) * kChunk + trow, orow, fp.scale);
-            bulk_wait_read<0>();
-            __syncwarp();
-          }
+          const int gi = 2 * m2 + tsel;
+          const long long s = (long long)(sp.c0 + gi) * kChunk + trow;
+          epilogue_row<Tout>(p, b, h, tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, gi < G && s < L, s,
+                             nonfinite);
         }
         tc_fence_before();
         wg_sync(wg);
         if (wtid == 0) mbar_arrive(&ms->set_free[sig]);
       }
-      bulk_wait_all<0>();
     }
   }
 
-  if (__any_sync(0xffffffffu, range_bad) && lane == 0) record_error(hdr, GTR_ERR_RANGE, 0x500u + warp);
+  if (__any_sync(0xffffffffu, nonfinite != nonfinite) && lane == 0) record_error(hdr, GTR_ERR_RANGE, 0x500u + warp);
 
   // ---- teardown
   tc_fence_before();
@@ -969,7 +988,6 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.Nc = p.n_chunks();
   fp.mode = pl.mode;
   fp.grid = pl.grid;
-  fp.scale = 1.0f / sqrtf((float)p.d_k);
   // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the
   // fp16 rounding of the small Qh values keep their precision
   fp.max_exp2 = 11.5f;
