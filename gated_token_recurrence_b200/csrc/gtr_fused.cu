@@ -68,7 +68,7 @@ constexpr int kOffS = kOffP + kTile;                       // [2] chunk-start st
 constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
 constexpr int kOffHeld = kOffSst + kTile;                  // [2 sets][kHeldPerSet]
 constexpr int kOffMisc = kOffHeld + 2 * kHeldPerSet * kTile;
-constexpr int kMiscBytes = 3072;
+constexpr int kMiscBytes = 6144;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 
 // tensor memory columns
@@ -83,14 +83,15 @@ static_assert(kColO + 2 * kSetCols <= kTmemCols, "tensor memory budget");
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
 constexpr size_t kMaxHoldSegments = 256;  // CTAs of one launch in HOLD mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxHoldSegments * sizeof(unsigned int);
+constexpr int kScanBlock = 12;           // segments one WG_C thread composes in registers
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
-constexpr int kMaxOwn = 16;               // state entries per WG_C thread (n_s >= 2)
 
 struct FusedParams {
   Problem p;
   WsHeader* hdr;
   unsigned int* counters;  // [n_seq][2], monotonic within a call, zero between calls
   float* agg;              // [n_seq][2 round parities][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
+  float* carry;            // [n_seq][64*64] state entering the current round, fp32
   uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
   int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD
   int grid;
@@ -101,7 +102,7 @@ struct Misc {
   uint64_t full[kStages], empty[kStages];
   uint64_t opready[2], su_full[2], su_free[2], sready[2], pready, pv_done;
   uint64_t o_full[2], o_free[2];
-  uint64_t agg_pub[2], corr_ready[2], corr_done[2], set_free[2];
+  uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
@@ -109,6 +110,9 @@ struct Misc {
   int fb[kStages];       // stage -> scores from the CUDA cores
   alignas(16) float red[4][64];   // WG_A cumsum: per-warp channel totals
   float a2last[kStages][64];      // stage -> in-chunk log2 decay per channel
+  long long rowoff[2][64];        // producer: token-head row of each chunk row (-1 past the end)
+  float xD[kWG];                  // WG_C scan: block transfers exchanged between threads
+  alignas(16) float4 xU[kWG];
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -208,62 +212,81 @@ template <> struct In2<__nv_bfloat16> {
 
 __device__ __forceinline__ void sts32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
 
-// Half an output row (32 values of a token-head starting at column col0, in registers)
-// -> its grid cell.  `nf` collects x * 0 over the stored values: it turns NaN once any
-// of them is not finite.
+// The 32 output rows of one warp (its lanes of a lane-tile pair region in tensor
+// memory) -> their grid cells, 32 columns at a time.  Each lane writes its row into a
+// per-warp staging tile in shared memory (16-byte chunks, XOR-swizzled by row so the
+// writes spread over all banks); after __syncwarp the warp copies the tile out with
+// whole rows per 8 (fp32) or 4 (16-bit) lanes, so every 16-byte global store
+// instruction covers 4 or 8 full row segments.  `nf` collects x * 0 over the values:
+// it turns NaN once any of them is not finite.
 template <typename Tout>
-__device__ __forceinline__ void store_out_half(const Problem& p, int b, int h, long long s, int col0,
-                                               const float* v, float& nf) {
-  const long long m = scan_to_token(s, p.direction, p.H, p.W);
-  Tout* dst = reinterpret_cast<Tout*>(p.out) + (((long long)b * p.L() + m) * p.heads + h) * 64 + col0;
-  if constexpr (sizeof(Tout) == 4) {
-#pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      nf = fmaf(v[e], 0.f, nf);
-      nf = fmaf(v[e + 1], 0.f, nf);
-      nf = fmaf(v[e + 2], 0.f, nf);
-      nf = fmaf(v[e + 3], 0.f, nf);
-      __stcs(reinterpret_cast<float4*>(dst + e), make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]));
-    }
-  } else {
-    __half2 acc = __float2half2_rn(0.f);
-    const __half2 zero = __float2half2_rn(0.f);
-#pragma unroll
-    for (int e = 0; e < 32; e += 8) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if constexpr (std::is_same<Tout, __half>::value) {
-          pk[u] = pack_h2(v[e + 2 * u], v[e + 2 * u + 1]);
-          acc = __hfma2(bits_h2(pk[u]), zero, acc);
-        } else {
-          __nv_bfloat162 hb = __floats2bfloat162_rn(v[e + 2 * u], v[e + 2 * u + 1]);
-          pk[u] = *reinterpret_cast<uint32_t*>(&hb);
-          nf = fmaf(v[e + 2 * u], 0.f, nf);
-          nf = fmaf(v[e + 2 * u + 1], 0.f, nf);
-        }
-      }
-      __stcs(reinterpret_cast<uint4*>(dst + e), make_uint4(pk[0], pk[1], pk[2], pk[3]));
-    }
-    if constexpr (std::is_same<Tout, __half>::value) {
-      const float2 a = __half22float2(acc);
-      nf += a.x + a.y;
-    }
-  }
-}
-
-// One output row of a lane-tile pair region in tensor memory (this thread's lane),
-// 32 columns at a time, -> its grid cell when `valid`.
-template <typename Tout>
-__device__ __forceinline__ void epilogue_row(const Problem& p, int b, int h, uint32_t taddr, bool valid,
-                                             long long s, float& nf) {
+__device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, uint32_t taddr, bool valid,
+                                              long long s, uint8_t* wstage, int lane, float& nf) {
+  constexpr int kRowB = 32 * (int)sizeof(Tout);  // staged bytes per row and half
+  constexpr int kLanesPerRow = kRowB / 16;       // 8 (fp32) or 4 (16-bit)
+  constexpr int kRowsPerOp = 32 / kLanesPerRow;
+  long long mrow = -1;
+  if (valid) mrow = ((long long)b * p.L() + scan_to_token(s, p.direction, p.H, p.W)) * p.heads + h;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     float v[32];
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
-    if (valid) store_out_half<Tout>(p, b, h, s, 32 * half, v, nf);
+    uint8_t* buf = wstage + half * 32 * kRowB;
+    // 16-byte chunk j of row R sits at R*kRowB + 16*(j ^ sw(R))
+    auto chunk_at = [&](int R, int j) -> int {
+      const int swz = (kLanesPerRow == 8) ? (R & 7) : ((R >> 1) & 3);
+      return R * kRowB + 16 * (j ^ swz);
+    };
+    if constexpr (sizeof(Tout) == 4) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        nf = fmaf(v[4 * j], 0.f, nf);
+        nf = fmaf(v[4 * j + 1], 0.f, nf);
+        nf = fmaf(v[4 * j + 2], 0.f, nf);
+        nf = fmaf(v[4 * j + 3], 0.f, nf);
+        *reinterpret_cast<float4*>(buf + chunk_at(lane, j)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      }
+    } else {
+      __half2 acc = __float2half2_rn(0.f);
+      const __half2 zero = __float2half2_rn(0.f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x0 = v[8 * j + 2 * u], x1 = v[8 * j + 2 * u + 1];
+          if constexpr (std::is_same<Tout, __half>::value) {
+            pk[u] = pack_h2(x0, x1);
+            acc = __hfma2(bits_h2(pk[u]), zero, acc);
+          } else {
+            __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+            pk[u] = *reinterpret_cast<uint32_t*>(&hb);
+            nf = fmaf(x0, 0.f, nf);
+            nf = fmaf(x1, 0.f, nf);
+          }
+        }
+        *reinterpret_cast<uint4*>(buf + chunk_at(lane, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      if constexpr (std::is_same<Tout, __half>::value) {
+        const float2 a = __half22float2(acc);
+        nf += a.x + a.y;
+      }
+    }
+    __syncwarp();
+    const int jj = lane % kLanesPerRow;
+#pragma unroll
+    for (int it = 0; it < kLanesPerRow; ++it) {
+      const int R = it * kRowsPerOp + lane / kLanesPerRow;
+      const long long mr = __shfl_sync(0xffffffffu, mrow, R);
+      const uint4 x = *reinterpret_cast<const uint4*>(buf + chunk_at(R, jj));
+      if (mr >= 0) {
+        Tout* dst = reinterpret_cast<Tout*>(p.out) + mr * 64 + 32 * half;
+        __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst) + 16 * jj), x);
+      }
+    }
   }
+  __syncwarp();  // the staging tile is free again
 }
 
 struct Span {
@@ -280,6 +303,35 @@ __device__ __forceinline__ Span round_span(const FusedParams& fp, int r, int s) 
   sp.c1 = min(fp.Nc, (r * fp.n_s + s + 1) * gr);
   return sp;
 }
+
+// Position in a CTA's chunk sequence: round r, chunk c, index g within the round.
+// Rounds without chunks only occur at the end of a sequence.
+struct Cursor {
+  int r, c, g;
+  Span sp;
+  __device__ void settle(const FusedParams& fp, int seg, int rounds) {
+    while (r < rounds && c >= sp.c1) {
+      ++r;
+      g = 0;
+      if (r < rounds) {
+        sp = round_span(fp, r, seg);
+        c = sp.c0;
+      }
+    }
+  }
+  __device__ void start(const FusedParams& fp, int seg, int rounds) {
+    r = 0;
+    g = 0;
+    sp = round_span(fp, 0, seg);
+    c = sp.c0;
+    settle(fp, seg, rounds);
+  }
+  __device__ void advance(const FusedParams& fp, int seg, int rounds) {
+    ++c;
+    ++g;
+    settle(fp, seg, rounds);
+  }
+};
 
 // Phase parity for the n-th use of a double-buffered barrier, and for waiting on its
 // release by use n-2 (passes at once for n < 2 on a fresh barrier).
@@ -319,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
       mbar_init(&ms->agg_pub[i], 1);
-      mbar_init(&ms->corr_ready[i], 1);
+      mbar_init(&ms->round_done[i], 1);
       mbar_init(&ms->corr_done[i], 1);
       mbar_init(&ms->set_free[i], 1);
     }
@@ -348,43 +400,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 12 || warp == 13) {
     // ===================================================================== producer (cp.async)
-    // Thread t loads row t (scan position c*64 + t) of Q, K, V (128 B each, placed in
-    // the 128-byte-swizzle layout) and of the log-gates (256 B, plain).  Rows past the
-    // sequence end are zero-filled (source size 0).
-    const int pt = tid - 12 * 32;  // 0..63 = chunk row
+    // Per chunk, thread t first resolves the grid row of scan position c*64 + t (the
+    // direction remap) into a shared table; then the 64 threads copy the tiles with
+    // whole 128-byte rows per group of 8 threads (Q, K, V: placed in the 128-byte-swizzle
+    // layout) and 256-byte gate rows per group of 16, so each warp-wide copy touches
+    // only 4 (2) full lines.  Rows past the sequence end are zero-filled (source size 0).
+    const int pt = tid - 12 * 32;  // 0..63
     int n = 0;
     bool stop = false;
     const uint8_t* gq = reinterpret_cast<const uint8_t*>(p.q);
     const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.k);
     const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.v);
     const uint8_t* gg = reinterpret_cast<const uint8_t*>(p.log_gamma);
+    const int j8 = pt & 7, rq = pt >> 3;     // 16-byte column, row within a group of 8
+    const int j16 = pt & 15, rg = pt >> 4;   // gate rows: 16-byte column, row within 4
     for (int r = 0; r < rounds && !stop; ++r) {
       const Span sp = round_span(fp, r, seg);
       for (int c = sp.c0; c < sp.c1; ++c, ++n) {
         const int st = n % kStages;
+        long long* rows = ms->rowoff[n & 1];
+        {
+          const long long s = (long long)c * kChunk + pt;
+          rows[pt] = s < L ? token_head_row(p, b, h, s) : -1ll;
+        }
         int ok = 0;
         if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
-        uint8_t* sb = smem + kOffStage + st * kStageBytes;
-        const long long s = (long long)c * kChunk + pt;
-        const bool valid = s < L;
-        const long long row = valid ? token_head_row(p, b, h, s) : 0;
-        const uint32_t nb = valid ? 16u : 0u;
-        const uint8_t* q16 = gq + row * 128;
-        const uint8_t* k16 = gk + row * 128;
-        const uint8_t* v16 = gv + row * 128;
-        const uint8_t* g32 = gg + row * 256;
-        const uint32_t d0 = smem_u32(sb) + pt * 128;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
+        asm volatile("bar.sync 4, 64;" ::: "memory");  // the row table is complete
+        if (*(volatile int*)&ms->abort) stop = true;
+        if (stop) break;
+        const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t sw = (uint32_t)((j ^ (pt & 7)) << 4);
-          cp_async16(d0 + sw, q16 + 16 * j, nb);
-          cp_async16(d0 + kTile + sw, k16 + 16 * j, nb);
-          cp_async16(d0 + 2 * kTile + sw, v16 + 16 * j, nb);
+        for (int it = 0; it < 8; ++it) {
+          const int row = 8 * it + rq;
+          const long long ro = rows[row];
+          const uint32_t nb = ro >= 0 ? 16u : 0u;
+          const long long src = (ro >= 0 ? ro : 0) * 128 + 16 * j8;
+          const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
+          cp_async16(dst, gq + src, nb);
+          cp_async16(dst + kTile, gk + src, nb);
+          cp_async16(dst + 2 * kTile, gv + src, nb);
         }
-        const uint32_t dg = smem_u32(sb) + 3 * kTile + pt * 256;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) cp_async16(dg + 16 * j, g32 + 16 * j, nb);
+        for (int it = 0; it < 16; ++it) {
+          const int row = 4 * it + rg;
+          const long long ro = rows[row];
+          const uint32_t nb = ro >= 0 ? 16u : 0u;
+          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16, gg + (ro >= 0 ? ro : 0) * 256 + 16 * j16, nb);
+        }
         cp_async_arrive_noinc(&ms->full[st]);
       }
     }
@@ -392,44 +455,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ===================================================================== MMA issuer
+    // Software-pipelined over the CTA's chunk sequence: stage 1 of chunk n (scores and
+    // U') is issued before stage 2 of chunk n-1 (O = Qh S + P V) waits for its masked
+    // scores, so the masking warps always find the next score tile ready.
     if (lane == 0) {
       const uint32_t id_qk = idesc_f16(0, 64, 64, 0, 0);  // A K-major, B K-major
       const uint32_t id_kv = idesc_f16(0, 64, 64, 1, 1);  // A MN-major, B MN-major
       const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);  // A K-major, B MN-major
       const uint32_t s_base = smem_u32(smem);
-      int n = 0;
-      int next_corr = 0;  // oldest round whose correction is not issued yet (HOLD)
-      bool ok = true;
-      // held outputs of round rc += (Q 2^(A_seg)) S_segment_start
-      auto issue_corr = [&](int rc, bool block) -> bool {
-        const int sig = rc & 1;
-        if (block) {
-          if (!wait_bar(&ms->corr_ready[sig], ph_of(rc), ms, hdr, 0x205)) return false;
-        } else if (!mbar_try_wait(&ms->corr_ready[sig], ph_of(rc))) {
-          return false;
-        }
-        tc_fence_after();
-        const Span spc = round_span(fp, rc, seg);
-        const int G = spc.c1 - spc.c0;
-        for (int g = 0; g < G; ++g) {
-          const uint32_t d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
-          const uint32_t a_h = s_base + kOffHeld + (sig * kHeldPerSet + g) * kTile;
-          for (int k = 0; k < 4; ++k)
-            mma_f16(d_o, sw128_desc(a_h + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
-        }
-        mma_commit(&ms->corr_done[sig]);
-        return true;
-      };
-      for (int r = 0; r < rounds && ok; ++r) {
+      int total = 0;
+      for (int r = 0; r < rounds; ++r) {
         const Span sp = round_span(fp, r, seg);
-        const int sig = r & 1;
-        if (hold && r >= 2) {
-          // this set's held slots are reused: round r-2's correction must be issued and its
-          // epilogue finished first
-          while (ok && next_corr <= r - 2) ok = issue_corr(next_corr++, true);
-          if (!ok || !wait_bar(&ms->set_free[sig], ph_free(r), ms, hdr, 0x206)) { ok = false; break; }
-        }
-        for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
+        total += sp.c1 - sp.c0;
+      }
+      Cursor z;  // stage-2 position (round, chunk, index in round)
+      z.start(fp, seg, rounds);
+      bool ok = true;
+      for (int n = 0; n <= total && ok; ++n) {
+        if (n < total) {
           const int bb = n & 1, st = n % kStages;
           const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
           const uint32_t a_k = a_q + kTile;                            // Kh
@@ -445,31 +488,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k)  // U' = Kh^T V
             mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
           mma_commit(&ms->su_full[bb]);
+        }
+        if (n >= 1) {
+          const int m = n - 1, bb = m & 1, st = m % kStages;
+          const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
+          const uint32_t a_v = a_q + 2 * kTile;
+          const int sig = z.r & 1;
           uint32_t d_o;
           if (hold) {
-            d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+            // a held set is reused: the epilogue of the round two back must be finished
+            if (z.g == 0 && z.r >= 2 && !wait_bar(&ms->set_free[sig], ph_free(z.r), ms, hdr, 0x206)) { ok = false; break; }
+            d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(z.g >> 1) + ((z.g & 1) ? kLaneTile1 : 0u);
           } else {
-            const int pr = n >> 1;  // output pair: chunks 2pr (lane tile 0) and 2pr+1 (lane tile 1)
-            d_o = tmem + kColO + 64u * (uint32_t)(pr & 1) + ((n & 1) ? kLaneTile1 : 0u);
-            if (!(n & 1) && !wait_bar(&ms->o_free[pr & 1], ph_free(pr), ms, hdr, 0x202)) { ok = false; break; }
+            const int pr = m >> 1;  // output pair: chunks 2pr (lane tile 0) and 2pr+1 (lane tile 1)
+            d_o = tmem + kColO + 64u * (uint32_t)(pr & 1) + ((m & 1) ? kLaneTile1 : 0u);
+            if (!(m & 1) && !wait_bar(&ms->o_free[pr & 1], ph_free(pr), ms, hdr, 0x202)) { ok = false; break; }
           }
-          if (!wait_bar(&ms->sready[bb], ph_of(n), ms, hdr, 0x203)) { ok = false; break; }
+          if (!wait_bar(&ms->sready[bb], ph_of(m), ms, hdr, 0x203)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_s = s_base + kOffS + bb * kTile;
           for (int k = 0; k < 4; ++k)  // O = Qh S
             mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-          if (!wait_bar(&ms->pready, (uint32_t)n & 1u, ms, hdr, 0x204)) { ok = false; break; }
+          if (!wait_bar(&ms->pready, (uint32_t)m & 1u, ms, hdr, 0x204)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_p = s_base + kOffP;
           for (int k = 0; k < 4; ++k)  // O += P V
             mma_f16(d_o, sw128_desc(a_p + 32 * k), sw128_desc(a_v + 2048 * k), id_qs, 1);
           mma_commit(&ms->pv_done);
           mma_commit(&ms->empty[st]);
-          if (!hold && ((n & 1) || c + 1 == sp.c1)) mma_commit(&ms->o_full[(n >> 1) & 1]);
-          if (hold && next_corr < r && issue_corr(next_corr, false)) ++next_corr;
+          const bool round_end = z.c + 1 == z.sp.c1;
+          if (!hold && ((m & 1) || round_end)) mma_commit(&ms->o_full[(m >> 1) & 1]);
+          if (hold && round_end) mma_commit(&ms->round_done[sig]);
+          z.advance(fp, seg, rounds);
         }
       }
-      while (ok && hold && next_corr < rounds) ok = issue_corr(next_corr++, true);
       // every MMA issued here has completed before tensor memory is freed
       mma_commit(&ms->mma_final);
       const uint64_t t0 = globaltimer();
@@ -783,81 +835,114 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int trow = wq * 16 + (lane & 15);
     const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    constexpr int kWarpStage = 2 * 32 * 32 * (int)sizeof(Tout);  // two half-row tiles per warp
+    static_assert(4 * kWarpStage <= kHeldPerSet * kTile, "output staging fits a held set");
     int slot = 0;
     if (!hold) {
+      // output staging: the held-tile area, unused in this mode
+      uint8_t* wstage = smem + kOffHeld + wq * kWarpStage;
       const int pairs = (fp.Nc + 1) / 2;
       for (int pr = 0; pr < pairs; ++pr) {
         if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) break;
         tc_fence_after();
         const long long s = (long long)(2 * pr + tsel) * kChunk + trow;
-        epilogue_row<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(pr & 1), 2 * pr + tsel < fp.Nc && s < L, s,
-                           nonfinite);
+        epilogue_warp<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(pr & 1), 2 * pr + tsel < fp.Nc && s < L, s, wstage,
+                            lane, nonfinite);
         tc_fence_before();
         wg_sync(wg);
         if (wtid == 0) mbar_arrive(&ms->o_free[pr & 1]);
       }
     } else {
-      // state entries owned by this CTA, in groups of 8 (one 16-byte chunk of a start-state row)
-      const int g0 = (int)((long long)seg * 512 / fp.n_s), g1 = (int)((long long)(seg + 1) * 512 / fp.n_s);
-      float Sin[kMaxOwn];  // owned entries' running state across rounds (two groups per thread)
-#pragma unroll
-      for (int u = 0; u < kMaxOwn; ++u) Sin[u] = 0.f;
+      // Round-end scan of the segment summaries.  This CTA owns state entries
+      // [4 f0, 4 f1) (float4 units f, F of them).  Threads split into nB blocks of bs
+      // consecutive segments x FP float4 columns (nB * FP <= 128): a thread loads its
+      // block's summaries for its f all at once (consecutive threads read consecutive
+      // float4s), composes them sequentially, and the block compositions are exchanged
+      // through shared memory; each thread then walks its segments again from its
+      // block's carry-in, writing each segment's start state (fp16, MMA layout).  The
+      // carry (state entering the round, fp32) lives in the workspace between rounds.
+      const int ns = fp.n_s;
+      const int f0 = (int)((long long)seg * 1024 / ns), f1 = (int)((long long)(seg + 1) * 1024 / ns);
+      const int F = f1 - f0;
+      int nB = kWG / (F > 0 ? F : 1);
+      nB = nB < 1 ? 1 : (nB > ns ? ns : nB);
+      if ((ns + nB - 1) / nB > kScanBlock) nB = (ns + kScanBlock - 1) / kScanBlock;
+      const int bs = (ns + nB - 1) / nB;
+      const int FP = kWG / nB;
+      const int bi = wtid / FP, fi = wtid % FP;
+      const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
       unsigned int* ctr = fp.counters + (size_t)seq * 2;
-      const float* aggs0 = fp.agg + (size_t)seq * 2 * fp.n_s * (4096 + 64);
-      uint16_t* sst = fp.sstart + (size_t)seq * fp.n_s * 4096;
+      const float* aggs0 = fp.agg + (size_t)seq * 2 * ns * (4096 + 64);
+      uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
+      float4* carry = reinterpret_cast<float4*>(fp.carry + (size_t)seq * 4096);
+      const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
+      const uint32_t s_base = smem_u32(smem);
       for (int r = 0; r < rounds; ++r) {
         const int sig = r & 1;
         const Span sp = round_span(fp, r, seg);
-        const float* aggs = aggs0 + (size_t)sig * fp.n_s * (4096 + 64);
+        const float* aggs = aggs0 + (size_t)sig * ns * (4096 + 64);
         if (!wg_wait(wg, wtid, &ms->agg_pub[sig], ph_of(r), ms, hdr, 0x600, slot)) break;
-        const unsigned int target = (unsigned int)(r + 1) * (unsigned int)fp.n_s;
+        const unsigned int target = (unsigned int)(r + 1) * (unsigned int)ns;
         bool ok0 = true;
         if (wtid == 0) {
           red_release_add(ctr, 1u);
           ok0 = wait_counter(ctr, target, ms, hdr, 0x601);
         }
         if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
-        // scan over the sequence's segments for my entries: S_start[s] in fp16, MMA layout.
-        // Loads for four segments are in flight at a time; each step writes 16 bytes.
+        for (int base = f0; base < f1; base += FP) {
+          const int f = base + fi;
+          const bool act = bi < nB && f < f1;
+          const int kk = f >> 4;
+          float4 u[kScanBlock];
+          float dd[kScanBlock];
+          float4 X = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (act && r > 0) X = __ldcg(carry + f);
 #pragma unroll
-        for (int u = 0; u < kMaxOwn / 8; ++u) {
-          const int gi = g0 + u * kWG + wtid;
-          if (gi < g1) {
-            const int kk = gi >> 3, e = gi * 8;
-            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)gi & 7u) ^ ((uint32_t)kk & 7u)) << 4);
-            float sv[8];
+          for (int j = 0; j < kScanBlock; ++j) {
+            const int sg = s_lo + j;
+            const bool on = act && sg < s_hi;
+            const float* a2p = aggs + (size_t)(on ? sg : 0) * (4096 + 64);
+            u[j] = on ? __ldcg(reinterpret_cast<const float4*>(a2p) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            dd[j] = on ? __ldcg(a2p + 4096 + kk) : 0.f;
+          }
+          // this block's transfer: state_after = D * state_before + U
+          float D = 1.f;
+          float4 U = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) sv[x] = Sin[u * 8 + x];
-            for (int sb = 0; sb < fp.n_s; sb += 4) {
-              float4 ua[4], ub[4];
-              float dk[4];
+          for (int j = 0; j < kScanBlock; ++j) {
+            dd[j] = ex2(dd[j]);  // inactive entries: 2^0 = 1 with a zero summary
+            U = make_float4(fmaf(dd[j], U.x, u[j].x), fmaf(dd[j], U.y, u[j].y), fmaf(dd[j], U.z, u[j].z),
+                            fmaf(dd[j], U.w, u[j].w));
+            D *= dd[j];
+          }
+          if (nB > 1) {
+            if (bi < nB) {
+              ms->xD[bi * FP + fi] = D;
+              ms->xU[bi * FP + fi] = U;
+            }
+            wg_sync(wg);
+            for (int b2 = 0; b2 < bi && b2 < nB; ++b2) {
+              const float d2 = ms->xD[b2 * FP + fi];
+              const float4 u2 = ms->xU[b2 * FP + fi];
+              X = make_float4(fmaf(d2, X.x, u2.x), fmaf(d2, X.y, u2.y), fmaf(d2, X.z, u2.z), fmaf(d2, X.w, u2.w));
+            }
+          }
+          if (act) {
+            const int v0 = 4 * (f & 15);
+            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (v0 & 7) * 2;
 #pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                if (sb + t < fp.n_s) {
-                  const float* a2p = aggs + (size_t)(sb + t) * (4096 + 64);
-                  ua[t] = __ldcg(reinterpret_cast<const float4*>(a2p + e));
-                  ub[t] = __ldcg(reinterpret_cast<const float4*>(a2p + e + 4));
-                  dk[t] = __ldcg(a2p + 4096 + kk);
-                }
-              }
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                if (sb + t < fp.n_s) {
-                  uint32_t pk[4];
-#pragma unroll
-                  for (int x = 0; x < 4; ++x) pk[x] = pack_h2(sv[2 * x], sv[2 * x + 1]);
-                  __stcg(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(sst + (size_t)(sb + t) * 4096) + soff),
-                         make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                  const float d = ex2(dk[t]);
-                  const float uu[8] = {ua[t].x, ua[t].y, ua[t].z, ua[t].w, ub[t].x, ub[t].y, ub[t].z, ub[t].w};
-#pragma unroll
-                  for (int x = 0; x < 8; ++x) sv[x] = fmaf(d, sv[x], uu[x]);
-                }
+            for (int j = 0; j < kScanBlock; ++j) {
+              const int sg = s_lo + j;
+              if (sg < s_hi) {
+                const uint2 w = make_uint2(pack_h2(X.x, X.y), pack_h2(X.z, X.w));
+                __stcg(reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(sst + (size_t)sg * 4096) + soff), w);
+                X = make_float4(fmaf(dd[j], X.x, u[j].x), fmaf(dd[j], X.y, u[j].y), fmaf(dd[j], X.z, u[j].z),
+                                fmaf(dd[j], X.w, u[j].w));
               }
             }
-#pragma unroll
-            for (int x = 0; x < 8; ++x) Sin[u * 8 + x] = sv[x];
+            if (s_hi == ns) __stcg(carry + f, X);  // the last block's end state enters the next round
           }
+          if (nB > 1) wg_sync(wg);  // the exchange slots are reused by the next column pass
         }
         __threadfence();
         wg_sync(wg);
@@ -874,16 +959,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->corr_ready[sig]);
+        const int G = sp.c1 - sp.c0;
+        ok0 = true;
+        if (wtid == 0) {
+          // held outputs of this round += (Q 2^(A_seg)) S_segment_start, once their own
+          // MMAs have completed
+          if (G > 0) ok0 = wait_bar(&ms->round_done[sig], ph_of(r), ms, hdr, 0x604);
+          if (ok0) {
+            tc_fence_after();
+            for (int g = 0; g < G; ++g) {
+              const uint32_t d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+              const uint32_t a_h = s_base + kOffHeld + (sig * kHeldPerSet + g) * kTile;
+              for (int k = 0; k < 4; ++k)
+                mma_f16(d_o, sw128_desc(a_h + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
+            }
+            mma_commit(&ms->corr_done[sig]);
+          }
+        }
+        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
         if (!wg_wait(wg, wtid, &ms->corr_done[sig], ph_of(r), ms, hdr, 0x603, slot)) break;
         tc_fence_after();
-        // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane tile 1)
-        const int G = sp.c1 - sp.c0;
+        // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane
+        // tile 1); the set's Qh tiles, consumed by the correction, stage the rows
+        uint8_t* wstage = smem + kOffHeld + sig * kHeldPerSet * kTile + wq * kWarpStage;
         for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
           const int gi = 2 * m2 + tsel;
           const long long s = (long long)(sp.c0 + gi) * kChunk + trow;
-          epilogue_row<Tout>(p, b, h, tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, gi < G && s < L, s,
-                             nonfinite);
+          epilogue_warp<Tout>(p, b, h, tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, gi < G && s < L, s, wstage,
+                              lane, nonfinite);
         }
         tc_fence_before();
         wg_sync(wg);
@@ -982,6 +1085,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.counters = w.counters;
   fp.agg = w.agg;
   fp.sstart = w.sstart;
+  fp.carry = w.carry;
   fp.n_seq = pl.n_seq;
   fp.n_s = pl.n_s;
   fp.rounds = pl.rounds;
@@ -1010,7 +1114,9 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
 
 size_t fused_workspace_bytes(const Problem& p) {
   const size_t segs = hold_segments(p);
-  return sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t);
+  const size_t carry_seqs = segs ? (size_t)p.B * p.heads : 0;
+  return sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t) +
+         carry_seqs * 4096 * sizeof(float);
 }
 
 FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
@@ -1024,6 +1130,8 @@ FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
   w.agg = reinterpret_cast<float*>(base);
   base += 2 * segs * (4096 + 64) * sizeof(float);
   w.sstart = reinterpret_cast<uint16_t*>(base);
+  base += segs * 4096 * sizeof(uint16_t);
+  w.carry = reinterpret_cast<float*>(base);
   return w;
 }
 

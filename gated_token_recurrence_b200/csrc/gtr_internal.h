@@ -23,6 +23,7 @@ struct FusedWorkspace {
   unsigned int* counters;  // per-sequence arrival counters (zero between calls)
   float* agg;              // per-segment summaries
   uint16_t* sstart;        // per-segment start states (16-bit, MMA layout)
+  float* carry;            // per-sequence state entering the current round (fp32)
 };
 
 size_t split_workspace_bytes(const Problem& p);
