@@ -63,16 +63,16 @@ constexpr int kTile = 8192;
 constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
 constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V, G
 constexpr int kOffStage = 0;
-constexpr int kOffP = kOffStage + kStages * kStageBytes;   // masked scores
-constexpr int kOffS = kOffP + kTile;                       // [2] chunk-start states
+constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [2] chunk-start states
 constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
 constexpr int kOffHeld = kOffSst + kTile;                  // [2 sets][kHeldPerSet]
 constexpr int kOffMisc = kOffHeld + 2 * kHeldPerSet * kTile;
-constexpr int kMiscBytes = 6144;
+constexpr int kMiscBytes = 1920;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 
 // tensor memory columns
-constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0) and U' (lane tile 1)
+constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0; masked fp16 P over their first 32
+                                   // columns) and U' (lane tile 1)
 constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 output pairs; HOLD: [2 sets] x kSetCols
 constexpr uint32_t kLaneTile1 = 16u << 16;
 constexpr uint32_t kSetCols = 64u * (kHeldPerSet / 2);
@@ -100,7 +100,7 @@ struct FusedParams {
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
-  uint64_t opready[2], su_full[2], su_free[2], sready[2], pready, pv_done;
+  uint64_t opready[2], su_full[2], su_free[2], sready[2], pready[2], s_done[2];
   uint64_t o_full[2], o_free[2];
   uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
   uint64_t mma_final;
@@ -109,11 +109,11 @@ struct Misc {
   int go[3][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
   alignas(16) float red[4][64];   // WG_A cumsum: per-warp channel totals
-  float a2last[kStages][64];      // stage -> in-chunk log2 decay per channel
-  long long rowoff[2][64];        // producer: token-head row of each chunk row (-1 past the end)
-  float xD[kWG];                  // WG_C scan: block transfers exchanged between threads
-  alignas(16) float4 xU[kWG];
+  int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
 };
+// The in-chunk log2 decay per channel (a) of a staged chunk is kept in row 0 of its
+// gate tile once the gates are consumed; the round-end scan exchanges its block
+// transfers through the segment-start-state tile, which is idle at that point.
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -368,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
       mbar_init(&ms->sready[i], 1);
+      mbar_init(&ms->pready[i], 1);
+      mbar_init(&ms->s_done[i], 1);
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
       mbar_init(&ms->agg_pub[i], 1);
@@ -375,8 +377,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->corr_done[i], 1);
       mbar_init(&ms->set_free[i], 1);
     }
-    mbar_init(&ms->pready, 1);
-    mbar_init(&ms->pv_done, 1);
     mbar_init(&ms->mma_final, 1);
     ms->abort = 0;
     for (int i = 0; i < 3; ++i) ms->go[i][0] = ms->go[i][1] = 0;
@@ -385,13 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tmem_alloc(&ms->tmem_base, kTmemCols);
     tmem_relinquish();
-  }
-  if (warp >= 4 && warp < 8) {
-    // the masked-score tile: entries above the diagonal blocks stay zero for good
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    uint4* pz = reinterpret_cast<uint4*>(smem + kOffP);
-    for (int i = tid - kWG; i < kTile / 16; i += kWG) pz[i] = z;
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -418,10 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Span sp = round_span(fp, r, seg);
       for (int c = sp.c0; c < sp.c1; ++c, ++n) {
         const int st = n % kStages;
-        long long* rows = ms->rowoff[n & 1];
+        int* rows = ms->rowoff[n & 1];
         {
           const long long s = (long long)c * kChunk + pt;
-          rows[pt] = s < L ? token_head_row(p, b, h, s) : -1ll;
+          rows[pt] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
         }
         int ok = 0;
         if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
@@ -433,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
           const int row = 8 * it + rq;
-          const long long ro = rows[row];
-          const uint32_t nb = ro >= 0 ? 16u : 0u;
-          const long long src = (ro >= 0 ? ro : 0) * 128 + 16 * j8;
+          const int cell = rows[row];
+          const uint32_t nb = cell >= 0 ? 16u : 0u;
+          const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
           const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
           cp_async16(dst, gq + src, nb);
           cp_async16(dst + kTile, gk + src, nb);
@@ -444,9 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int it = 0; it < 16; ++it) {
           const int row = 4 * it + rg;
-          const long long ro = rows[row];
-          const uint32_t nb = ro >= 0 ? 16u : 0u;
-          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16, gg + (ro >= 0 ? ro : 0) * 256 + 16 * j16, nb);
+          const int cell = rows[row];
+          const uint32_t nb = cell >= 0 ? 16u : 0u;
+          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
+                     gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
         }
         cp_async_arrive_noinc(&ms->full[st]);
       }
@@ -455,9 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ===================================================================== MMA issuer
-    // Software-pipelined over the CTA's chunk sequence: stage 1 of chunk n (scores and
-    // U') is issued before stage 2 of chunk n-1 (O = Qh S + P V) waits for its masked
-    // scores, so the masking warps always find the next score tile ready.
+    // Event-driven over the CTA's chunk sequence: whichever of stage 1 (scores, U'),
+    // stage 2a (O = Qh S) and stage 2b (O += P V) has its inputs ready is issued, so a
+    // slow operand build never holds back the products of earlier chunks (and with
+    // them the release of their staging buffers).
     if (lane == 0) {
       const uint32_t id_qk = idesc_f16(0, 64, 64, 0, 0);  // A K-major, B K-major
       const uint32_t id_kv = idesc_f16(0, 64, 64, 1, 1);  // A MN-major, B MN-major
@@ -468,58 +463,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Span sp = round_span(fp, r, seg);
         total += sp.c1 - sp.c0;
       }
-      Cursor z;  // stage-2 position (round, chunk, index in round)
-      z.start(fp, seg, rounds);
-      bool ok = true;
-      for (int n = 0; n <= total && ok; ++n) {
-        if (n < total) {
-          const int bb = n & 1, st = n % kStages;
+      // output region of chunk m at cursor position z
+      auto out_region = [&](const Cursor& z, int m) -> uint32_t {
+        if (hold)
+          return tmem + kColO + kSetCols * (uint32_t)(z.r & 1) + 64u * (uint32_t)(z.g >> 1) + ((z.g & 1) ? kLaneTile1 : 0u);
+        return tmem + kColO + 64u * (uint32_t)((m >> 1) & 1) + ((m & 1) ? kLaneTile1 : 0u);
+      };
+      Cursor za, zb;  // positions of stage 2a and 2b
+      za.start(fp, seg, rounds);
+      zb.start(fp, seg, rounds);
+      int n1 = 0, n2a = 0, n2b = 0;
+      uint64_t t_last = globaltimer();
+      while (n2b < total) {
+        bool prog = false;
+        if (n2b < n2a && mbar_test(&ms->pready[n2b & 1], ph_of(n2b))) {
+          // stage 2b of chunk m: O += P V with P in tensor memory; the chunk's staging
+          // buffer and score region are free afterwards
+          const int m = n2b, bb = m & 1, st = m % kStages;
+          const uint32_t a_v = s_base + kOffStage + st * kStageBytes + 2 * kTile;
+          // P sits in the lane tile of the chunk's output (A and D rows share lanes)
+          const bool otile = hold ? (zb.g & 1) != 0 : (m & 1) != 0;
+          const uint32_t a_p = tmem + kColSU + 64u * bb + (otile ? kLaneTile1 : 0u);
+          const uint32_t d_o = out_region(zb, m);
+          tc_fence_after();
+          for (int k = 0; k < 4; ++k)
+            mma_f16_ta(d_o, a_p + 8 * k, sw128_desc(a_v + 2048 * k), id_qs, 1);
+          mma_commit(&ms->su_free[bb]);
+          mma_commit(&ms->empty[st]);
+          const bool round_end = zb.c + 1 == zb.sp.c1;
+          if (!hold && ((m & 1) || round_end)) mma_commit(&ms->o_full[(m >> 1) & 1]);
+          if (hold && round_end) mma_commit(&ms->round_done[zb.r & 1]);
+          zb.advance(fp, seg, rounds);
+          ++n2b;
+          prog = true;
+        }
+        if (n2a < n1) {
+          // stage 2a of chunk m: O = Qh S (S = the chunk-start state tile)
+          const int m = n2a, bb = m & 1, st = m % kStages;
+          bool rdy = mbar_test(&ms->sready[bb], ph_of(m));
+          if (hold) {
+            // a held set is reused: the epilogue of the round two back must be finished
+            if (za.g == 0 && za.r >= 2) rdy = rdy && mbar_test(&ms->set_free[za.r & 1], ph_free(za.r));
+          } else if (!(m & 1)) {
+            rdy = rdy && mbar_test(&ms->o_free[(m >> 1) & 1], ph_free(m >> 1));
+          }
+          if (rdy) {
+            const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
+            const uint32_t a_s = s_base + kOffS + bb * kTile;
+            const uint32_t d_o = out_region(za, m);
+            tc_fence_after();
+            for (int k = 0; k < 4; ++k)
+              mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
+            mma_commit(&ms->s_done[bb]);
+            za.advance(fp, seg, rounds);
+            ++n2a;
+            prog = true;
+          }
+        }
+        if (n1 < total && mbar_test(&ms->opready[n1 & 1], ph_of(n1)) && mbar_test(&ms->su_free[n1 & 1], ph_free(n1))) {
+          // stage 1 of chunk n: scores = Qh Kh^T (tensor-core chunks), U' = Kh^T V
+          const int n = n1, bb = n & 1, st = n % kStages;
           const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
           const uint32_t a_k = a_q + kTile;                            // Kh
           const uint32_t a_v = a_q + 2 * kTile;
-          if (!wait_bar(&ms->opready[bb], ph_of(n), ms, hdr, 0x200) ||
-              !wait_bar(&ms->su_free[bb], ph_free(n), ms, hdr, 0x201)) { ok = false; break; }
           tc_fence_after();
           const uint32_t su = tmem + kColSU + 64u * bb;
           if (!*(volatile int*)&ms->fb[st]) {
-            for (int k = 0; k < 4; ++k)  // scores = Qh Kh^T
+            for (int k = 0; k < 4; ++k)
               mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
           }
-          for (int k = 0; k < 4; ++k)  // U' = Kh^T V
+          for (int k = 0; k < 4; ++k)
             mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
           mma_commit(&ms->su_full[bb]);
+          ++n1;
+          prog = true;
         }
-        if (n >= 1) {
-          const int m = n - 1, bb = m & 1, st = m % kStages;
-          const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
-          const uint32_t a_v = a_q + 2 * kTile;
-          const int sig = z.r & 1;
-          uint32_t d_o;
-          if (hold) {
-            // a held set is reused: the epilogue of the round two back must be finished
-            if (z.g == 0 && z.r >= 2 && !wait_bar(&ms->set_free[sig], ph_free(z.r), ms, hdr, 0x206)) { ok = false; break; }
-            d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(z.g >> 1) + ((z.g & 1) ? kLaneTile1 : 0u);
-          } else {
-            const int pr = m >> 1;  // output pair: chunks 2pr (lane tile 0) and 2pr+1 (lane tile 1)
-            d_o = tmem + kColO + 64u * (uint32_t)(pr & 1) + ((m & 1) ? kLaneTile1 : 0u);
-            if (!(m & 1) && !wait_bar(&ms->o_free[pr & 1], ph_free(pr), ms, hdr, 0x202)) { ok = false; break; }
+        if (prog) {
+          t_last = globaltimer();
+        } else {
+          if (*(volatile int*)&ms->abort) break;
+          if (globaltimer() - t_last > 1000000000ull) {
+            record_error(hdr, GTR_ERR_TIMEOUT, 0x207);
+            *(volatile int*)&ms->abort = 1;
+            break;
           }
-          if (!wait_bar(&ms->sready[bb], ph_of(m), ms, hdr, 0x203)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_s = s_base + kOffS + bb * kTile;
-          for (int k = 0; k < 4; ++k)  // O = Qh S
-            mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-          if (!wait_bar(&ms->pready, (uint32_t)m & 1u, ms, hdr, 0x204)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_p = s_base + kOffP;
-          for (int k = 0; k < 4; ++k)  // O += P V
-            mma_f16(d_o, sw128_desc(a_p + 32 * k), sw128_desc(a_v + 2048 * k), id_qs, 1);
-          mma_commit(&ms->pv_done);
-          mma_commit(&ms->empty[st]);
-          const bool round_end = z.c + 1 == z.sp.c1;
-          if (!hold && ((m & 1) || round_end)) mma_commit(&ms->o_full[(m >> 1) & 1]);
-          if (hold && round_end) mma_commit(&ms->round_done[sig]);
-          z.advance(fp, seg, rounds);
+          __nanosleep(32);
         }
       }
       // every MMA issued here has completed before tensor memory is freed
@@ -695,9 +723,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             vt[i] = x;
           }
         }
-        if (rb == 0) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ms->a2last[st][8 * cc + e] = last[e];
+        if (rb == 0) {  // every gate read of this chunk is behind a warpgroup barrier by now
+          float4* lw = reinterpret_cast<float4*>(G + 8 * cc);
+          lw[0] = make_float4(last[0], last[1], last[2], last[3]);
+          lw[1] = make_float4(last[4], last[5], last[6], last[7]);
         }
         if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
 #pragma unroll
@@ -714,8 +743,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = 1, wtid = tid - kWG, wq = warp & 3;
     const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
-    uint8_t* prow0 = smem + kOffP + r0 * 128;
-    uint8_t* prow1 = smem + kOffP + r1 * 128;
     float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
     float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
     int slot = 0, n = 0;
@@ -743,7 +770,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
       a2r0 = a2r1 = 0.f;
-      {  // zero start state for this round's first chunk
+      {  // zero start state for this round's first chunk (its tile's last reader, the
+         // O = Qh S of chunk n-2, must be done)
+        if (n >= 2 && !wg_wait(wg, wtid, &ms->s_done[n & 1], ph_of(n - 2), ms, hdr, 0x403, slot)) break;
         const uint4 z = make_uint4(0, 0, 0, 0);
         uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n & 1) * kTile);
         for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
@@ -755,43 +784,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bb = n & 1, st = n % kStages;
         const bool last_chunk = (c + 1 == sp.c1);
         if (!wg_wait(wg, wtid, &ms->su_full[bb], ph_of(n), ms, hdr, 0x400, slot)) { alive = false; break; }
-        // P and the next state tile are free once the previous chunk's P V has completed
-        if (n >= 1 && !wg_wait(wg, wtid, &ms->pv_done, (uint32_t)(n - 1) & 1u, ms, hdr, 0x401, slot)) {
-          alive = false;
-          break;
-        }
         tc_fence_after();
         const bool fbk = ms->fb[st] != 0;
-        const float l0 = ms->a2last[st][r0], l1 = ms->a2last[st][r1];
+        const float* alast = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes + 3 * kTile);
+        const float l0 = alast[r0], l1 = alast[r1];
         const float dl0 = ex2(l0), dl1 = ex2(l1);
         float sc[32], u[32];
         tmem_ld16x256_x8(tl + kColSU + 64u * bb, sc);
         tmem_ld16x256_x8(tl + kColSU + 64u * bb + kLaneTile1, u);
         tmem_wait_ld();
-        // masked scores -> P (blocks right of the warp's diagonal stay zero)
-#pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-          if (cb <= 2 * wq + 1) {
-            float x0 = sc[4 * cb], x1 = sc[4 * cb + 1], x2 = sc[4 * cb + 2], x3 = sc[4 * cb + 3];
-            if (cb >= 2 * wq) {
-              const int j = 8 * cb + cq;
-              x0 = (j <= r0) ? x0 : 0.f;
-              x1 = (j + 1 <= r0) ? x1 : 0.f;
-              x2 = (j <= r1) ? x2 : 0.f;
-              x3 = (j + 1 <= r1) ? x3 : 0.f;
-            }
-            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
-            sts32(prow0 + o, pack_h2(x0, x1));
-            sts32(prow1 + o, pack_h2(x2, x3));
-          }
-        }
         // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           const float d = (x & 2) ? dl1 : dl0;
           Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
         }
+        a2r0 += l0;
+        a2r1 += l1;
         if (!last_chunk) {
+          // the next chunk's start state; its tile was last read by O = Qh S of chunk n-1
+          if (n >= 1 && !wg_wait(wg, wtid, &ms->s_done[(n + 1) & 1], ph_of(n - 1), ms, hdr, 0x402, slot)) {
+            alive = false;
+            break;
+          }
           uint8_t* srow0 = smem + kOffS + ((n + 1) & 1) * kTile + r0 * 128;
           uint8_t* srow1 = srow0 + 8 * 128;
 #pragma unroll
@@ -800,15 +815,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
             sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
           }
+          fence_proxy_async_smem();
         }
-        a2r0 += l0;
-        a2r1 += l1;
-        fence_proxy_async_smem();
+        // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
+        // the A operand of P V.  A rows are read from the lanes of the output rows, so P
+        // goes to the lane tile of the chunk's output region (tile 1: over U', already
+        // loaded).  Register 2c+q of the 16x128b shape is row r0 + 8q, column 4c + lane%4,
+        // i.e. the score pair (8c + cq, 8c + cq + 1) of that row.
+        uint32_t pw[16];
+#pragma unroll
+        for (int cb = 0; cb < 8; ++cb) {
+          float x0 = sc[4 * cb], x1 = sc[4 * cb + 1], x2 = sc[4 * cb + 2], x3 = sc[4 * cb + 3];
+          if (cb > 2 * wq + 1) {
+            x0 = x1 = x2 = x3 = 0.f;
+          } else if (cb >= 2 * wq) {
+            const int j = 8 * cb + cq;
+            x0 = (j <= r0) ? x0 : 0.f;
+            x1 = (j + 1 <= r0) ? x1 : 0.f;
+            x2 = (j <= r1) ? x2 : 0.f;
+            x3 = (j + 1 <= r1) ? x3 : 0.f;
+          }
+          pw[2 * cb] = pack_h2(x0, x1);
+          pw[2 * cb + 1] = pack_h2(x2, x3);
+        }
+        const bool otile = hold ? ((c - sp.c0) & 1) != 0 : (n & 1) != 0;
+        tmem_st16x128_x8(tl + kColSU + 64u * bb + (otile ? kLaneTile1 : 0u), pw);
+        tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);
         if (wtid == 0) {
-          mbar_arrive(&ms->su_free[bb]);
-          mbar_arrive(&ms->pready);
+          mbar_arrive(&ms->pready[bb]);
           if (!last_chunk) mbar_arrive(&ms->sready[(n + 1) & 1]);
         }
       }
@@ -875,6 +911,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* aggs0 = fp.agg + (size_t)seq * 2 * ns * (4096 + 64);
       uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
       float4* carry = reinterpret_cast<float4*>(fp.carry + (size_t)seq * 4096);
+      float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
+      float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
       const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
       const uint32_t s_base = smem_u32(smem);
       for (int r = 0; r < rounds; ++r) {
@@ -917,13 +955,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (nB > 1) {
             if (bi < nB) {
-              ms->xD[bi * FP + fi] = D;
-              ms->xU[bi * FP + fi] = U;
+              xD[bi * FP + fi] = D;
+              xU[bi * FP + fi] = U;
             }
             wg_sync(wg);
             for (int b2 = 0; b2 < bi && b2 < nB; ++b2) {
-              const float d2 = ms->xD[b2 * FP + fi];
-              const float4 u2 = ms->xU[b2 * FP + fi];
+              const float d2 = xD[b2 * FP + fi];
+              const float4 u2 = xU[b2 * FP + fi];
               X = make_float4(fmaf(d2, X.x, u2.x), fmaf(d2, X.y, u2.y), fmaf(d2, X.z, u2.z), fmaf(d2, X.w, u2.w));
             }
           }
