@@ -36,6 +36,9 @@
 //   warps 12-13 producer: cp.async of one token row per thread (direction remap,
 //               128-byte-swizzled placement, zero fill past the sequence end)
 //   warp 14     tcgen05 MMA issuer and tensor-memory owner
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <atomic>
 #include <mutex>
 #include <type_traits>
@@ -87,6 +90,10 @@ constexpr int kScanBlock = 12;           // segments one WG_C thread composes in
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 struct FusedParams {
+  // TMA tensor maps for Q, K, V (16-bit, 128-byte swizzle) and the log-gates (fp32):
+  // row view [B][L][heads][64] (4-D) or column view [B][H][W][heads][64] (5-D), boxes of
+  // 64 consecutive scan positions of one (batch, head)
+  CUtensorMap tq, tk, tv, tg;
   Problem p;
   WsHeader* hdr;
   unsigned int* counters;  // [n_seq][2], monotonic within a call, zero between calls
@@ -96,7 +103,10 @@ struct FusedParams {
   int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD
   int grid;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
+  int tma;                 // 1: every chunk is one TMA box per tensor; 0: cp.async row copies
+  int rev;                 // 1: chunks are staged in reverse scan order (right-to-left, bottom-to-top)
 };
+static_assert(alignof(FusedParams) >= 64, "tensor maps need 64-byte alignment");
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
@@ -232,7 +242,7 @@ __device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, ui
     float v[32];
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
-    uint8_t* buf = wstage + half * 32 * kRowB;
+    uint8_t* buf = wstage;  // one 32-row tile, reused by both halves
     // 16-byte chunk j of row R sits at R*kRowB + 16*(j ^ sw(R))
     auto chunk_at = [&](int R, int j) -> int {
       const int swz = (kLanesPerRow == 8) ? (R & 7) : ((R >> 1) & 3);
@@ -285,8 +295,8 @@ __device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, ui
         __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst) + 16 * jj), x);
       }
     }
+    __syncwarp();  // the staging tile is free again
   }
-  __syncwarp();  // the staging tile is free again
 }
 
 struct Span {
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&ms->full[i], kProducerThreads);
+      mbar_init(&ms->full[i], fp.tma ? 1 : kProducerThreads);
       mbar_init(&ms->empty[i], 1);
       ms->fb[i] = 0;
     }
@@ -392,61 +402,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ms->tmem_base;
 
   if (warp == 12 || warp == 13) {
-    // ===================================================================== producer (cp.async)
-    // Per chunk, thread t first resolves the grid row of scan position c*64 + t (the
-    // direction remap) into a shared table; then the 64 threads copy the tiles with
-    // whole 128-byte rows per group of 8 threads (Q, K, V: placed in the 128-byte-swizzle
-    // layout) and 256-byte gate rows per group of 16, so each warp-wide copy touches
-    // only 4 (2) full lines.  Rows past the sequence end are zero-filled (source size 0).
+    // ===================================================================== producer
+    // Staged chunk row r holds scan position c*64 + r, or c*64 + 63 - r for the reversed
+    // directions (right-to-left, bottom-to-top), where a chunk is stored in memory order.
     const int pt = tid - 12 * 32;  // 0..63
     int n = 0;
     bool stop = false;
-    const uint8_t* gq = reinterpret_cast<const uint8_t*>(p.q);
-    const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.k);
-    const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.v);
-    const uint8_t* gg = reinterpret_cast<const uint8_t*>(p.log_gamma);
-    const int j8 = pt & 7, rq = pt >> 3;     // 16-byte column, row within a group of 8
-    const int j16 = pt & 15, rg = pt >> 4;   // gate rows: 16-byte column, row within 4
-    for (int r = 0; r < rounds && !stop; ++r) {
-      const Span sp = round_span(fp, r, seg);
-      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
-        const int st = n % kStages;
-        int* rows = ms->rowoff[n & 1];
-        {
-          const long long s = (long long)c * kChunk + pt;
-          rows[pt] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
+    if (fp.tma) {
+      // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
+      // plain); rows past the sequence end arrive zero-filled.
+      if (pt == 0) {
+        for (int r = 0; r < rounds && !stop; ++r) {
+          const Span sp = round_span(fp, r, seg);
+          for (int c = sp.c0; c < sp.c1; ++c, ++n) {
+            const int st = n % kStages;
+            if (!wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100)) { stop = true; break; }
+            uint8_t* sb = smem + kOffStage + st * kStageBytes;
+            mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);
+            const long long s0 = (long long)c * kChunk;
+            if (p.direction <= GTR_R2L) {
+              // row view: 64 consecutive grid cells m (right-to-left: one image row)
+              long long m0 = s0;
+              if (p.direction == GTR_R2L) {
+                const long long y = s0 / p.W;
+                m0 = y * p.W + (p.W - 64 - (s0 - y * p.W));
+              }
+              tma_load_4d(sb, &fp.tq, &ms->full[st], 0, h, (int)m0, b);
+              tma_load_4d(sb + kTile, &fp.tk, &ms->full[st], 0, h, (int)m0, b);
+              tma_load_4d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, (int)m0, b);
+              tma_load_4d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, (int)m0, b);
+            } else {
+              // column view: 64 consecutive y of one column x
+              const int x = (int)(s0 / p.H);
+              int y0 = (int)(s0 - (long long)x * p.H);
+              if (p.direction == GTR_B2T) y0 = p.H - 64 - y0;
+              tma_load_5d(sb, &fp.tq, &ms->full[st], 0, h, x, y0, b);
+              tma_load_5d(sb + kTile, &fp.tk, &ms->full[st], 0, h, x, y0, b);
+              tma_load_5d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, x, y0, b);
+              tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, x, y0, b);
+            }
+          }
         }
-        int ok = 0;
-        if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
-        asm volatile("bar.sync 4, 64;" ::: "memory");  // the row table is complete
-        if (*(volatile int*)&ms->abort) stop = true;
-        if (stop) break;
-        const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int row = 8 * it + rq;
-          const int cell = rows[row];
-          const uint32_t nb = cell >= 0 ? 16u : 0u;
-          const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
-          const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
-          cp_async16(dst, gq + src, nb);
-          cp_async16(dst + kTile, gk + src, nb);
-          cp_async16(dst + 2 * kTile, gv + src, nb);
-        }
-#pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const int row = 4 * it + rg;
-          const int cell = rows[row];
-          const uint32_t nb = cell >= 0 ? 16u : 0u;
-          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
-                     gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
-        }
-        cp_async_arrive_noinc(&ms->full[st]);
       }
+    } else {
+      // Per chunk, thread t first resolves the grid cell of scan position c*64 + t (the
+      // direction remap) into a shared table; then the 64 threads copy the tiles with
+      // whole 128-byte rows per group of 8 threads (Q, K, V: placed in the 128-byte-swizzle
+      // layout) and 256-byte gate rows per group of 16, so each warp-wide copy touches
+      // only 4 (2) full lines.  Rows past the sequence end are zero-filled (source size 0).
+      const uint8_t* gq = reinterpret_cast<const uint8_t*>(p.q);
+      const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.k);
+      const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.v);
+      const uint8_t* gg = reinterpret_cast<const uint8_t*>(p.log_gamma);
+      const int j8 = pt & 7, rq = pt >> 3;     // 16-byte column, row within a group of 8
+      const int j16 = pt & 15, rg = pt >> 4;   // gate rows: 16-byte column, row within 4
+      const int srow = fp.rev ? 63 - pt : pt;  // staged row of scan position c*64 + pt
+      for (int r = 0; r < rounds && !stop; ++r) {
+        const Span sp = round_span(fp, r, seg);
+        for (int c = sp.c0; c < sp.c1; ++c, ++n) {
+          const int st = n % kStages;
+          int* rows = ms->rowoff[n & 1];
+          {
+            const long long s = (long long)c * kChunk + pt;
+            rows[srow] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
+          }
+          int ok = 0;
+          if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
+          if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
+          asm volatile("bar.sync 4, 64;" ::: "memory");  // the row table is complete
+          if (*(volatile int*)&ms->abort) stop = true;
+          if (stop) break;
+          const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = 8 * it + rq;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
+            const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
+            cp_async16(dst, gq + src, nb);
+            cp_async16(dst + kTile, gk + src, nb);
+            cp_async16(dst + 2 * kTile, gv + src, nb);
+          }
+#pragma unroll
+          for (int it = 0; it < 16; ++it) {
+            const int row = 4 * it + rg;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
+                       gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
+          }
+          cp_async_arrive_noinc(&ms->full[st]);
+        }
+      }
+      // copies already issued must land before this CTA's shared memory is released
+      asm volatile("cp.async.wait_all;" ::: "memory");
     }
-    // copies already issued must land before this CTA's shared memory is released
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ===================================================================== MMA issuer
     // Event-driven over the CTA's chunk sequence: whichever of stage 1 (scores, U'),
@@ -561,6 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = 0, wtid = tid;
     const int cc = wtid & 7;   // channels 8cc .. 8cc+7
     const int rb = wtid >> 3;  // rows 4rb .. 4rb+3
+    const bool rev = fp.rev != 0;
     float a2seg[8];            // log2 decay from the segment start, per channel (HOLD)
     int slot = 0, n = 0;
     bool alive = true;
@@ -579,32 +631,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* sb = smem + kOffStage + st * kStageBytes;
         float* G = reinterpret_cast<float*>(sb + 3 * kTile);
-        // ---- in-chunk cumulative log2-gates: my 4 rows, then a scan over the 16 row blocks
+        // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, then a scan over the
+        // 16 row blocks (staged rows run backwards in scan order when the chunk is reversed)
         float A[4][8];
         float run[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) run[e] = 0.f;
+        {
+          float gv[4][8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4* gp = reinterpret_cast<const float4*>(G + (4 * rb + i) * 64 + 8 * cc);
-          const float4 g0 = gp[0], g1 = gp[1];
-          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          for (int i = 0; i < 4; ++i) {
+            const float4* gp = reinterpret_cast<const float4*>(G + (4 * rb + i) * 64 + 8 * cc);
+            const float4 g0 = gp[0], g1 = gp[1];
+            gv[i][0] = g0.x; gv[i][1] = g0.y; gv[i][2] = g0.z; gv[i][3] = g0.w;
+            gv[i][4] = g1.x; gv[i][5] = g1.y; gv[i][6] = g1.z; gv[i][7] = g1.w;
+          }
+          if (!rev) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            run[e] = fmaf(gv[e], kLog2e, run[e]);
-            A[i][e] = run[e];
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                run[e] = fmaf(gv[i][e], kLog2e, run[e]);
+                A[i][e] = run[e];
+              }
+          } else {
+#pragma unroll
+            for (int i = 3; i >= 0; --i)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                run[e] = fmaf(gv[i][e], kLog2e, run[e]);
+                A[i][e] = run[e];
+              }
           }
         }
         float incl[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           incl[e] = run[e];
-          float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
-          if (lane >= 8) incl[e] += x;
-          x = __shfl_up_sync(0xffffffffu, incl[e], 16);
-          if (lane >= 16) incl[e] += x;
+          if (!rev) {
+            float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
+            if (lane >= 8) incl[e] += x;
+            x = __shfl_up_sync(0xffffffffu, incl[e], 16);
+            if (lane >= 16) incl[e] += x;
+          } else {
+            float x = __shfl_down_sync(0xffffffffu, incl[e], 8);
+            if (lane < 24) incl[e] += x;
+            x = __shfl_down_sync(0xffffffffu, incl[e], 16);
+            if (lane < 16) incl[e] += x;
+          }
         }
-        if (lane >= 24) {
+        if (rev ? lane < 8 : lane >= 24) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) ms->red[warp][8 * cc + e] = incl[e];
         }
@@ -622,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if (w < warp) off[e] += t[e];
+            if (rev ? w > warp : w < warp) off[e] += t[e];
             last[e] += t[e];
           }
         }
@@ -655,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int i = r0 + 8 * ((x & 3) >> 1);
             const int j = 8 * (x >> 2) + cq + (x & 1);
             float acc = 0.f;
-            if (j <= i) {
+            if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
               for (int k = 0; k < 64; k += 2) {
                 const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
                 const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
@@ -743,6 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = 1, wtid = tid - kWG, wq = warp & 3;
     const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
+    const bool rev = fp.rev != 0;
     float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
     float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
     int slot = 0, n = 0;
@@ -826,14 +903,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cb = 0; cb < 8; ++cb) {
           float x0 = sc[4 * cb], x1 = sc[4 * cb + 1], x2 = sc[4 * cb + 2], x3 = sc[4 * cb + 3];
-          if (cb > 2 * wq + 1) {
-            x0 = x1 = x2 = x3 = 0.f;
-          } else if (cb >= 2 * wq) {
+          if (rev ? cb < 2 * wq : cb > 2 * wq + 1) {
+            x0 = x1 = x2 = x3 = 0.f;  // scan(j) > scan(i) for the whole block
+          } else if (cb >= 2 * wq && cb <= 2 * wq + 1) {
             const int j = 8 * cb + cq;
-            x0 = (j <= r0) ? x0 : 0.f;
-            x1 = (j + 1 <= r0) ? x1 : 0.f;
-            x2 = (j <= r1) ? x2 : 0.f;
-            x3 = (j + 1 <= r1) ? x3 : 0.f;
+            if (!rev) {
+              x0 = (j <= r0) ? x0 : 0.f;
+              x1 = (j + 1 <= r0) ? x1 : 0.f;
+              x2 = (j <= r1) ? x2 : 0.f;
+              x3 = (j + 1 <= r1) ? x3 : 0.f;
+            } else {
+              x0 = (j >= r0) ? x0 : 0.f;
+              x1 = (j + 1 >= r0) ? x1 : 0.f;
+              x2 = (j >= r1) ? x2 : 0.f;
+              x3 = (j + 1 >= r1) ? x3 : 0.f;
+            }
           }
           pw[2 * cb] = pack_h2(x0, x1);
           pw[2 * cb + 1] = pack_h2(x2, x3);
@@ -871,7 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int trow = wq * 16 + (lane & 15);
     const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-    constexpr int kWarpStage = 2 * 32 * 32 * (int)sizeof(Tout);  // two half-row tiles per warp
+    constexpr int kWarpStage = 32 * 32 * (int)sizeof(Tout);  // one half-row tile per warp
     static_assert(4 * kWarpStage <= kHeldPerSet * kTile, "output staging fits a held set");
     int slot = 0;
     if (!hold) {
@@ -881,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int pr = 0; pr < pairs; ++pr) {
         if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) break;
         tc_fence_after();
-        const long long s = (long long)(2 * pr + tsel) * kChunk + trow;
+        const long long s = (long long)(2 * pr + tsel) * kChunk + (fp.rev ? 63 - trow : trow);
         epilogue_warp<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(pr & 1), 2 * pr + tsel < fp.Nc && s < L, s, wstage,
                             lane, nonfinite);
         tc_fence_before();
@@ -1022,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* wstage = smem + kOffHeld + sig * kHeldPerSet * kTile + wq * kWarpStage;
         for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
           const int gi = 2 * m2 + tsel;
-          const long long s = (long long)(sp.c0 + gi) * kChunk + trow;
+          const long long s = (long long)(sp.c0 + gi) * kChunk + (fp.rev ? 63 - trow : trow);
           epilogue_warp<Tout>(p, b, h, tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, gi < G && s < L, s, wstage,
                               lane, nonfinite);
         }
@@ -1053,6 +1137,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Tensor map over a [B][H][W][heads][64] tensor (row-major grid cells m = y*W + x) whose
+// box is 64 consecutive scan positions of one (batch, head): the row view [B][L][heads][64]
+// with a box of 64 cells m, or the column view with a box of 64 rows y of one column x.
+bool make_chunk_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, const Problem& p,
+                    bool column, bool swizzle) {
+  auto enc = get_encode();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
+  const cuuint64_t e = (cuuint64_t)esize, hd = (cuuint64_t)p.heads;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r;
+  if (!column) {
+    cuuint64_t dims[4] = {64, hd, (cuuint64_t)p.L(), (cuuint64_t)p.B};
+    cuuint64_t strides[3] = {64 * e, hd * 64 * e, (cuuint64_t)p.L() * hd * 64 * e};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    r = enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    cuuint64_t dims[5] = {64, hd, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)p.B};
+    cuuint64_t strides[4] = {64 * e, hd * 64 * e, (cuuint64_t)p.W * hd * 64 * e,
+                             (cuuint64_t)p.H * p.W * hd * 64 * e};
+    cuuint32_t box[5] = {64, 1, 1, 64, 1};
+    r = enc(m, dt, 5, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS;
+}
+
 struct Plan {
   int mode, n_seq, n_s, rounds, grid;
 };
@@ -1133,6 +1258,22 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the
   // fp16 rounding of the small Qh values keep their precision
   fp.max_exp2 = 11.5f;
+  // chunks are staged in reverse scan order for the reversed directions; a chunk is one
+  // TMA box per tensor when its 64 scan positions are consecutive cells of one row view
+  // (left-to-right always; right-to-left when rows hold whole chunks) or of one column
+  // (top-to-bottom / bottom-to-top when columns hold whole chunks)
+  fp.rev = (p.direction == GTR_R2L || p.direction == GTR_B2T) ? 1 : 0;
+  const bool column = p.direction >= GTR_T2B;
+  const bool one_box = p.direction == GTR_L2R || (p.direction == GTR_R2L && p.W % 64 == 0) ||
+                       (column && p.H % 64 == 0);
+  const CUtensorMapDataType dt16 =
+      std::is_same<Tin, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  fp.tma = one_box && make_chunk_map(&fp.tq, p.q, dt16, 2, p, column, true) &&
+                   make_chunk_map(&fp.tk, p.k, dt16, 2, p, column, true) &&
+                   make_chunk_map(&fp.tv, p.v, dt16, 2, p, column, true) &&
+                   make_chunk_map(&fp.tg, p.log_gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, column, false)
+               ? 1
+               : 0;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
