@@ -29,7 +29,7 @@
 // epilogue overlap round r+1's chunks (two held sets).
 //
 // Warp roles (480 threads):
-//   warps 0-3   WG_A  cumulative gates, Qh / Kh in place, held tiles, CUDA-core scores
+//   warps 0-3   WG_A  cumulative gates, Qh / Kh in place, CUDA-core scores
 //   warps 4-7   WG_B  score masking and fp32 state update (16-lane tensor-memory loads,
 //               so every lane of a warp does the same work)
 //   warps 8-11  WG_C  epilogue (both modes); HOLD round end: summary scan, correction
@@ -52,7 +52,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 3;          // staging depth (chunks in flight)
+constexpr int kStages = 4;          // staging depth (chunks in flight)
 constexpr int kHeldPerSet = 4;      // chunks held per CTA per round (HOLD)
 constexpr int kThreads = 480;
 constexpr int kProducerThreads = 64;
@@ -68,8 +68,8 @@ constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V,
 constexpr int kOffStage = 0;
 constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [2] chunk-start states
 constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
-constexpr int kOffHeld = kOffSst + kTile;                  // [2 sets][kHeldPerSet]
-constexpr int kOffMisc = kOffHeld + 2 * kHeldPerSet * kTile;
+constexpr int kOffStg = kOffSst + kTile;                   // output staging, 4 warps x 32 rows x 128 B
+constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
 constexpr int kMiscBytes = 1920;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 
@@ -79,8 +79,9 @@ constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0; masked fp16
 constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 output pairs; HOLD: [2 sets] x kSetCols
 constexpr uint32_t kLaneTile1 = 16u << 16;
 constexpr uint32_t kSetCols = 64u * (kHeldPerSet / 2);
+constexpr uint32_t kColHQ = kColO + 2 * kSetCols;  // HOLD: [2 sets] x kSetCols/2 held fp16 Qh' (A operands)
 static_assert(kHeldPerSet % 2 == 0, "held chunks come in lane-tile pairs");
-static_assert(kColO + 2 * kSetCols <= kTmemCols, "tensor memory budget");
+static_assert(kColHQ + kSetCols <= kTmemCols, "tensor memory budget");
 
 // HOLD-mode counters sit at a fixed place right after the workspace header, whatever
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
@@ -110,7 +111,9 @@ static_assert(alignof(FusedParams) >= 64, "tensor maps need 64-byte alignment");
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
-  uint64_t opready[2], su_full[2], su_free[2], sready[2], pready[2], s_done[2];
+  // opready is per stage: the operand builder may run up to kStages chunks ahead of the
+  // MMA warp, so a two-deep ring could complete a phase twice before it is observed
+  uint64_t opready[kStages], su_full[2], su_free[2], sready[2], pready[2], s_done[2];
   uint64_t o_full[2], o_free[2];
   uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
   uint64_t mma_final;
@@ -371,10 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&ms->full[i], fp.tma ? 1 : kProducerThreads);
       mbar_init(&ms->empty[i], 1);
+      mbar_init(&ms->opready[i], 1);
       ms->fb[i] = 0;
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&ms->opready[i], 1);
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
       mbar_init(&ms->sready[i], 1);
@@ -571,7 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             prog = true;
           }
         }
-        if (n1 < total && mbar_test(&ms->opready[n1 & 1], ph_of(n1)) && mbar_test(&ms->su_free[n1 & 1], ph_free(n1))) {
+        if (n1 < total && mbar_test(&ms->opready[n1 % kStages], (uint32_t)(n1 / kStages) & 1u) &&
+            mbar_test(&ms->su_free[n1 & 1], ph_free(n1))) {
           // stage 1 of chunk n: scores = Qh Kh^T (tensor-core chunks), U' = Kh^T V
           const int n = n1, bb = n & 1, st = n % kStages;
           const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
@@ -613,17 +617,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cc = wtid & 7;   // channels 8cc .. 8cc+7
     const int rb = wtid >> 3;  // rows 4rb .. 4rb+3
     const bool rev = fp.rev != 0;
-    float a2seg[8];            // log2 decay from the segment start, per channel (HOLD)
     int slot = 0, n = 0;
     bool alive = true;
     for (int r = 0; r < rounds && alive; ++r) {
       const Span sp = round_span(fp, r, seg);
-      const int sig = r & 1;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a2seg[e] = 0.f;
-      if (hold && r >= 2 && sp.c1 > sp.c0 &&
-          !wg_wait(wg, wtid, &ms->set_free[sig], ph_free(r), ms, hdr, 0x300, slot)) { alive = false; break; }
-      for (int c = sp.c0, g = 0; c < sp.c1; ++c, ++n, ++g) {
+      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
         const int bb = n & 1, st = n % kStages;
         if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot)) {
           alive = false;
@@ -746,13 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           wg_sync(wg);  // every raw q / k read is done before the tiles are overwritten
         }
-        // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place;
-        // held Qh 2^(A_seg) (HOLD)
-        __half2 eseg[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) eseg[e2] = bits_h2(pack_h2(ex2(a2seg[2 * e2]), ex2(a2seg[2 * e2 + 1])));
+        // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
         const __half2 eighth = __float2half2_rn(0.125f);
-        uint8_t* held = smem + kOffHeld + (sig * kHeldPerSet + (g < kHeldPerSet ? g : 0)) * kTile;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = 4 * rb + i;
@@ -761,7 +754,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint4 kraw = *reinterpret_cast<const uint4*>(sb + kTile + off16);
           uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
           uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
-          uint32_t oh[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
@@ -778,11 +770,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             qw[e2] = h2_bits(qh);
             kw[e2] = h2_bits(kh);
-            oh[e2] = h2_bits(__hmul2(qh, eseg[e2]));
           }
           *reinterpret_cast<uint4*>(sb + off16) = qraw;
           *reinterpret_cast<uint4*>(sb + kTile + off16) = kraw;
-          if (hold) *reinterpret_cast<uint4*>(held + off16) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
         }
         if constexpr (!std::is_same<Tin, __half>::value) {
           // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
@@ -805,11 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           lw[1] = make_float4(last[4], last[5], last[6], last[7]);
         }
         if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a2seg[e] += last[e];
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->opready[bb]);
+        if (wtid == 0) mbar_arrive(&ms->opready[st]);
       }
     }
   } else if (warp < 8) {
@@ -822,6 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool rev = fp.rev != 0;
     float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
     float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
+    float a2c[16];         // log2 segment decay of channels 8c + cq (+1) (HOLD, held Qh')
     int slot = 0, n = 0;
     bool alive = true;
     for (int r = 0; r < rounds && alive; ++r) {
@@ -846,7 +835,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) a2c[e] = 0.f;
       a2r0 = a2r1 = 0.f;
+      // held Qh' of this round reuse the tensor-memory set of the round two back
+      if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
       {  // zero start state for this round's first chunk (its tile's last reader, the
          // O = Qh S of chunk n-2, must be done)
         if (n >= 2 && !wg_wait(wg, wtid, &ms->s_done[n & 1], ph_of(n - 2), ms, hdr, 0x403, slot)) break;
@@ -866,15 +859,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* alast = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes + 3 * kTile);
         const float l0 = alast[r0], l1 = alast[r1];
         const float dl0 = ex2(l0), dl1 = ex2(l1);
-        float sc[32], u[32];
-        tmem_ld16x256_x8(tl + kColSU + 64u * bb, sc);
-        tmem_ld16x256_x8(tl + kColSU + 64u * bb + kLaneTile1, u);
-        tmem_wait_ld();
-        // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
+        {
+          float u[32];
+          tmem_ld16x256_x8(tl + kColSU + 64u * bb + kLaneTile1, u);
+          tmem_wait_ld();
+          // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float d = (x & 2) ? dl1 : dl0;
-          Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
+          for (int x = 0; x < 32; ++x) {
+            const float d = (x & 2) ? dl1 : dl0;
+            Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
+          }
         }
         a2r0 += l0;
         a2r1 += l1;
@@ -894,15 +888,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_smem();
         }
+        if (hold) {
+          // held Qh' = Qh 2^(A from the segment start) of this chunk -> tensor memory, in the
+          // lane tile of its held output (16x128b: register 2c+q is row r0 + 8q, channels
+          // 8c + cq, 8c + cq + 1)
+          const int g = c - sp.c0;
+          const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
+          const float* a_ch = reinterpret_cast<const float*>(qt + 3 * kTile);  // a per channel (row 0)
+          uint32_t hw[16];
+#pragma unroll
+          for (int cb = 0; cb < 8; ++cb) {
+            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
+            const __half2 e2 = __floats2half2_rn(ex2(a2c[2 * cb]), ex2(a2c[2 * cb + 1]));
+            hw[2 * cb] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
+            hw[2 * cb + 1] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
+            const float2 ac = *reinterpret_cast<const float2*>(a_ch + 8 * cb + cq);
+            a2c[2 * cb] += ac.x;
+            a2c[2 * cb + 1] += ac.y;
+          }
+          tmem_st16x128_x8(tl + kColHQ + (kSetCols / 2) * (uint32_t)(r & 1) + 32u * (uint32_t)(g >> 1) +
+                               ((g & 1) ? kLaneTile1 : 0u),
+                           hw);
+        }
         // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
         // the A operand of P V.  A rows are read from the lanes of the output rows, so P
         // goes to the lane tile of the chunk's output region (tile 1: over U', already
         // loaded).  Register 2c+q of the 16x128b shape is row r0 + 8q, column 4c + lane%4,
         // i.e. the score pair (8c + cq, 8c + cq + 1) of that row.
-        uint32_t pw[16];
+        const uint32_t pdst = tl + kColSU + 64u * bb + (((hold ? (c - sp.c0) : n) & 1) ? kLaneTile1 : 0u);
 #pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-          float x0 = sc[4 * cb], x1 = sc[4 * cb + 1], x2 = sc[4 * cb + 2], x3 = sc[4 * cb + 3];
+        for (int hf = 0; hf < 2; ++hf) {  // score columns 32hf .. 32hf+31 -> P columns 16hf .. 16hf+15
+        float sc[16];
+        tmem_ld16x256_x4(tl + kColSU + 64u * bb + 32u * hf, sc);
+        tmem_wait_ld();
+        uint32_t pw[8];
+#pragma unroll
+        for (int cl = 0; cl < 4; ++cl) {
+          const int cb = 4 * hf + cl;
+          float x0 = sc[4 * cl], x1 = sc[4 * cl + 1], x2 = sc[4 * cl + 2], x3 = sc[4 * cl + 3];
           if (rev ? cb < 2 * wq : cb > 2 * wq + 1) {
             x0 = x1 = x2 = x3 = 0.f;  // scan(j) > scan(i) for the whole block
           } else if (cb >= 2 * wq && cb <= 2 * wq + 1) {
@@ -919,11 +942,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               x3 = (j + 1 >= r1) ? x3 : 0.f;
             }
           }
-          pw[2 * cb] = pack_h2(x0, x1);
-          pw[2 * cb + 1] = pack_h2(x2, x3);
+          pw[2 * cl] = pack_h2(x0, x1);
+          pw[2 * cl + 1] = pack_h2(x2, x3);
         }
-        const bool otile = hold ? ((c - sp.c0) & 1) != 0 : (n & 1) != 0;
-        tmem_st16x128_x8(tl + kColSU + 64u * bb + (otile ? kLaneTile1 : 0u), pw);
+        tmem_st16x128_x4(pdst + 16u * hf, pw);
+        }
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);
@@ -955,12 +978,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int trow = wq * 16 + (lane & 15);
     const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-    constexpr int kWarpStage = 32 * 32 * (int)sizeof(Tout);  // one half-row tile per warp
-    static_assert(4 * kWarpStage <= kHeldPerSet * kTile, "output staging fits a held set");
+    uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
     if (!hold) {
-      // output staging: the held-tile area, unused in this mode
-      uint8_t* wstage = smem + kOffHeld + wq * kWarpStage;
       const int pairs = (fp.Nc + 1) / 2;
       for (int pr = 0; pr < pairs; ++pr) {
         if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) break;
@@ -1091,9 +1111,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             for (int g = 0; g < G; ++g) {
               const uint32_t d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
-              const uint32_t a_h = s_base + kOffHeld + (sig * kHeldPerSet + g) * kTile;
+              const uint32_t a_h = tmem + kColHQ + (kSetCols / 2) * sig + 32u * (uint32_t)(g >> 1) +
+                                   ((g & 1) ? kLaneTile1 : 0u);  // held Qh', same lanes as the output
               for (int k = 0; k < 4; ++k)
-                mma_f16(d_o, sw128_desc(a_h + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
+                mma_f16_ta(d_o, a_h + 8 * k, sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
             }
             mma_commit(&ms->corr_done[sig]);
           }
@@ -1102,8 +1123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_wait(wg, wtid, &ms->corr_done[sig], ph_of(r), ms, hdr, 0x603, slot)) break;
         tc_fence_after();
         // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane
-        // tile 1); the set's Qh tiles, consumed by the correction, stage the rows
-        uint8_t* wstage = smem + kOffHeld + sig * kHeldPerSet * kTile + wq * kWarpStage;
+        // tile 1)
         for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
           const int gi = 2 * m2 + tsel;
           const long long s = (long long)(sp.c0 + gi) * kChunk + (fp.rev ? 63 - trow : trow);

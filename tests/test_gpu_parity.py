@@ -272,3 +272,24 @@ def test_paths_interleaved_on_the_shared_workspace():
         assert rel_err(o_s, ref_s) <= 1e-5
         assert rel_err(o_f, ref_f) <= 1e-2
     assert gtr.read_error() == 0
+
+
+@pytest.mark.parametrize("name", ["640", "1024", "2048", "stack"])
+def test_back_to_back_calls_leave_no_device_error(name):
+    """Many back-to-back fused calls in every direction: every bounded wait inside the
+    kernel must be met (a barrier phase that is signalled twice before it is observed
+    would surface as GTR_ERR_TIMEOUT), and the last output still matches the oracle."""
+    w = WORKLOADS[name]
+    q, k, v, lg = make_inputs(w, 81)
+    dev = torch.device("cuda:0")
+    tq, tk, tv, tg = (t.to(dev) for t in (q, k, v, lg))
+    in_dtype = {"f16": gtr.F16, "bf16": gtr.BF16}[w.dtype]
+    for d in range(4):
+        ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, in_dtype=in_dtype, path="fused", device=dev)
+        out = gtr.gla_fwd(tq, tk, tv, tg, grid=(w.H, w.W), direction=d, path="fused", workspace=ws)
+        for _ in range(40):
+            gtr.gla_fwd(tq, tk, tv, tg, grid=(w.H, w.W), direction=d, path="fused", workspace=ws, out=out)
+        torch.cuda.synchronize()
+        assert gtr.read_error(ws) == 0, f"{name} dir={d}: device error after back-to-back calls"
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 3)
+    assert rel_err(out, ref) <= TOL[w.dtype]
