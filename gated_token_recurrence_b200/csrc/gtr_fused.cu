@@ -28,14 +28,15 @@
 // times its segment-start state to the held outputs.  Round r's scan and
 // epilogue overlap round r+1's chunks (two held sets).
 //
-// Warp roles (480 threads):
-//   warps 0-3   WG_A  cumulative gates, Qh / Kh in place, CUDA-core scores
-//   warps 4-7   WG_B  score masking and fp32 state update (16-lane tensor-memory loads,
-//               so every lane of a warp does the same work)
-//   warps 8-11  WG_C  epilogue (both modes); HOLD round end: summary scan, correction
-//   warps 12-13 producer: cp.async of one token row per thread (direction remap,
+// Warp roles (608 threads):
+//   warps 0-7   WG_A  two warpgroups, one per half of the key channels: cumulative
+//               gates, Qh / Kh in place, CUDA-core scores
+//   warps 8-11  WG_B  score masking, fp32 state update, held Qh' (16-lane tensor-memory
+//               loads, so every lane of a warp does the same work)
+//   warps 12-15 WG_C  epilogue (both modes); HOLD round end: summary scan, correction
+//   warps 16-17 producer: TMA boxes, or cp.async row copies (direction remap,
 //               128-byte-swizzled placement, zero fill past the sequence end)
-//   warp 14     tcgen05 MMA issuer and tensor-memory owner
+//   warp 18     tcgen05 MMA issuer and tensor-memory owner
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,9 +55,9 @@ using namespace sm100;
 
 constexpr int kStages = 4;          // staging depth (chunks in flight)
 constexpr int kHeldPerSet = 4;      // chunks held per CTA per round (HOLD)
-constexpr int kThreads = 480;
+constexpr int kThreads = 608;
 constexpr int kProducerThreads = 64;
-constexpr int kMmaWarp = 14;
+constexpr int kMmaWarp = 18;
 constexpr int kWG = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,8 +67,8 @@ constexpr int kTile = 8192;
 constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
 constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V, G
 constexpr int kOffStage = 0;
-constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [2] chunk-start states
-constexpr int kOffSst = kOffS + 2 * kTile;                 // segment start state
+constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [3] chunk-start states
+constexpr int kOffSst = kOffS + 3 * kTile;                 // segment start state
 constexpr int kOffStg = kOffSst + kTile;                   // output staging, 4 warps x 32 rows x 128 B
 constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
 constexpr int kMiscBytes = 1920;
@@ -87,7 +88,7 @@ static_assert(kColHQ + kSetCols <= kTmemCols, "tensor memory budget");
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
 constexpr size_t kMaxHoldSegments = 256;  // CTAs of one launch in HOLD mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxHoldSegments * sizeof(unsigned int);
-constexpr int kScanBlock = 12;           // segments one WG_C thread composes in registers
+constexpr int kScanBlock = 8;            // segments one WG_C thread composes in registers
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 struct FusedParams {
@@ -113,15 +114,16 @@ struct Misc {
   uint64_t full[kStages], empty[kStages];
   // opready is per stage: the operand builder may run up to kStages chunks ahead of the
   // MMA warp, so a two-deep ring could complete a phase twice before it is observed
-  uint64_t opready[kStages], su_full[2], su_free[2], sready[2], pready[2], s_done[2];
+  uint64_t opready[kStages], su_full[2], su_free[2], sready[3], pready[2];
   uint64_t o_full[2], o_free[2];
   uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort;
-  int go[3][2];          // per-warpgroup wait decisions, alternating slots
+  int go[4][2];          // per-warpgroup wait decisions, alternating slots
+  int fbh[2][2];         // chunk parity x channel half -> CUDA-core scores needed
   int fb[kStages];       // stage -> scores from the CUDA cores
-  alignas(16) float red[4][64];   // WG_A cumsum: per-warp channel totals
+  alignas(16) float red[2][4][32];  // WG_A cumsum: per channel half and warp, channel totals
   int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
 };
 // The in-chunk log2 decay per channel (a) of a staged chunk is kept in row 0 of its
@@ -173,7 +175,6 @@ __device__ bool wait_counter(const unsigned int* ctr, unsigned int target, Misc*
       *(volatile int*)&ms->abort = 1;
       return false;
     }
-    __nanosleep(64);
   }
 }
 
@@ -374,15 +375,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&ms->full[i], fp.tma ? 1 : kProducerThreads);
       mbar_init(&ms->empty[i], 1);
-      mbar_init(&ms->opready[i], 1);
+      mbar_init(&ms->opready[i], 2);  // one arrival per channel half
       ms->fb[i] = 0;
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
-      mbar_init(&ms->sready[i], 1);
       mbar_init(&ms->pready[i], 1);
-      mbar_init(&ms->s_done[i], 1);
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
       mbar_init(&ms->agg_pub[i], 1);
@@ -391,8 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->set_free[i], 1);
     }
     mbar_init(&ms->mma_final, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&ms->sready[i], 1);
     ms->abort = 0;
-    for (int i = 0; i < 3; ++i) ms->go[i][0] = ms->go[i][1] = 0;
+    for (int i = 0; i < 4; ++i) ms->go[i][0] = ms->go[i][1] = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -404,11 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
 
-  if (warp == 12 || warp == 13) {
+  if (warp == 16 || warp == 17) {
     // ===================================================================== producer
     // Staged chunk row r holds scan position c*64 + r, or c*64 + 63 - r for the reversed
     // directions (right-to-left, bottom-to-top), where a chunk is stored in memory order.
-    const int pt = tid - 12 * 32;  // 0..63
+    const int pt = tid - 16 * 32;  // 0..63
     int n = 0;
     bool stop = false;
     if (fp.tma) {
@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int ok = 0;
           if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
           if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
-          asm volatile("bar.sync 4, 64;" ::: "memory");  // the row table is complete
+          asm volatile("bar.sync 5, 64;" ::: "memory");  // the row table is complete
           if (*(volatile int*)&ms->abort) stop = true;
           if (stop) break;
           const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
@@ -554,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n2a < n1) {
           // stage 2a of chunk m: O = Qh S (S = the chunk-start state tile)
           const int m = n2a, bb = m & 1, st = m % kStages;
-          bool rdy = mbar_test(&ms->sready[bb], ph_of(m));
+          bool rdy = mbar_test(&ms->sready[m % 3], (uint32_t)(m / 3) & 1u);
           if (hold) {
             // a held set is reused: the epilogue of the round two back must be finished
             if (za.g == 0 && za.r >= 2) rdy = rdy && mbar_test(&ms->set_free[za.r & 1], ph_free(za.r));
@@ -563,12 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (rdy) {
             const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
-            const uint32_t a_s = s_base + kOffS + bb * kTile;
+            const uint32_t a_s = s_base + kOffS + (m % 3) * kTile;
             const uint32_t d_o = out_region(za, m);
             tc_fence_after();
             for (int k = 0; k < 4; ++k)
               mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-            mma_commit(&ms->s_done[bb]);
             za.advance(fp, seg, rounds);
             ++n2a;
             prog = true;
@@ -602,7 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             *(volatile int*)&ms->abort = 1;
             break;
           }
-          __nanosleep(32);
+          // sleep in hardware on the oldest pending step's barrier (woken when it
+          // completes, at most half a microsecond); the loop then re-polls every step
+          if (n2b < n2a)
+            (void)mbar_wait_sleep(&ms->pready[n2b & 1], ph_of(n2b), 500u);
+          else if (n2a < n1)
+            (void)mbar_wait_sleep(&ms->sready[n2a % 3], (uint32_t)(n2a / 3) & 1u, 500u);
+          else
+            (void)mbar_wait_sleep(&ms->opready[n1 % kStages], (uint32_t)(n1 / kStages) & 1u, 500u);
         }
       }
       // every MMA issued here has completed before tensor memory is freed
@@ -611,16 +617,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!mbar_try_wait(&ms->mma_final, 0) && globaltimer() - t0 < 1000000000ull) {
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ===================================================================== WG_A: operand tiles
-    const int wg = 0, wtid = tid;
-    const int cc = wtid & 7;   // channels 8cc .. 8cc+7
-    const int rb = wtid >> 3;  // rows 4rb .. 4rb+3
+    // Two warpgroups share every chunk: warpgroup hh takes channels 32hh .. 32hh+31, its
+    // warp w4 the rows 16w4 .. 16w4+15, a thread 4 rows x 4 channels.
+    const int hh = warp >> 2, w4 = warp & 3;
+    const int wg = hh, wtid = tid - kWG * hh;
+    const int cc = lane & 7;                  // channels ch0 .. ch0+3
+    const int ch0 = 32 * hh + 4 * cc;
+    const int row0 = 16 * w4 + 4 * (lane >> 3);  // rows row0 .. row0+3
     const bool rev = fp.rev != 0;
     int slot = 0, n = 0;
     bool alive = true;
     for (int r = 0; r < rounds && alive; ++r) {
       const Span sp = round_span(fp, r, seg);
+      float a2s[4] = {0.f, 0.f, 0.f, 0.f};  // log2 decay from the segment start, channels ch0..ch0+3
       for (int c = sp.c0; c < sp.c1; ++c, ++n) {
         const int bb = n & 1, st = n % kStages;
         if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot)) {
@@ -629,26 +640,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* sb = smem + kOffStage + st * kStageBytes;
         float* G = reinterpret_cast<float*>(sb + 3 * kTile);
-        // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, then a scan over the
-        // 16 row blocks (staged rows run backwards in scan order when the chunk is reversed)
-        float A[4][8];
-        float run[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) run[e] = 0.f;
+        // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, a scan over the
+        // warp's 4 row blocks, then over the 4 warps (staged rows run backwards in scan
+        // order when the chunk is reversed)
+        float A[4][4];
+        float run[4] = {0.f, 0.f, 0.f, 0.f};
         {
-          float gv[4][8];
+          float gv[4][4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float4* gp = reinterpret_cast<const float4*>(G + (4 * rb + i) * 64 + 8 * cc);
-            const float4 g0 = gp[0], g1 = gp[1];
-            gv[i][0] = g0.x; gv[i][1] = g0.y; gv[i][2] = g0.z; gv[i][3] = g0.w;
-            gv[i][4] = g1.x; gv[i][5] = g1.y; gv[i][6] = g1.z; gv[i][7] = g1.w;
+            const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * 64 + ch0);
+            gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
           }
           if (!rev) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 4; ++e) {
                 run[e] = fmaf(gv[i][e], kLog2e, run[e]);
                 A[i][e] = run[e];
               }
@@ -656,15 +664,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 3; i >= 0; --i)
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 4; ++e) {
                 run[e] = fmaf(gv[i][e], kLog2e, run[e]);
                 A[i][e] = run[e];
               }
           }
         }
-        float incl[8];
+        float incl[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           incl[e] = run[e];
           if (!rev) {
             float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
@@ -678,56 +686,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane < 16) incl[e] += x;
           }
         }
-        if (rev ? lane < 8 : lane >= 24) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ms->red[warp][8 * cc + e] = incl[e];
-        }
+        float* redh = &ms->red[hh][0][0];  // [4 warps][32 channels] of this channel half
+        if (rev ? lane < 8 : lane >= 24)
+          *reinterpret_cast<float4*>(redh + w4 * 32 + 4 * cc) = make_float4(incl[0], incl[1], incl[2], incl[3]);
         wg_sync(wg);
-        float off[8], last[8];
+        float off[4], last[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           off[e] = incl[e] - run[e];
           last[e] = 0.f;
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const float4 t0 = *reinterpret_cast<const float4*>(&ms->red[w][8 * cc]);
-          const float4 t1 = *reinterpret_cast<const float4*>(&ms->red[w][8 * cc + 4]);
-          const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          const float4 t4 = *reinterpret_cast<const float4*>(redh + w * 32 + 4 * cc);
+          const float t[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (rev ? w > warp : w < warp) off[e] += t[e];
+          for (int e = 0; e < 4; ++e) {
+            if (rev ? w > w4 : w < w4) off[e] += t[e];
             last[e] += t[e];
           }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) A[i][e] += off[e];
+          for (int e = 0; e < 4; ++e) A[i][e] += off[e];
+        // CUDA-core decision over all 64 channels: each warp covers its half's 32 channels,
+        // the two halves meet at a 256-thread barrier
         bool exp_unsafe = false;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < 4; ++e)
           if (-last[e] > fp.max_exp2) exp_unsafe = true;
-        // every warp holds all 64 channels (lanes cover cc = 0..7), so this vote is the
-        // same in all four warps
-        const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
+        const bool half_unsafe = __any_sync(0xffffffffu, exp_unsafe);
+        if (wtid == 0) ms->fbh[bb][hh] = half_unsafe ? 1 : 0;
+        asm volatile("bar.sync 6, 256;" ::: "memory");
+        const bool fbx = (*(volatile int*)&ms->fbh[bb][0] | *(volatile int*)&ms->fbh[bb][1]) != 0;
         if (fbx) {
-          // ---- CUDA-core scores for this chunk, straight into tensor memory (lane tile 0
-          // of the chunk's score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk), j <= i.
-          // A goes to the gate tile so every thread can read every row.
+          // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
+          // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i);
+          // warpgroup hh fills score columns 32hh .. 32hh+31 of its warps' rows.  A goes to
+          // the gate tile so that every thread can read every row and channel.
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float4* gw = reinterpret_cast<float4*>(G + (4 * rb + i) * 64 + 8 * cc);
-            gw[0] = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
-            gw[1] = make_float4(A[i][4], A[i][5], A[i][6], A[i][7]);
-          }
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
           if (!wg_wait(wg, wtid, &ms->su_free[bb], ph_free(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+          asm volatile("bar.sync 6, 256;" ::: "memory");  // A of both channel halves is in place
           tc_fence_after();
-          const int r0 = 16 * warp + (lane >> 2), cq = 2 * (lane & 3);
-          float sv[32];
-          for (int x = 0; x < 32; ++x) {
+          const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
+          float sv[16];
+          for (int x = 0; x < 16; ++x) {
             const int i = r0 + 8 * ((x & 3) >> 1);
-            const int j = 8 * (x >> 2) + cq + (x & 1);
+            const int j = 32 * hh + 8 * (x >> 2) + cq + (x & 1);
             float acc = 0.f;
             if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
               for (int k = 0; k < 64; k += 2) {
@@ -739,23 +747,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             sv[x] = acc * 0.125f;
           }
-          tmem_st16x256_x8(tmem + ((uint32_t)(32 * warp) << 16) + kColSU + 64u * bb, sv);
+          tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * bb + 32u * hh, sv);
           tmem_wait_st();
           tc_fence_before();
-          wg_sync(wg);  // every raw q / k read is done before the tiles are overwritten
+          asm volatile("bar.sync 6, 256;" ::: "memory");  // raw q / k reads done before the overwrite
         }
         // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
         const __half2 eighth = __float2half2_rn(0.125f);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int row = 4 * rb + i;
-          const uint32_t off16 = row * 128u + (((uint32_t)cc ^ ((uint32_t)row & 7u)) << 4);
-          uint4 qraw = *reinterpret_cast<const uint4*>(sb + off16);
-          uint4 kraw = *reinterpret_cast<const uint4*>(sb + kTile + off16);
+          const int row = row0 + i;
+          // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
+          const uint32_t off8 = row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
+          uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
+          uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
           uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
           uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
+          for (int e2 = 0; e2 < 2; ++e2) {
             const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
             const float xk0 = fbx ? last[2 * e2] - A0 : -A0;
             const float xk1 = fbx ? last[2 * e2 + 1] - A1 : -A1;
@@ -771,14 +780,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             qw[e2] = h2_bits(qh);
             kw[e2] = h2_bits(kh);
           }
-          *reinterpret_cast<uint4*>(sb + off16) = qraw;
-          *reinterpret_cast<uint4*>(sb + kTile + off16) = kraw;
+          *reinterpret_cast<uint2*>(sb + off8) = qraw;
+          *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
         }
         if constexpr (!std::is_same<Tin, __half>::value) {
-          // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
+          // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range);
+          // the two warpgroups take alternate 16-byte chunks
           uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
 #pragma unroll
-          for (int i = wtid; i < kTile / 16; i += kWG) {
+          for (int i = tid; i < kTile / 16; i += 2 * kWG) {
             uint4 x = vt[i];
             uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
@@ -789,28 +799,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             vt[i] = x;
           }
         }
-        if (rb == 0) {  // every gate read of this chunk is behind a warpgroup barrier by now
-          float4* lw = reinterpret_cast<float4*>(G + 8 * cc);
-          lw[0] = make_float4(last[0], last[1], last[2], last[3]);
-          lw[1] = make_float4(last[4], last[5], last[6], last[7]);
+        if (w4 == 0 && lane < 8) {
+          // gate row 0 now holds the chunk's decay a per channel, row 1 the factor
+          // 2^(decay from the segment start to this chunk) of the held Qh'
+          *reinterpret_cast<float4*>(G + ch0) = make_float4(last[0], last[1], last[2], last[3]);
+          *reinterpret_cast<float4*>(G + 64 + ch0) = make_float4(ex2(a2s[0]), ex2(a2s[1]), ex2(a2s[2]), ex2(a2s[3]));
         }
-        if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a2s[e] += last[e];
+        if (tid == 0) ms->fb[st] = fbx ? 1 : 0;
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->opready[st]);
+        if (wtid == 0) mbar_arrive(&ms->opready[st]);  // one arrival per channel half
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ===================================================================== WG_B: masking, state
     // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
     // r0 + 8(q>>1), column 8c + cq + (q&1) of the warp's 16-row slice.
-    const int wg = 1, wtid = tid - kWG, wq = warp & 3;
+    const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
     const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
     const bool rev = fp.rev != 0;
     float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
     float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
-    float a2c[16];         // log2 segment decay of channels 8c + cq (+1) (HOLD, held Qh')
     int slot = 0, n = 0;
     bool alive = true;
     for (int r = 0; r < rounds && alive; ++r) {
@@ -835,20 +847,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) a2c[e] = 0.f;
       a2r0 = a2r1 = 0.f;
       // held Qh' of this round reuse the tensor-memory set of the round two back
       if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
       {  // zero start state for this round's first chunk (its tile's last reader, the
-         // O = Qh S of chunk n-2, must be done)
-        if (n >= 2 && !wg_wait(wg, wtid, &ms->s_done[n & 1], ph_of(n - 2), ms, hdr, 0x403, slot)) break;
+         // O = Qh S of chunk n-3, completed before chunk n-1's scores were issued)
         const uint4 z = make_uint4(0, 0, 0, 0);
-        uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n & 1) * kTile);
+        uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n % 3) * kTile);
         for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->sready[n & 1]);
+        if (wtid == 0) mbar_arrive(&ms->sready[n % 3]);
       }
       for (int c = sp.c0; c < sp.c1; ++c, ++n) {
         const int bb = n & 1, st = n % kStages;
@@ -872,39 +881,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         a2r0 += l0;
         a2r1 += l1;
-        if (!last_chunk) {
-          // the next chunk's start state; its tile was last read by O = Qh S of chunk n-1
-          if (n >= 1 && !wg_wait(wg, wtid, &ms->s_done[(n + 1) & 1], ph_of(n - 1), ms, hdr, 0x402, slot)) {
-            alive = false;
-            break;
-          }
-          uint8_t* srow0 = smem + kOffS + ((n + 1) & 1) * kTile + r0 * 128;
-          uint8_t* srow1 = srow0 + 8 * 128;
-#pragma unroll
-          for (int cb = 0; cb < 8; ++cb) {
-            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;
-            sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
-            sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
-          }
-          fence_proxy_async_smem();
-        }
         if (hold) {
+          // (read from the staged Qh before P is signalled: P V's completion frees the stage)
           // held Qh' = Qh 2^(A from the segment start) of this chunk -> tensor memory, in the
           // lane tile of its held output (16x128b: register 2c+q is row r0 + 8q, channels
           // 8c + cq, 8c + cq + 1)
           const int g = c - sp.c0;
           const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
-          const float* a_ch = reinterpret_cast<const float*>(qt + 3 * kTile);  // a per channel (row 0)
+          const float* eseg = reinterpret_cast<const float*>(qt + 3 * kTile) + 64;  // gate row 1
           uint32_t hw[16];
 #pragma unroll
           for (int cb = 0; cb < 8; ++cb) {
             const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
-            const __half2 e2 = __floats2half2_rn(ex2(a2c[2 * cb]), ex2(a2c[2 * cb + 1]));
+            const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
+            const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
             hw[2 * cb] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
             hw[2 * cb + 1] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
-            const float2 ac = *reinterpret_cast<const float2*>(a_ch + 8 * cb + cq);
-            a2c[2 * cb] += ac.x;
-            a2c[2 * cb + 1] += ac.y;
           }
           tmem_st16x128_x8(tl + kColHQ + (kSetCols / 2) * (uint32_t)(r & 1) + 32u * (uint32_t)(g >> 1) +
                                ((g & 1) ? kLaneTile1 : 0u),
@@ -950,10 +942,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);
-        if (wtid == 0) {
-          mbar_arrive(&ms->pready[bb]);
-          if (!last_chunk) mbar_arrive(&ms->sready[(n + 1) & 1]);
+        if (wtid == 0) mbar_arrive(&ms->pready[bb]);
+        if (!last_chunk) {
+          // the next chunk's start state (three tiles: the one written here was last read
+          // by O = Qh S of chunk n-2, complete since chunk n's scores were issued)
+          uint8_t* srow0 = smem + kOffS + ((n + 1) % 3) * kTile + r0 * 128;
+          uint8_t* srow1 = srow0 + 8 * 128;
+#pragma unroll
+          for (int cb = 0; cb < 8; ++cb) {
+            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;
+            sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
+            sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+          }
+          fence_proxy_async_smem();
         }
+        wg_sync(wg);
+        if (wtid == 0 && !last_chunk) mbar_arrive(&ms->sready[(n + 1) % 3]);
       }
       if (!alive) break;
       if (hold) {
@@ -972,9 +976,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
       }
     }
-  } else if (warp < 12) {
+  } else if (warp < 16) {
     // ===================================================================== WG_C: epilogue, HOLD round end
-    const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
+    const int wg = 3, wtid = tid - 3 * kWG, wq = warp & 3;
     const int trow = wq * 16 + (lane & 15);
     const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
