@@ -828,6 +828,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; r < rounds && alive; ++r) {
       const Span sp = round_span(fp, r, seg);
       float* mine = hold ? fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64) : nullptr;
+      // The summary slot and the held Qh' set of this round were used by the round two
+      // back: wait until that round's epilogue, which every CTA's scan of that round
+      // precedes, is finished -- also for a round without chunks, whose neutral summary
+      // would otherwise overwrite a slot other CTAs may still be scanning.
+      if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
       if (sp.c1 <= sp.c0) {
         if (hold) {  // an empty segment still publishes a neutral summary
 #pragma unroll
@@ -848,8 +853,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
       a2r0 = a2r1 = 0.f;
-      // held Qh' of this round reuse the tensor-memory set of the round two back
-      if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
       {  // zero start state for this round's first chunk (its tile's last reader, the
          // O = Qh S of chunk n-3, completed before chunk n-1's scores were issued)
         const uint4 z = make_uint4(0, 0, 0, 0);
