@@ -40,6 +40,40 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FLOPS_PER_TOKEN_HEAD = 24704  # chunkwise, causal: 4*dk*dv + (C+1)(dk+dv)
 
 
+KERNEL_SOURCES = ("gtr_fused.cu", "gtr_sm100.cuh", "gtr_common.cuh")
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "fused_gla_kernel_dram_traffic.md")
+
+
+def kernel_fingerprint() -> str:
+    """sha256 (first 16 hex digits) over the fused kernel's sources, in a fixed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "gated_token_recurrence_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch (read + write) that an ncu capture recorded for this workload
+    in profiles/fused_gla_kernel_dram_traffic.md -- only when the capture was taken on the
+    current kernel sources (same fingerprint); None otherwise."""
+    try:
+        with open(TRAFFIC_TABLE) as f:
+            lines = f.read().splitlines()
+    except OSError:
+        return None
+    fp = kernel_fingerprint()
+    for line in lines:
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == workload and cells[1] == fp:
+            try:
+                return int(cells[2]) + int(cells[3])
+            except ValueError:
+                return None
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -364,7 +398,8 @@ def run_ours(args):
                        "l2": f"inputs and outputs rotate over {len(sets)} buffer sets "
                              f"({len(sets) * w.algorithmic_bytes() / 2**20:.0f} MiB > L2)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / hbm, "traffic": measured_traffic(w.name) if path_name == "fused" else None,
+                         "peak_kind": peak_kind,
                          "kernel": f"gtr_gla_fwd call ({launches} launch"
                                    f"{'es' if launches != 1 else ''}, {path_name} path)",
                          "bytes_per_call": w.algorithmic_bytes(),
