@@ -41,6 +41,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 #include <type_traits>
 
@@ -71,7 +72,7 @@ constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [3] chunk-start st
 constexpr int kOffSst = kOffS + 3 * kTile;                 // segment start state
 constexpr int kOffStg = kOffSst + kTile;                   // output staging, 4 warps x 32 rows x 128 B
 constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
-constexpr int kMiscBytes = 1920;
+constexpr int kMiscBytes = 2048;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 
 // tensor memory columns
@@ -102,7 +103,9 @@ struct FusedParams {
   float* agg;              // [n_seq][2 round parities][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
   float* carry;            // [n_seq][64*64] state entering the current round, fp32
   uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
-  int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD
+  uint16_t* qhp;           // SEGMENTED: [n_seq][Nc][64*64] held Qh' per chunk, fp16, MMA layout
+  uint16_t* olc;           // SEGMENTED: [n_seq][Nc][64][64] outputs from a zero segment start, fp16
+  int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD, 2 = SEGMENTED
   int grid;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
   int tma;                 // 1: every chunk is one TMA box per tensor; 0: cp.async row copies
@@ -118,6 +121,7 @@ struct Misc {
   uint64_t o_full[2], o_free[2];
   uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
   uint64_t mma_final;
+  uint64_t p2_full[4], p2_mma[4];  // SEGMENTED second phase: tiles landed, correction done
   uint32_t tmem_base;
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
@@ -226,32 +230,34 @@ template <> struct In2<__nv_bfloat16> {
 
 __device__ __forceinline__ void sts32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
 
-// The 32 output rows of one warp (its lanes of a lane-tile pair region in tensor
-// memory) -> their grid cells, 32 columns at a time.  Each lane writes its row into a
-// per-warp staging tile in shared memory (16-byte chunks, XOR-swizzled by row so the
-// writes spread over all banks); after __syncwarp the warp copies the tile out with
-// whole rows per 8 (fp32) or 4 (16-bit) lanes, so every 16-byte global store
-// instruction covers 4 or 8 full row segments.  `nf` collects x * 0 over the values:
-// it turns NaN once any of them is not finite.
+// 16-byte chunk j of staged row R (rows of kRowB bytes) sits at R*kRowB + 16*(j ^ sw(R)),
+// so the row-per-lane writes and the row-per-group reads both spread over all banks.
+template <int kRowB>
+__device__ __forceinline__ int stage_chunk(int R, int j) {
+  constexpr int kLanesPerRow = kRowB / 16;
+  const int swz = (kLanesPerRow == 8) ? (R & 7) : ((R >> 1) & 3);
+  return R * kRowB + 16 * (j ^ swz);
+}
+
+// The 32 rows of one warp (its lanes of a tensor-memory region, 64 fp32 columns) ->
+// memory as Tout, 32 columns at a time.  Each lane writes its row into a per-warp
+// staging tile in shared memory; after __syncwarp the warp copies the tile out with
+// whole rows per 8 (fp32) or 4 (16-bit) lanes, so every 16-byte global store covers
+// 4 or 8 full row segments.  `rowdst` is this lane's destination row (nullptr: not
+// stored).  `nf` collects x * 0 over the values: it turns NaN once any is not finite.
 template <typename Tout>
-__device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, uint32_t taddr, bool valid,
-                                              long long s, uint8_t* wstage, int lane, float& nf) {
+__device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, uint8_t* wstage, int lane,
+                                              float& nf) {
   constexpr int kRowB = 32 * (int)sizeof(Tout);  // staged bytes per row and half
   constexpr int kLanesPerRow = kRowB / 16;       // 8 (fp32) or 4 (16-bit)
   constexpr int kRowsPerOp = 32 / kLanesPerRow;
-  long long mrow = -1;
-  if (valid) mrow = ((long long)b * p.L() + scan_to_token(s, p.direction, p.H, p.W)) * p.heads + h;
+  const unsigned long long myrow = reinterpret_cast<unsigned long long>(rowdst);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     float v[32];
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
     uint8_t* buf = wstage;  // one 32-row tile, reused by both halves
-    // 16-byte chunk j of row R sits at R*kRowB + 16*(j ^ sw(R))
-    auto chunk_at = [&](int R, int j) -> int {
-      const int swz = (kLanesPerRow == 8) ? (R & 7) : ((R >> 1) & 3);
-      return R * kRowB + 16 * (j ^ swz);
-    };
     if constexpr (sizeof(Tout) == 4) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -259,7 +265,8 @@ __device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, ui
         nf = fmaf(v[4 * j + 1], 0.f, nf);
         nf = fmaf(v[4 * j + 2], 0.f, nf);
         nf = fmaf(v[4 * j + 3], 0.f, nf);
-        *reinterpret_cast<float4*>(buf + chunk_at(lane, j)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        *reinterpret_cast<float4*>(buf + stage_chunk<kRowB>(lane, j)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       }
     } else {
       __half2 acc = __float2half2_rn(0.f);
@@ -280,7 +287,7 @@ __device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, ui
             nf = fmaf(x1, 0.f, nf);
           }
         }
-        *reinterpret_cast<uint4*>(buf + chunk_at(lane, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(buf + stage_chunk<kRowB>(lane, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       if constexpr (std::is_same<Tout, __half>::value) {
         const float2 a = __half22float2(acc);
@@ -292,14 +299,67 @@ __device__ __forceinline__ void epilogue_warp(const Problem& p, int b, int h, ui
 #pragma unroll
     for (int it = 0; it < kLanesPerRow; ++it) {
       const int R = it * kRowsPerOp + lane / kLanesPerRow;
-      const long long mr = __shfl_sync(0xffffffffu, mrow, R);
-      const uint4 x = *reinterpret_cast<const uint4*>(buf + chunk_at(R, jj));
-      if (mr >= 0) {
-        Tout* dst = reinterpret_cast<Tout*>(p.out) + mr * 64 + 32 * half;
-        __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst) + 16 * jj), x);
-      }
+      const unsigned long long dr = __shfl_sync(0xffffffffu, myrow, R);
+      const uint4 x = *reinterpret_cast<const uint4*>(buf + stage_chunk<kRowB>(R, jj));
+      if (dr) __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dr) + kRowB * half + 16 * jj), x);
     }
     __syncwarp();  // the staging tile is free again
+  }
+}
+
+// Grid-cell destination of output row s of (b, h), or nullptr when not `valid`.
+template <typename Tout>
+__device__ __forceinline__ uint8_t* out_row(const Problem& p, int b, int h, bool valid, long long s) {
+  if (!valid) return nullptr;
+  const long long m = ((long long)b * p.L() + scan_to_token(s, p.direction, p.H, p.W)) * p.heads + h;
+  return reinterpret_cast<uint8_t*>(reinterpret_cast<Tout*>(p.out) + m * 64);
+}
+
+// Segmented mode, second phase: the 32 rows of one warp hold the correction Qh' S_start
+// (fp32, tensor memory); the row's partial output O_local (fp16, row-major 128 B rows at
+// `olc_rows` in shared memory) is added on the way out and the sum stored as Tout.
+template <typename Tout>
+__device__ __forceinline__ void epilogue_rows_add(uint32_t taddr, uint8_t* rowdst, const uint8_t* olc_rows,
+                                                  uint8_t* wstage, int lane, float& nf) {
+  constexpr int kRowB = 128;  // fp32 staging, 32 columns per half
+  const unsigned long long myrow = reinterpret_cast<unsigned long long>(rowdst);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float v[32];
+    tmem_ld32(taddr + 32u * half, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(wstage + stage_chunk<kRowB>(lane, j)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    __syncwarp();
+    const int jj = lane & 7;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int R = it * 4 + (lane >> 3);
+      const unsigned long long dr = __shfl_sync(0xffffffffu, myrow, R);
+      const float4 c = *reinterpret_cast<const float4*>(wstage + stage_chunk<kRowB>(R, jj));
+      const uint2 ol = *reinterpret_cast<const uint2*>(olc_rows + R * 128 + (32 * half + 4 * jj) * 2);
+      const float2 o01 = __half22float2(bits_h2(ol.x)), o23 = __half22float2(bits_h2(ol.y));
+      const float y0 = c.x + o01.x, y1 = c.y + o01.y, y2 = c.z + o23.x, y3 = c.w + o23.y;
+      if (dr) {  // (rows past the sequence end hold stale partials: neither checked nor stored)
+        nf = fmaf(y0, 0.f, nf);
+        nf = fmaf(y1, 0.f, nf);
+        nf = fmaf(y2, 0.f, nf);
+        nf = fmaf(y3, 0.f, nf);
+        uint8_t* d = reinterpret_cast<uint8_t*>(dr) + (32 * half + 4 * jj) * (int)sizeof(Tout);
+        if constexpr (sizeof(Tout) == 4) {
+          __stcs(reinterpret_cast<float4*>(d), make_float4(y0, y1, y2, y3));
+        } else if constexpr (std::is_same<Tout, __half>::value) {
+          __stcs(reinterpret_cast<uint2*>(d), make_uint2(pack_h2(y0, y1), pack_h2(y2, y3)));
+        } else {
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(y0, y1), b1 = __floats2bfloat162_rn(y2, y3);
+          __stcs(reinterpret_cast<uint2*>(d),
+                 make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1)));
+        }
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -311,6 +371,8 @@ struct Span {
 // (Gr = ceil(Nc / (n_s * rounds)) <= kHeldPerSet) except at the sequence end.
 __device__ __forceinline__ Span round_span(const FusedParams& fp, int r, int s) {
   if (fp.mode == 0) return Span{0, fp.Nc};
+  if (fp.mode == 2)  // one contiguous, balanced run of chunks per segment
+    return Span{(int)((long long)s * fp.Nc / fp.n_s), (int)((long long)(s + 1) * fp.Nc / fp.n_s)};
   const int gr = (fp.Nc + fp.n_s * fp.rounds - 1) / (fp.n_s * fp.rounds);
   Span sp;
   sp.c0 = min(fp.Nc, (r * fp.n_s + s) * gr);
@@ -363,9 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Problem& p = fp.p;
   WsHeader* hdr = fp.hdr;
 
-  const bool hold = fp.mode == 1;
-  const int seq = hold ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
-  const int seg = hold ? (int)blockIdx.x % fp.n_s : 0;
+  const bool hold = fp.mode == 1;   // rounds of held outputs (tensor memory)
+  const bool segm = fp.mode == 2;   // one run per segment, corrected in a second phase
+  const bool xcta = hold || segm;   // the CTAs of a sequence exchange segment summaries
+  const int seq = xcta ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
+  const int seg = xcta ? (int)blockIdx.x % fp.n_s : 0;
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
   const int rounds = hold ? fp.rounds : 1;
@@ -391,6 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&ms->mma_final, 1);
     for (int i = 0; i < 3; ++i) mbar_init(&ms->sready[i], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&ms->p2_full[i], 1);
+      mbar_init(&ms->p2_mma[i], 1);
+    }
     ms->abort = 0;
     for (int i = 0; i < 4; ++i) ms->go[i][0] = ms->go[i][1] = 0;
     fence_mbar_init();
@@ -827,14 +895,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool alive = true;
     for (int r = 0; r < rounds && alive; ++r) {
       const Span sp = round_span(fp, r, seg);
-      float* mine = hold ? fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64) : nullptr;
+      float* mine = xcta ? fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64) : nullptr;
       // The summary slot and the held Qh' set of this round were used by the round two
       // back: wait until that round's epilogue, which every CTA's scan of that round
       // precedes, is finished -- also for a round without chunks, whose neutral summary
       // would otherwise overwrite a slot other CTAs may still be scanning.
       if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
       if (sp.c1 <= sp.c0) {
-        if (hold) {  // an empty segment still publishes a neutral summary
+        if (xcta) {  // an empty segment still publishes a neutral summary
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * c + cq), make_float2(0.f, 0.f));
@@ -904,6 +972,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16x128_x8(tl + kColHQ + (kSetCols / 2) * (uint32_t)(r & 1) + 32u * (uint32_t)(g >> 1) +
                                ((g & 1) ? kLaneTile1 : 0u),
                            hw);
+        } else if (segm && seg > 0) {
+          // segmented: this chunk's Qh' = Qh 2^(A from the segment start) -> its workspace
+          // tile (fp16, the 128-byte-swizzle MMA layout), the A operand of the second phase
+          const uint8_t* qt = smem + kOffStage + st * kStageBytes;
+          const float* eseg = reinterpret_cast<const float*>(qt + 3 * kTile) + 64;  // gate row 1
+          uint8_t* dst = reinterpret_cast<uint8_t*>(fp.qhp + ((size_t)seq * fp.Nc + c) * 4096);
+#pragma unroll
+          for (int cb = 0; cb < 8; ++cb) {
+            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
+            const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
+            const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
+            *reinterpret_cast<uint32_t*>(dst + r0 * 128 + o) =
+                h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
+            *reinterpret_cast<uint32_t*>(dst + r1 * 128 + o) =
+                h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
+          }
         }
         // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
         // the A operand of P V.  A rows are read from the lanes of the output rows, so P
@@ -963,7 +1047,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (wtid == 0 && !last_chunk) mbar_arrive(&ms->sready[(n + 1) % 3]);
       }
       if (!alive) break;
-      if (hold) {
+      // the Qh' tiles written above are read back by bulk copy (async proxy)
+      if (segm && seg > 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+      if (xcta) {
         // segment summary of this round: U_seg = local end state, its log2 decay
 #pragma unroll
         for (int cb = 0; cb < 8; ++cb) {
@@ -987,19 +1073,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
+    bool alive_c = true;
     if (!hold) {
-      const int pairs = (fp.Nc + 1) / 2;
+      // STREAM: the whole sequence; SEGMENTED: this segment's run, whose outputs (but
+      // segment 0's) are partial -- fp16 rows of the workspace, corrected in phase two
+      const Span sp0 = round_span(fp, 0, seg);
+      const int cnt = sp0.c1 - sp0.c0;
+      const bool partial = segm && seg > 0;
+      const int pairs = (cnt + 1) / 2;
       for (int pr = 0; pr < pairs; ++pr) {
-        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) break;
+        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) { alive_c = false; break; }
         tc_fence_after();
-        const long long s = (long long)(2 * pr + tsel) * kChunk + (fp.rev ? 63 - trow : trow);
-        epilogue_warp<Tout>(p, b, h, tl + kColO + 64u * (uint32_t)(pr & 1), 2 * pr + tsel < fp.Nc && s < L, s, wstage,
-                            lane, nonfinite);
+        const int ci = 2 * pr + tsel;
+        const long long s = (long long)(sp0.c0 + ci) * kChunk + (fp.rev ? 63 - trow : trow);
+        const bool valid = ci < cnt && s < L;
+        if (partial) {
+          uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp0.c0 + ci) * 4096) + trow * 128
+                              : nullptr;
+          epilogue_rows<__half>(tl + kColO + 64u * (uint32_t)(pr & 1), od, wstage, lane, nonfinite);
+        } else {
+          epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)(pr & 1), out_row<Tout>(p, b, h, valid, s), wstage, lane,
+                              nonfinite);
+        }
         tc_fence_before();
         wg_sync(wg);
         if (wtid == 0) mbar_arrive(&ms->o_free[pr & 1]);
       }
-    } else {
+      // the O_local rows written above are read back by bulk copy (async proxy)
+      if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    if (xcta && alive_c) {
       // Round-end scan of the segment summaries.  This CTA owns state entries
       // [4 f0, 4 f1) (float4 units f, F of them).  Threads split into nB blocks of bs
       // consecutive segments x FP float4 columns (nB * FP <= 128): a thread loads its
@@ -1108,6 +1211,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         wg_sync(wg);
+        if (segm) {
+          // ---- second phase: outputs of segment s > 0 = O_local + Qh' S_start.  Chunk
+          // pairs: Qh' and O_local tiles (2 x 8 KB each, consecutive in the workspace) come
+          // back by bulk copy into the free staging buffers; one M = 128 MMA per pair
+          // puts chunk 2m's rows in lanes 0-63 and chunk 2m+1's in lanes 64-127.
+          if (seg > 0) {
+            const int cnt = sp.c1 - sp.c0, npairs = (cnt + 1) / 2;
+            const uint32_t id_128 = idesc_f16(0, 128, 64, 0, 1);
+            auto issue_loads = [&](int m2) {
+              const int sl = m2 & 3;
+              uint8_t* sbuf = smem + kOffStage + sl * kStageBytes;
+              const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
+              mbar_arrive_expect_tx(&ms->p2_full[sl], (uint32_t)(2 * nb * 8192));
+              bulk_load(sbuf, fp.qhp + ((size_t)seq * fp.Nc + c) * 4096, (uint32_t)(nb * 8192), &ms->p2_full[sl]);
+              bulk_load(sbuf + 16384, fp.olc + ((size_t)seq * fp.Nc + c) * 4096, (uint32_t)(nb * 8192), &ms->p2_full[sl]);
+            };
+            if (wtid == 0)
+              for (int m2 = 0; m2 < npairs && m2 < 4; ++m2) issue_loads(m2);
+            for (int m2 = 0; m2 < npairs; ++m2) {
+              const int sl = m2 & 3;
+              const uint32_t par = (uint32_t)(m2 >> 2) & 1u;
+              if (!wg_wait(wg, wtid, &ms->p2_full[sl], par, ms, hdr, 0x605, slot)) break;
+              if (wtid == 0) {
+                tc_fence_after();
+                const uint32_t a0 = s_base + kOffStage + sl * kStageBytes;
+                for (int k = 0; k < 4; ++k)
+                  mma_f16(tmem + 64u * sl, sw128_desc(a0 + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_128, k > 0);
+                mma_commit(&ms->p2_mma[sl]);
+              }
+              if (!wg_wait(wg, wtid, &ms->p2_mma[sl], par, ms, hdr, 0x606, slot)) break;
+              tc_fence_after();
+              const int ci = 2 * m2 + (wq >> 1), row = 32 * (wq & 1) + lane;
+              const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
+              const uint8_t* olc_rows = smem + kOffStage + sl * kStageBytes + 16384 + (wq >> 1) * 8192 + 32 * (wq & 1) * 128;
+              epilogue_rows_add<Tout>(tl + 64u * sl, out_row<Tout>(p, b, h, ci < cnt && s < L, s), olc_rows, wstage, lane,
+                                      nonfinite);
+              tc_fence_before();
+              wg_sync(wg);  // the pair's buffers are read out
+              if (wtid == 0 && m2 + 4 < npairs) issue_loads(m2 + 4);
+            }
+          }
+          continue;
+        }
         const int G = sp.c1 - sp.c0;
         ok0 = true;
         if (wtid == 0) {
@@ -1134,8 +1280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
           const int gi = 2 * m2 + tsel;
           const long long s = (long long)(sp.c0 + gi) * kChunk + (fp.rev ? 63 - trow : trow);
-          epilogue_warp<Tout>(p, b, h, tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, gi < G && s < L, s, wstage,
-                              lane, nonfinite);
+          epilogue_rows<Tout>(tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, out_row<Tout>(p, b, h, gi < G && s < L, s),
+                              wstage, lane, nonfinite);
         }
         tc_fence_before();
         wg_sync(wg);
@@ -1152,7 +1298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
   // last CTA out resets this call's counters: the workspace is ready for the next call
-  if (hold && tid == 0) {
+  if (xcta && tid == 0) {
     __threadfence();
     const unsigned int done = atomicAdd(&hdr->ticket, 1u);
     if (done == (unsigned int)fp.grid - 1) {
@@ -1228,6 +1374,13 @@ Plan make_plan(const Problem& p, int sms) {
     const int per_round = pl.n_s * kHeldPerSet;
     pl.rounds = (Nc + per_round - 1) / per_round;
     pl.grid = pl.n_seq * pl.n_s;
+    // GTR_FUSED_MODE=2: one contiguous run per segment, corrected in a second phase
+    if (const char* e = getenv("GTR_FUSED_MODE")) {
+      if (e[0] == '2') {
+        pl.mode = 2;
+        pl.rounds = 1;
+      }
+    }
   }
   return pl;
 }
@@ -1276,6 +1429,8 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.agg = w.agg;
   fp.sstart = w.sstart;
   fp.carry = w.carry;
+  fp.qhp = w.qhp;
+  fp.olc = w.olc;
   fp.n_seq = pl.n_seq;
   fp.n_s = pl.n_s;
   fp.rounds = pl.rounds;
@@ -1309,7 +1464,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;
+  attr[0].val.cooperative = pl.mode != 0 ? 1 : 0;  // the CTAs of a sequence wait on one another
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;
@@ -1318,11 +1473,19 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
 
 }  // namespace
 
+// Per-chunk tiles of the segmented mode's second phase (Qh' and O_local, fp16): only when
+// sequences are split over CTAs.
+size_t segmented_tile_bytes(const Problem& p) {
+  return hold_segments(p) ? (size_t)p.B * p.heads * p.n_chunks() * 4096 * sizeof(uint16_t) : 0;
+}
+
 size_t fused_workspace_bytes(const Problem& p) {
   const size_t segs = hold_segments(p);
   const size_t carry_seqs = segs ? (size_t)p.B * p.heads : 0;
-  return sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t) +
-         carry_seqs * 4096 * sizeof(float);
+  size_t b = sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t) +
+             carry_seqs * 4096 * sizeof(float);
+  b = (b + 1023) & ~size_t(1023);  // 1 KB-aligned tiles for the bulk copies
+  return b + 2 * segmented_tile_bytes(p);
 }
 
 FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
@@ -1338,6 +1501,12 @@ FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
   w.sstart = reinterpret_cast<uint16_t*>(base);
   base += segs * 4096 * sizeof(uint16_t);
   w.carry = reinterpret_cast<float*>(base);
+  base += (hold_segments(p) ? (size_t)p.B * p.heads : 0) * 4096 * sizeof(float);
+  const size_t used = (size_t)(base - reinterpret_cast<uint8_t*>(ws));
+  base = reinterpret_cast<uint8_t*>(ws) + ((used + 1023) & ~size_t(1023));
+  const size_t tiles = segmented_tile_bytes(p);
+  w.qhp = tiles ? reinterpret_cast<uint16_t*>(base) : nullptr;
+  w.olc = tiles ? reinterpret_cast<uint16_t*>(base + tiles) : nullptr;
   return w;
 }
 

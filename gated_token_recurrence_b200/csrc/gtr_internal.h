@@ -24,6 +24,8 @@ struct FusedWorkspace {
   float* agg;              // per-segment summaries
   uint16_t* sstart;        // per-segment start states (16-bit, MMA layout)
   float* carry;            // per-sequence state entering the current round (fp32)
+  uint16_t* qhp;           // segmented mode: per-chunk Qh' tiles (fp16, MMA layout)
+  uint16_t* olc;           // segmented mode: per-chunk outputs from a zero segment start (fp16)
 };
 
 size_t split_workspace_bytes(const Problem& p);
