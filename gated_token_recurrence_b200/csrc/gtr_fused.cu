@@ -21,27 +21,29 @@
 // fp16 range) are reported as GTR_ERR_RANGE.
 //
 // Two modes.  STREAM: one CTA walks a whole sequence, carrying the exact fp32
-// state.  HOLD: the n_s CTAs of a sequence each take a segment of every round;
-// a CTA computes its chunks from a zero segment-start state and keeps the outputs
-// in tensor memory, the n_s CTAs scan the segment summaries (each owns a slice of
-// the 64x64 state entries), and each CTA adds (Q * 2^(A from its segment start))
-// times its segment-start state to the held outputs.  Round r's scan and
-// epilogue overlap round r+1's chunks (two held sets).
+// state.  SEGMENTED: the n_s CTAs of a sequence each walk one contiguous run of
+// its chunks (a segment) from a zero start state.  Segment 0's outputs are final;
+// the others write their partial outputs O_local and Qh' = Qh * 2^(A from the
+// segment start) to the workspace and publish the segment summary (end state,
+// log2 decay).  The n_s CTAs then scan the summaries (each owns a slice of the
+// 64x64 state entries), and in a second phase every CTA of a segment s > 0 adds
+// Qh' S_start(s) to O_local, one M = 128 MMA per chunk pair, spread over all four
+// of its warpgroups.
 //
 // Warp roles (608 threads):
 //   warps 0-7   WG_A  two warpgroups, one per half of the key channels: cumulative
 //               gates, Qh / Kh in place, CUDA-core scores
-//   warps 8-11  WG_B  score masking, fp32 state update, held Qh' (16-lane tensor-memory
+//   warps 8-11  WG_B  score masking, fp32 state update, Qh' (16-lane tensor-memory
 //               loads, so every lane of a warp does the same work)
-//   warps 12-15 WG_C  epilogue (both modes); HOLD round end: summary scan, correction
+//   warps 12-15 WG_C  epilogue; SEGMENTED: summary scan
 //   warps 16-17 producer: TMA boxes, or cp.async row copies (direction remap,
 //               128-byte-swizzled placement, zero fill past the sequence end)
 //   warp 18     tcgen05 MMA issuer and tensor-memory owner
+//   SEGMENTED second phase: warpgroups 0-3 (warps 0-15) each take every fourth pair
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
-#include <cstdlib>
 #include <mutex>
 #include <type_traits>
 
@@ -55,7 +57,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kStages = 4;          // staging depth (chunks in flight)
-constexpr int kHeldPerSet = 4;      // chunks held per CTA per round (HOLD)
+constexpr int kSU = 4;              // score / U' regions in tensor memory (chunks in flight)
 constexpr int kThreads = 608;
 constexpr int kProducerThreads = 64;
 constexpr int kMmaWarp = 18;
@@ -74,25 +76,27 @@ constexpr int kOffStg = kOffSst + kTile;                   // output staging, 4 
 constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
 constexpr int kMiscBytes = 2048;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+// second phase, pair slot q (one per warpgroup) in staging buffer q: Qh' of the pair
+// (16 KB, the A operand; then the warps' fp32 output staging) and O_local (16 KB)
+constexpr int kP2Olc = 16384;
+static_assert(2 * kP2Olc <= kStageBytes, "a chunk pair's second-phase tiles fit one staging buffer");
 
 // tensor memory columns
-constexpr uint32_t kColSU = 0;     // [2] x 64: scores (lane tile 0; masked fp16 P over their first 32
-                                   // columns) and U' (lane tile 1)
-constexpr uint32_t kColO = 128;    // STREAM: [2] x 64 output pairs; HOLD: [2 sets] x kSetCols
+constexpr uint32_t kColSU = 0;     // [kSU] x 64: scores (lane tile 0; masked fp16 P over their first
+                                   // 32 columns) and U' (lane tile 1)
+constexpr uint32_t kColO = kColSU + 64u * kSU;  // [2] x 64 output pairs (chunk 2m lane tile 0, 2m+1 tile 1)
 constexpr uint32_t kLaneTile1 = 16u << 16;
-constexpr uint32_t kSetCols = 64u * (kHeldPerSet / 2);
-constexpr uint32_t kColHQ = kColO + 2 * kSetCols;  // HOLD: [2 sets] x kSetCols/2 held fp16 Qh' (A operands)
-static_assert(kHeldPerSet % 2 == 0, "held chunks come in lane-tile pairs");
-static_assert(kColHQ + kSetCols <= kTmemCols, "tensor memory budget");
+static_assert(kColO + 128 <= kTmemCols, "tensor memory budget");
+static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) reuse the score regions");
 
-// HOLD-mode counters sit at a fixed place right after the workspace header, whatever
+// Segment counters sit at a fixed place right after the workspace header, whatever
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
-constexpr size_t kMaxHoldSegments = 256;  // CTAs of one launch in HOLD mode (>= the SM count)
-constexpr size_t kCounterBytes = 2 * kMaxHoldSegments * sizeof(unsigned int);
-constexpr int kScanBlock = 8;            // segments one WG_C thread composes in registers
+constexpr size_t kMaxSegCtas = 256;  // CTAs of one launch in SEGMENTED mode (>= the SM count)
+constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
+constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
-struct FusedParams {
+struct alignas(64) FusedParams {
   // TMA tensor maps for Q, K, V (16-bit, 128-byte swizzle) and the log-gates (fp32):
   // row view [B][L][heads][64] (4-D) or column view [B][H][W][heads][64] (5-D), boxes of
   // 64 consecutive scan positions of one (batch, head)
@@ -100,12 +104,11 @@ struct FusedParams {
   Problem p;
   WsHeader* hdr;
   unsigned int* counters;  // [n_seq][2], monotonic within a call, zero between calls
-  float* agg;              // [n_seq][2 round parities][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
-  float* carry;            // [n_seq][64*64] state entering the current round, fp32
+  float* agg;              // [n_seq][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
   uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
-  uint16_t* qhp;           // SEGMENTED: [n_seq][Nc][64*64] held Qh' per chunk, fp16, MMA layout
-  uint16_t* olc;           // SEGMENTED: [n_seq][Nc][64][64] outputs from a zero segment start, fp16
-  int n_seq, n_s, rounds, Nc, mode;  // mode 0 = STREAM, 1 = HOLD, 2 = SEGMENTED
+  uint16_t* qhp;           // [n_seq][Nc][64*64] Qh' per chunk, fp16, MMA layout
+  uint16_t* olc;           // [n_seq][Nc][64][64] outputs from a zero segment start, fp16
+  int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED
   int grid;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
   int tma;                 // 1: every chunk is one TMA box per tensor; 0: cp.async row copies
@@ -117,11 +120,12 @@ struct Misc {
   uint64_t full[kStages], empty[kStages];
   // opready is per stage: the operand builder may run up to kStages chunks ahead of the
   // MMA warp, so a two-deep ring could complete a phase twice before it is observed
-  uint64_t opready[kStages], su_full[2], su_free[2], sready[3], pready[2];
-  uint64_t o_full[2], o_free[2];
-  uint64_t agg_pub[2], round_done[2], corr_done[2], set_free[2];
-  uint64_t mma_final;
-  uint64_t p2_full[4], p2_mma[4];  // SEGMENTED second phase: tiles landed, correction done
+  uint64_t opready[kStages];
+  uint64_t su_full[kSU], su_free[kSU], pready[kSU];  // per score / U' region
+  uint64_t sready[3], sfree[3];                      // per chunk-start state tile
+  uint64_t o_full[2], o_free[2];                     // per output pair
+  uint64_t agg_pub, p2_go, mma_final;
+  uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
   uint32_t tmem_base;
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
@@ -131,8 +135,9 @@ struct Misc {
   int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
 };
 // The in-chunk log2 decay per channel (a) of a staged chunk is kept in row 0 of its
-// gate tile once the gates are consumed; the round-end scan exchanges its block
-// transfers through the segment-start-state tile, which is idle at that point.
+// gate tile once the gates are consumed, the factor 2^(decay from the segment start)
+// in row 1; the summary scan exchanges its block transfers through the segment-start-
+// state tile, which is idle at that point.
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -367,52 +372,69 @@ struct Span {
   int c0, c1;
 };
 
-// Chunk range of segment s in round r: every segment of every round holds Gr chunks
-// (Gr = ceil(Nc / (n_s * rounds)) <= kHeldPerSet) except at the sequence end.
-__device__ __forceinline__ Span round_span(const FusedParams& fp, int r, int s) {
+// Chunk run of segment s: one contiguous, balanced run per segment (STREAM: the whole
+// sequence).  With n_s <= Nc every segment holds at least one chunk.
+__device__ __forceinline__ Span seg_span(const FusedParams& fp, int s) {
   if (fp.mode == 0) return Span{0, fp.Nc};
-  if (fp.mode == 2)  // one contiguous, balanced run of chunks per segment
-    return Span{(int)((long long)s * fp.Nc / fp.n_s), (int)((long long)(s + 1) * fp.Nc / fp.n_s)};
-  const int gr = (fp.Nc + fp.n_s * fp.rounds - 1) / (fp.n_s * fp.rounds);
-  Span sp;
-  sp.c0 = min(fp.Nc, (r * fp.n_s + s) * gr);
-  sp.c1 = min(fp.Nc, (r * fp.n_s + s + 1) * gr);
-  return sp;
+  return Span{(int)((long long)s * fp.Nc / fp.n_s), (int)((long long)(s + 1) * fp.Nc / fp.n_s)};
 }
 
-// Position in a CTA's chunk sequence: round r, chunk c, index g within the round.
-// Rounds without chunks only occur at the end of a sequence.
-struct Cursor {
-  int r, c, g;
-  Span sp;
-  __device__ void settle(const FusedParams& fp, int seg, int rounds) {
-    while (r < rounds && c >= sp.c1) {
-      ++r;
-      g = 0;
-      if (r < rounds) {
-        sp = round_span(fp, r, seg);
-        c = sp.c0;
-      }
-    }
-  }
-  __device__ void start(const FusedParams& fp, int seg, int rounds) {
-    r = 0;
-    g = 0;
-    sp = round_span(fp, 0, seg);
-    c = sp.c0;
-    settle(fp, seg, rounds);
-  }
-  __device__ void advance(const FusedParams& fp, int seg, int rounds) {
-    ++c;
-    ++g;
-    settle(fp, seg, rounds);
-  }
-};
+// Phase parity for the n-th use of a barrier of a ring `depth` deep, and for waiting on
+// the release of use n - depth (passes at once for n < depth on a fresh barrier).
+template <int depth>
+__device__ __forceinline__ uint32_t ph_use(int n) { return (uint32_t)(n / depth) & 1u; }
+template <int depth>
+__device__ __forceinline__ uint32_t ph_rel(int n) { return ((uint32_t)(n / depth) & 1u) ^ 1u; }
 
-// Phase parity for the n-th use of a double-buffered barrier, and for waiting on its
-// release by use n-2 (passes at once for n < 2 on a fresh barrier).
-__device__ __forceinline__ uint32_t ph_of(int n) { return (uint32_t)(n >> 1) & 1u; }
-__device__ __forceinline__ uint32_t ph_free(int n) { return ((uint32_t)(n >> 1) & 1u) ^ 1u; }
+// Second phase of a segment s > 0, run by warpgroup q (named barrier q + 1) once the
+// segment start state S_start is in shared memory: for chunk pairs m = q, q+4, ...
+//   out = O_local + Qh' S_start,
+// Qh' and O_local of the pair (two chunks each, consecutive in the workspace) come back
+// by bulk copy into staging buffer q; one M = 128 MMA puts chunk 2m's rows in lanes
+// 0-63 and chunk 2m+1's in lanes 64-127 of tensor-memory slot q; warp wq of the group
+// takes lanes 32wq .. 32wq+31 (chunk 2m + wq/2, rows 32(wq%2) ..).
+template <typename Tout>
+__device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem, uint32_t tmem, int q,
+                             int wtid, int lane, int seq, int b, int h, Span sp, int& slot, float& nf) {
+  const int wq = (wtid >> 5) & 3;
+  if (!wg_wait(q, wtid, &ms->p2_go, 0u, ms, hdr, 0x700u + q, slot)) return;
+  const long long L = fp.p.L();
+  const int cnt = sp.c1 - sp.c0, npairs = (cnt + 1) / 2;
+  uint8_t* sbuf = smem + kOffStage + q * kStageBytes;
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t a0 = s_base + kOffStage + q * kStageBytes;
+  const uint32_t id_128 = idesc_f16(0, 128, 64, 0, 1);  // A K-major, B MN-major
+  const uint32_t dq = tmem + 64u * (uint32_t)q;
+  int u = 0;
+  for (int m2 = q; m2 < npairs; m2 += 4, ++u) {
+    const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
+    if (wtid == 0) {
+      const size_t t0 = ((size_t)seq * fp.Nc + c) * 4096;
+      mbar_arrive_expect_tx(&ms->p2_full[q], (uint32_t)(2 * nb * kTile));
+      bulk_load(sbuf, fp.qhp + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
+      bulk_load(sbuf + kP2Olc, fp.olc + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
+    }
+    if (!wg_wait(q, wtid, &ms->p2_full[q], (uint32_t)u & 1u, ms, hdr, 0x710u + q, slot)) return;
+    if (wtid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_f16(dq, sw128_desc(a0 + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_128, k > 0);
+      mma_commit(&ms->p2_mma[q]);
+    }
+    if (!wg_wait(q, wtid, &ms->p2_mma[q], (uint32_t)u & 1u, ms, hdr, 0x720u + q, slot)) return;
+    tc_fence_after();
+    const int ci = 2 * m2 + (wq >> 1), row = 32 * (wq & 1) + lane;
+    const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
+    const uint8_t* olc_rows = sbuf + kP2Olc + (wq >> 1) * kTile + 32 * (wq & 1) * 128;
+    // fp32 staging over the pair's Qh' (its MMA has completed)
+    epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp.p, b, h, ci < cnt && s < L, s),
+                            olc_rows, sbuf + wq * 4096, lane, nf);
+    tc_fence_before();
+    fence_proxy_async_smem();  // generic accesses of the buffer before the next pair's copies
+    wg_sync(q);
+  }
+}
 
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -425,14 +447,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Problem& p = fp.p;
   WsHeader* hdr = fp.hdr;
 
-  const bool hold = fp.mode == 1;   // rounds of held outputs (tensor memory)
-  const bool segm = fp.mode == 2;   // one run per segment, corrected in a second phase
-  const bool xcta = hold || segm;   // the CTAs of a sequence exchange segment summaries
-  const int seq = xcta ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
-  const int seg = xcta ? (int)blockIdx.x % fp.n_s : 0;
+  const bool segm = fp.mode == 1;          // the CTAs of a sequence exchange segment summaries
+  const int seq = segm ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
+  const int seg = segm ? (int)blockIdx.x % fp.n_s : 0;
+  const bool partial = segm && seg > 0;    // outputs completed in the second phase
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
-  const int rounds = hold ? fp.rounds : 1;
+  const Span sp = seg_span(fp, seg);
+  const int cnt = sp.c1 - sp.c0;           // chunks of this CTA
   float nonfinite = 0.f;
 
   if (tid == 0) {
@@ -442,23 +464,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->opready[i], 2);  // one arrival per channel half
       ms->fb[i] = 0;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSU; ++i) {
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
       mbar_init(&ms->pready[i], 1);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&ms->sready[i], 1);
+      mbar_init(&ms->sfree[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
-      mbar_init(&ms->agg_pub[i], 1);
-      mbar_init(&ms->round_done[i], 1);
-      mbar_init(&ms->corr_done[i], 1);
-      mbar_init(&ms->set_free[i], 1);
     }
-    mbar_init(&ms->mma_final, 1);
-    for (int i = 0; i < 3; ++i) mbar_init(&ms->sready[i], 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&ms->p2_full[i], 1);
       mbar_init(&ms->p2_mma[i], 1);
     }
+    mbar_init(&ms->agg_pub, 1);
+    mbar_init(&ms->p2_go, 1);
+    mbar_init(&ms->mma_final, 1);
     ms->abort = 0;
     for (int i = 0; i < 4; ++i) ms->go[i][0] = ms->go[i][1] = 0;
     fence_mbar_init();
@@ -477,41 +502,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Staged chunk row r holds scan position c*64 + r, or c*64 + 63 - r for the reversed
     // directions (right-to-left, bottom-to-top), where a chunk is stored in memory order.
     const int pt = tid - 16 * 32;  // 0..63
-    int n = 0;
-    bool stop = false;
     if (fp.tma) {
       // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
       // plain); rows past the sequence end arrive zero-filled.
       if (pt == 0) {
-        for (int r = 0; r < rounds && !stop; ++r) {
-          const Span sp = round_span(fp, r, seg);
-          for (int c = sp.c0; c < sp.c1; ++c, ++n) {
-            const int st = n % kStages;
-            if (!wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100)) { stop = true; break; }
-            uint8_t* sb = smem + kOffStage + st * kStageBytes;
-            mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);
-            const long long s0 = (long long)c * kChunk;
-            if (p.direction <= GTR_R2L) {
-              // row view: 64 consecutive grid cells m (right-to-left: one image row)
-              long long m0 = s0;
-              if (p.direction == GTR_R2L) {
-                const long long y = s0 / p.W;
-                m0 = y * p.W + (p.W - 64 - (s0 - y * p.W));
-              }
-              tma_load_4d(sb, &fp.tq, &ms->full[st], 0, h, (int)m0, b);
-              tma_load_4d(sb + kTile, &fp.tk, &ms->full[st], 0, h, (int)m0, b);
-              tma_load_4d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, (int)m0, b);
-              tma_load_4d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, (int)m0, b);
-            } else {
-              // column view: 64 consecutive y of one column x
-              const int x = (int)(s0 / p.H);
-              int y0 = (int)(s0 - (long long)x * p.H);
-              if (p.direction == GTR_B2T) y0 = p.H - 64 - y0;
-              tma_load_5d(sb, &fp.tq, &ms->full[st], 0, h, x, y0, b);
-              tma_load_5d(sb + kTile, &fp.tk, &ms->full[st], 0, h, x, y0, b);
-              tma_load_5d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, x, y0, b);
-              tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, x, y0, b);
+        for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
+          const int st = n % kStages;
+          if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) break;
+          uint8_t* sb = smem + kOffStage + st * kStageBytes;
+          mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);
+          const long long s0 = (long long)c * kChunk;
+          if (p.direction <= GTR_R2L) {
+            // row view: 64 consecutive grid cells m (right-to-left: one image row)
+            long long m0 = s0;
+            if (p.direction == GTR_R2L) {
+              const long long y = s0 / p.W;
+              m0 = y * p.W + (p.W - 64 - (s0 - y * p.W));
             }
+            tma_load_4d(sb, &fp.tq, &ms->full[st], 0, h, (int)m0, b);
+            tma_load_4d(sb + kTile, &fp.tk, &ms->full[st], 0, h, (int)m0, b);
+            tma_load_4d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, (int)m0, b);
+            tma_load_4d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, (int)m0, b);
+          } else {
+            // column view: 64 consecutive y of one column x
+            const int x = (int)(s0 / p.H);
+            int y0 = (int)(s0 - (long long)x * p.H);
+            if (p.direction == GTR_B2T) y0 = p.H - 64 - y0;
+            tma_load_5d(sb, &fp.tq, &ms->full[st], 0, h, x, y0, b);
+            tma_load_5d(sb + kTile, &fp.tk, &ms->full[st], 0, h, x, y0, b);
+            tma_load_5d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, x, y0, b);
+            tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, x, y0, b);
           }
         }
       }
@@ -528,135 +548,113 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j8 = pt & 7, rq = pt >> 3;     // 16-byte column, row within a group of 8
       const int j16 = pt & 15, rg = pt >> 4;   // gate rows: 16-byte column, row within 4
       const int srow = fp.rev ? 63 - pt : pt;  // staged row of scan position c*64 + pt
-      for (int r = 0; r < rounds && !stop; ++r) {
-        const Span sp = round_span(fp, r, seg);
-        for (int c = sp.c0; c < sp.c1; ++c, ++n) {
-          const int st = n % kStages;
-          int* rows = ms->rowoff[n & 1];
-          {
-            const long long s = (long long)c * kChunk + pt;
-            rows[srow] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
-          }
-          int ok = 0;
-          if (lane == 0) ok = wait_bar(&ms->empty[st], ((uint32_t)(n / kStages) & 1u) ^ 1u, ms, hdr, 0x100);
-          if (!__shfl_sync(0xffffffffu, ok, 0)) stop = true;
-          asm volatile("bar.sync 5, 64;" ::: "memory");  // the row table is complete
-          if (*(volatile int*)&ms->abort) stop = true;
-          if (stop) break;
-          const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int row = 8 * it + rq;
-            const int cell = rows[row];
-            const uint32_t nb = cell >= 0 ? 16u : 0u;
-            const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
-            const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
-            cp_async16(dst, gq + src, nb);
-            cp_async16(dst + kTile, gk + src, nb);
-            cp_async16(dst + 2 * kTile, gv + src, nb);
-          }
-#pragma unroll
-          for (int it = 0; it < 16; ++it) {
-            const int row = 4 * it + rg;
-            const int cell = rows[row];
-            const uint32_t nb = cell >= 0 ? 16u : 0u;
-            cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
-                       gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
-          }
-          cp_async_arrive_noinc(&ms->full[st]);
+      for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
+        const int st = n % kStages;
+        int* rows = ms->rowoff[n & 1];
+        {
+          const long long s = (long long)c * kChunk + pt;
+          rows[srow] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
         }
+        int ok = 0;
+        if (lane == 0) ok = wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100);
+        bool stop = !__shfl_sync(0xffffffffu, ok, 0);
+        asm volatile("bar.sync 5, 64;" ::: "memory");  // the row table is complete
+        if (*(volatile int*)&ms->abort) stop = true;
+        if (stop) break;
+        const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int row = 8 * it + rq;
+          const int cell = rows[row];
+          const uint32_t nb = cell >= 0 ? 16u : 0u;
+          const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
+          const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
+          cp_async16(dst, gq + src, nb);
+          cp_async16(dst + kTile, gk + src, nb);
+          cp_async16(dst + 2 * kTile, gv + src, nb);
+        }
+#pragma unroll
+        for (int it = 0; it < 16; ++it) {
+          const int row = 4 * it + rg;
+          const int cell = rows[row];
+          const uint32_t nb = cell >= 0 ? 16u : 0u;
+          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
+                     gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
+        }
+        cp_async_arrive_noinc(&ms->full[st]);
       }
       // copies already issued must land before this CTA's shared memory is released
       asm volatile("cp.async.wait_all;" ::: "memory");
     }
   } else if (warp == kMmaWarp) {
     // ===================================================================== MMA issuer
-    // Event-driven over the CTA's chunk sequence: whichever of stage 1 (scores, U'),
-    // stage 2a (O = Qh S) and stage 2b (O += P V) has its inputs ready is issued, so a
-    // slow operand build never holds back the products of earlier chunks (and with
-    // them the release of their staging buffers).
+    // Event-driven over the CTA's chunks: whichever of stage 1 (scores, U'), stage 2a
+    // (O = Qh S) and stage 2b (O += P V) has its inputs ready is issued, so a slow
+    // operand build never holds back the products of earlier chunks (and with them the
+    // release of their staging buffers).  Stage 1 runs up to kSU chunks ahead of 2b.
     if (lane == 0) {
       const uint32_t id_qk = idesc_f16(0, 64, 64, 0, 0);  // A K-major, B K-major
       const uint32_t id_kv = idesc_f16(0, 64, 64, 1, 1);  // A MN-major, B MN-major
       const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);  // A K-major, B MN-major
       const uint32_t s_base = smem_u32(smem);
-      int total = 0;
-      for (int r = 0; r < rounds; ++r) {
-        const Span sp = round_span(fp, r, seg);
-        total += sp.c1 - sp.c0;
-      }
-      // output region of chunk m at cursor position z
-      auto out_region = [&](const Cursor& z, int m) -> uint32_t {
-        if (hold)
-          return tmem + kColO + kSetCols * (uint32_t)(z.r & 1) + 64u * (uint32_t)(z.g >> 1) + ((z.g & 1) ? kLaneTile1 : 0u);
+      // output region of chunk m: pair (m/2) % 2, lane tile m % 2
+      auto out_region = [&](int m) -> uint32_t {
         return tmem + kColO + 64u * (uint32_t)((m >> 1) & 1) + ((m & 1) ? kLaneTile1 : 0u);
       };
-      Cursor za, zb;  // positions of stage 2a and 2b
-      za.start(fp, seg, rounds);
-      zb.start(fp, seg, rounds);
       int n1 = 0, n2a = 0, n2b = 0;
       uint64_t t_last = globaltimer();
-      while (n2b < total) {
+      while (n2b < cnt) {
         bool prog = false;
-        if (n2b < n2a && mbar_test(&ms->pready[n2b & 1], ph_of(n2b))) {
+        if (n2b < n2a && mbar_test(&ms->pready[n2b % kSU], ph_use<kSU>(n2b))) {
           // stage 2b of chunk m: O += P V with P in tensor memory; the chunk's staging
           // buffer and score region are free afterwards
-          const int m = n2b, bb = m & 1, st = m % kStages;
+          const int m = n2b, st = m % kStages, su = m % kSU;
           const uint32_t a_v = s_base + kOffStage + st * kStageBytes + 2 * kTile;
           // P sits in the lane tile of the chunk's output (A and D rows share lanes)
-          const bool otile = hold ? (zb.g & 1) != 0 : (m & 1) != 0;
-          const uint32_t a_p = tmem + kColSU + 64u * bb + (otile ? kLaneTile1 : 0u);
-          const uint32_t d_o = out_region(zb, m);
+          const uint32_t a_p = tmem + kColSU + 64u * su + ((m & 1) ? kLaneTile1 : 0u);
+          const uint32_t d_o = out_region(m);
           tc_fence_after();
           for (int k = 0; k < 4; ++k)
             mma_f16_ta(d_o, a_p + 8 * k, sw128_desc(a_v + 2048 * k), id_qs, 1);
-          mma_commit(&ms->su_free[bb]);
+          mma_commit(&ms->su_free[su]);
           mma_commit(&ms->empty[st]);
-          const bool round_end = zb.c + 1 == zb.sp.c1;
-          if (!hold && ((m & 1) || round_end)) mma_commit(&ms->o_full[(m >> 1) & 1]);
-          if (hold && round_end) mma_commit(&ms->round_done[zb.r & 1]);
-          zb.advance(fp, seg, rounds);
+          if ((m & 1) || m + 1 == cnt) mma_commit(&ms->o_full[(m >> 1) & 1]);
           ++n2b;
           prog = true;
         }
         if (n2a < n1) {
-          // stage 2a of chunk m: O = Qh S (S = the chunk-start state tile)
-          const int m = n2a, bb = m & 1, st = m % kStages;
-          bool rdy = mbar_test(&ms->sready[m % 3], (uint32_t)(m / 3) & 1u);
-          if (hold) {
-            // a held set is reused: the epilogue of the round two back must be finished
-            if (za.g == 0 && za.r >= 2) rdy = rdy && mbar_test(&ms->set_free[za.r & 1], ph_free(za.r));
-          } else if (!(m & 1)) {
-            rdy = rdy && mbar_test(&ms->o_free[(m >> 1) & 1], ph_free(m >> 1));
-          }
+          // stage 2a of chunk m: O = Qh S (S = the chunk-start state tile); an output
+          // pair's region is reused once the epilogue of the pair two back is done
+          const int m = n2a, st = m % kStages;
+          bool rdy = mbar_test(&ms->sready[m % 3], ph_use<3>(m));
+          if (!(m & 1)) rdy = rdy && mbar_test(&ms->o_free[(m >> 1) & 1], ph_rel<2>(m >> 1));
           if (rdy) {
             const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
             const uint32_t a_s = s_base + kOffS + (m % 3) * kTile;
-            const uint32_t d_o = out_region(za, m);
             tc_fence_after();
             for (int k = 0; k < 4; ++k)
-              mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-            za.advance(fp, seg, rounds);
+              mma_f16(out_region(m), sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
+            mma_commit(&ms->sfree[m % 3]);
             ++n2a;
             prog = true;
           }
         }
-        if (n1 < total && mbar_test(&ms->opready[n1 % kStages], (uint32_t)(n1 / kStages) & 1u) &&
-            mbar_test(&ms->su_free[n1 & 1], ph_free(n1))) {
+        if (n1 < cnt && mbar_test(&ms->opready[n1 % kStages], ph_use<kStages>(n1)) &&
+            mbar_test(&ms->su_free[n1 % kSU], ph_rel<kSU>(n1))) {
           // stage 1 of chunk n: scores = Qh Kh^T (tensor-core chunks), U' = Kh^T V
-          const int n = n1, bb = n & 1, st = n % kStages;
+          const int n = n1, st = n % kStages;
           const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
           const uint32_t a_k = a_q + kTile;                            // Kh
           const uint32_t a_v = a_q + 2 * kTile;
           tc_fence_after();
-          const uint32_t su = tmem + kColSU + 64u * bb;
+          const uint32_t su = tmem + kColSU + 64u * (uint32_t)(n % kSU);
           if (!*(volatile int*)&ms->fb[st]) {
             for (int k = 0; k < 4; ++k)
               mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
           }
           for (int k = 0; k < 4; ++k)
             mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
-          mma_commit(&ms->su_full[bb]);
+          mma_commit(&ms->su_full[n % kSU]);
           ++n1;
           prog = true;
         }
@@ -672,11 +670,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // sleep in hardware on the oldest pending step's barrier (woken when it
           // completes, at most half a microsecond); the loop then re-polls every step
           if (n2b < n2a)
-            (void)mbar_wait_sleep(&ms->pready[n2b & 1], ph_of(n2b), 500u);
+            (void)mbar_wait_sleep(&ms->pready[n2b % kSU], ph_use<kSU>(n2b), 500u);
           else if (n2a < n1)
-            (void)mbar_wait_sleep(&ms->sready[n2a % 3], (uint32_t)(n2a / 3) & 1u, 500u);
+            (void)mbar_wait_sleep(&ms->sready[n2a % 3], ph_use<3>(n2a), 500u);
           else
-            (void)mbar_wait_sleep(&ms->opready[n1 % kStages], (uint32_t)(n1 / kStages) & 1u, 500u);
+            (void)mbar_wait_sleep(&ms->opready[n1 % kStages], ph_use<kStages>(n1), 500u);
         }
       }
       // every MMA issued here has completed before tensor memory is freed
@@ -695,192 +693,191 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ch0 = 32 * hh + 4 * cc;
     const int row0 = 16 * w4 + 4 * (lane >> 3);  // rows row0 .. row0+3
     const bool rev = fp.rev != 0;
-    int slot = 0, n = 0;
+    int slot = 0;
     bool alive = true;
-    for (int r = 0; r < rounds && alive; ++r) {
-      const Span sp = round_span(fp, r, seg);
-      float a2s[4] = {0.f, 0.f, 0.f, 0.f};  // log2 decay from the segment start, channels ch0..ch0+3
-      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
-        const int bb = n & 1, st = n % kStages;
-        if (!wg_wait(wg, wtid, &ms->full[st], (uint32_t)(n / kStages) & 1u, ms, hdr, 0x301, slot)) {
-          alive = false;
-          break;
-        }
-        uint8_t* sb = smem + kOffStage + st * kStageBytes;
-        float* G = reinterpret_cast<float*>(sb + 3 * kTile);
-        // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, a scan over the
-        // warp's 4 row blocks, then over the 4 warps (staged rows run backwards in scan
-        // order when the chunk is reversed)
-        float A[4][4];
-        float run[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-          float gv[4][4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * 64 + ch0);
-            gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
-          }
-          if (!rev) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                run[e] = fmaf(gv[i][e], kLog2e, run[e]);
-                A[i][e] = run[e];
-              }
-          } else {
-#pragma unroll
-            for (int i = 3; i >= 0; --i)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                run[e] = fmaf(gv[i][e], kLog2e, run[e]);
-                A[i][e] = run[e];
-              }
-          }
-        }
-        float incl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          incl[e] = run[e];
-          if (!rev) {
-            float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
-            if (lane >= 8) incl[e] += x;
-            x = __shfl_up_sync(0xffffffffu, incl[e], 16);
-            if (lane >= 16) incl[e] += x;
-          } else {
-            float x = __shfl_down_sync(0xffffffffu, incl[e], 8);
-            if (lane < 24) incl[e] += x;
-            x = __shfl_down_sync(0xffffffffu, incl[e], 16);
-            if (lane < 16) incl[e] += x;
-          }
-        }
-        float* redh = &ms->red[hh][0][0];  // [4 warps][32 channels] of this channel half
-        if (rev ? lane < 8 : lane >= 24)
-          *reinterpret_cast<float4*>(redh + w4 * 32 + 4 * cc) = make_float4(incl[0], incl[1], incl[2], incl[3]);
-        wg_sync(wg);
-        float off[4], last[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          off[e] = incl[e] - run[e];
-          last[e] = 0.f;
-        }
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 t4 = *reinterpret_cast<const float4*>(redh + w * 32 + 4 * cc);
-          const float t[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (rev ? w > w4 : w < w4) off[e] += t[e];
-            last[e] += t[e];
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) A[i][e] += off[e];
-        // CUDA-core decision over all 64 channels: each warp covers its half's 32 channels,
-        // the two halves meet at a 256-thread barrier
-        bool exp_unsafe = false;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (-last[e] > fp.max_exp2) exp_unsafe = true;
-        const bool half_unsafe = __any_sync(0xffffffffu, exp_unsafe);
-        if (wtid == 0) ms->fbh[bb][hh] = half_unsafe ? 1 : 0;
-        asm volatile("bar.sync 6, 256;" ::: "memory");
-        const bool fbx = (*(volatile int*)&ms->fbh[bb][0] | *(volatile int*)&ms->fbh[bb][1]) != 0;
-        if (fbx) {
-          // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
-          // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i);
-          // warpgroup hh fills score columns 32hh .. 32hh+31 of its warps' rows.  A goes to
-          // the gate tile so that every thread can read every row and channel.
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
-          if (!wg_wait(wg, wtid, &ms->su_free[bb], ph_free(n), ms, hdr, 0x302, slot)) { alive = false; break; }
-          asm volatile("bar.sync 6, 256;" ::: "memory");  // A of both channel halves is in place
-          tc_fence_after();
-          const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
-          float sv[16];
-          for (int x = 0; x < 16; ++x) {
-            const int i = r0 + 8 * ((x & 3) >> 1);
-            const int j = 32 * hh + 8 * (x >> 2) + cq + (x & 1);
-            float acc = 0.f;
-            if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
-              for (int k = 0; k < 64; k += 2) {
-                const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
-                const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
-                acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
-                acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
-              }
-            }
-            sv[x] = acc * 0.125f;
-          }
-          tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * bb + 32u * hh, sv);
-          tmem_wait_st();
-          tc_fence_before();
-          asm volatile("bar.sync 6, 256;" ::: "memory");  // raw q / k reads done before the overwrite
-        }
-        // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
-        const __half2 eighth = __float2half2_rn(0.125f);
+    float a2s[4] = {0.f, 0.f, 0.f, 0.f};  // log2 decay from the segment start, channels ch0..ch0+3
+    for (int n = 0; n < cnt; ++n) {
+      const int bb = n & 1, st = n % kStages;
+      if (!wg_wait(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
+        alive = false;
+        break;
+      }
+      uint8_t* sb = smem + kOffStage + st * kStageBytes;
+      float* G = reinterpret_cast<float*>(sb + 3 * kTile);
+      // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, a scan over the
+      // warp's 4 row blocks, then over the 4 warps (staged rows run backwards in scan
+      // order when the chunk is reversed)
+      float A[4][4];
+      float run[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        float gv[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int row = row0 + i;
-          // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
-          const uint32_t off8 = row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
-          uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
-          uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
-          uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
-          uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
-            const float xk0 = fbx ? last[2 * e2] - A0 : -A0;
-            const float xk1 = fbx ? last[2 * e2 + 1] - A1 : -A1;
-            __half2 qh, kh;
-            if constexpr (std::is_same<Tin, __half>::value) {
-              qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
-              kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
-            } else {
-              const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
-              qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
-              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
-            }
-            qw[e2] = h2_bits(qh);
-            kw[e2] = h2_bits(kh);
-          }
-          *reinterpret_cast<uint2*>(sb + off8) = qraw;
-          *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
+          const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * 64 + ch0);
+          gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
         }
-        if constexpr (!std::is_same<Tin, __half>::value) {
-          // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range);
-          // the two warpgroups take alternate 16-byte chunks
-          uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
+        if (!rev) {
 #pragma unroll
-          for (int i = tid; i < kTile / 16; i += 2 * kWG) {
-            uint4 x = vt[i];
-            uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+          for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float2 f = In2<Tin>::unpack(w[e]);
-              w[e] = pack_h2(f.x, f.y);
+              run[e] = fmaf(gv[i][e], kLog2e, run[e]);
+              A[i][e] = run[e];
             }
-            vt[i] = x;
-          }
-        }
-        if (w4 == 0 && lane < 8) {
-          // gate row 0 now holds the chunk's decay a per channel, row 1 the factor
-          // 2^(decay from the segment start to this chunk) of the held Qh'
-          *reinterpret_cast<float4*>(G + ch0) = make_float4(last[0], last[1], last[2], last[3]);
-          *reinterpret_cast<float4*>(G + 64 + ch0) = make_float4(ex2(a2s[0]), ex2(a2s[1]), ex2(a2s[2]), ex2(a2s[3]));
-        }
+        } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) a2s[e] += last[e];
-        if (tid == 0) ms->fb[st] = fbx ? 1 : 0;
-        fence_proxy_async_smem();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->opready[st]);  // one arrival per channel half
+          for (int i = 3; i >= 0; --i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              run[e] = fmaf(gv[i][e], kLog2e, run[e]);
+              A[i][e] = run[e];
+            }
+        }
       }
+      float incl[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        incl[e] = run[e];
+        if (!rev) {
+          float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
+          if (lane >= 8) incl[e] += x;
+          x = __shfl_up_sync(0xffffffffu, incl[e], 16);
+          if (lane >= 16) incl[e] += x;
+        } else {
+          float x = __shfl_down_sync(0xffffffffu, incl[e], 8);
+          if (lane < 24) incl[e] += x;
+          x = __shfl_down_sync(0xffffffffu, incl[e], 16);
+          if (lane < 16) incl[e] += x;
+        }
+      }
+      float* redh = &ms->red[hh][0][0];  // [4 warps][32 channels] of this channel half
+      if (rev ? lane < 8 : lane >= 24)
+        *reinterpret_cast<float4*>(redh + w4 * 32 + 4 * cc) = make_float4(incl[0], incl[1], incl[2], incl[3]);
+      wg_sync(wg);
+      float off[4], last[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        off[e] = incl[e] - run[e];
+        last[e] = 0.f;
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 t4 = *reinterpret_cast<const float4*>(redh + w * 32 + 4 * cc);
+        const float t[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (rev ? w > w4 : w < w4) off[e] += t[e];
+          last[e] += t[e];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) A[i][e] += off[e];
+      // CUDA-core decision over all 64 channels: each warp covers its half's 32 channels,
+      // the two halves meet at a 256-thread barrier
+      bool exp_unsafe = false;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (-last[e] > fp.max_exp2) exp_unsafe = true;
+      const bool half_unsafe = __any_sync(0xffffffffu, exp_unsafe);
+      if (wtid == 0) ms->fbh[bb][hh] = half_unsafe ? 1 : 0;
+      asm volatile("bar.sync 6, 256;" ::: "memory");
+      const bool fbx = (*(volatile int*)&ms->fbh[bb][0] | *(volatile int*)&ms->fbh[bb][1]) != 0;
+      if (fbx) {
+        // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
+        // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i);
+        // warpgroup hh fills score columns 32hh .. 32hh+31 of its warps' rows.  A goes to
+        // the gate tile so that every thread can read every row and channel.
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
+        if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+        asm volatile("bar.sync 6, 256;" ::: "memory");  // A of both channel halves is in place
+        tc_fence_after();
+        const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
+        float sv[16];
+        for (int x = 0; x < 16; ++x) {
+          const int i = r0 + 8 * ((x & 3) >> 1);
+          const int j = 32 * hh + 8 * (x >> 2) + cq + (x & 1);
+          float acc = 0.f;
+          if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
+            for (int k = 0; k < 64; k += 2) {
+              const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
+              const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
+              acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
+              acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
+            }
+          }
+          sv[x] = acc * 0.125f;
+        }
+        tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU) + 32u * hh, sv);
+        tmem_wait_st();
+        tc_fence_before();
+        asm volatile("bar.sync 6, 256;" ::: "memory");  // raw q / k reads done before the overwrite
+      }
+      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
+      const __half2 eighth = __float2half2_rn(0.125f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = row0 + i;
+        // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
+        const uint32_t off8 = row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
+        uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
+        uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
+        uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
+        uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
+          const float xk0 = fbx ? last[2 * e2] - A0 : -A0;
+          const float xk1 = fbx ? last[2 * e2 + 1] - A1 : -A1;
+          __half2 qh, kh;
+          if constexpr (std::is_same<Tin, __half>::value) {
+            qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
+            kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
+          } else {
+            const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
+            qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
+            kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+          }
+          qw[e2] = h2_bits(qh);
+          kw[e2] = h2_bits(kh);
+        }
+        *reinterpret_cast<uint2*>(sb + off8) = qraw;
+        *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
+      }
+      if constexpr (!std::is_same<Tin, __half>::value) {
+        // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range);
+        // the two warpgroups take alternate 16-byte chunks
+        uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
+#pragma unroll
+        for (int i = tid; i < kTile / 16; i += 2 * kWG) {
+          uint4 x = vt[i];
+          uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = In2<Tin>::unpack(w[e]);
+            w[e] = pack_h2(f.x, f.y);
+          }
+          vt[i] = x;
+        }
+      }
+      if (w4 == 0 && lane < 8) {
+        // gate row 0 now holds the chunk's decay a per channel, row 1 the factor
+        // 2^(decay from the segment start to this chunk) of Qh'
+        *reinterpret_cast<float4*>(G + ch0) = make_float4(last[0], last[1], last[2], last[3]);
+        *reinterpret_cast<float4*>(G + 64 + ch0) = make_float4(ex2(a2s[0]), ex2(a2s[1]), ex2(a2s[2]), ex2(a2s[3]));
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a2s[e] += last[e];
+      if (tid == 0) ms->fb[st] = fbx ? 1 : 0;
+      fence_proxy_async_smem();
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->opready[st]);  // one arrival per channel half
     }
+    if (partial && alive) second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
+
   } else if (warp < 12) {
     // ===================================================================== WG_B: masking, state
     // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
@@ -889,116 +886,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
     const bool rev = fp.rev != 0;
-    float Ls[32];          // fp32 state entries (rows r0 / r1 = key channels)
-    float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1 (HOLD)
-    int slot = 0, n = 0;
+    float Ls[32];                  // fp32 state entries (rows r0 / r1 = key channels)
+    float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1
+    int slot = 0;
     bool alive = true;
-    for (int r = 0; r < rounds && alive; ++r) {
-      const Span sp = round_span(fp, r, seg);
-      float* mine = xcta ? fp.agg + (((size_t)seq * 2 + (r & 1)) * fp.n_s + seg) * (4096 + 64) : nullptr;
-      // The summary slot and the held Qh' set of this round were used by the round two
-      // back: wait until that round's epilogue, which every CTA's scan of that round
-      // precedes, is finished -- also for a round without chunks, whose neutral summary
-      // would otherwise overwrite a slot other CTAs may still be scanning.
-      if (hold && r >= 2 && !wg_wait(wg, wtid, &ms->set_free[r & 1], ph_free(r), ms, hdr, 0x404, slot)) break;
-      if (sp.c1 <= sp.c0) {
-        if (xcta) {  // an empty segment still publishes a neutral summary
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * c + cq), make_float2(0.f, 0.f));
-            __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * c + cq), make_float2(0.f, 0.f));
-          }
-          if ((lane & 3) == 0) {
-            mine[4096 + r0] = 0.f;
-            mine[4096 + r1] = 0.f;
-          }
-          __threadfence();
-          wg_sync(wg);
-          if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
+    for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
+    {  // zero start state of the segment's first chunk (state tile 0, first use)
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      uint4* sz = reinterpret_cast<uint4*>(smem + kOffS);
+      for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
+      fence_proxy_async_smem();
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->sready[0]);
+    }
+    for (int n = 0; n < cnt; ++n) {
+      const int c = sp.c0 + n, st = n % kStages, su = n % kSU;
+      const bool last_chunk = n + 1 == cnt;
+      if (!wg_wait(wg, wtid, &ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400, slot)) { alive = false; break; }
+      tc_fence_after();
+      const bool fbk = ms->fb[st] != 0;
+      const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
+      const float* alast = reinterpret_cast<const float*>(qt + 3 * kTile);
+      const float l0 = alast[r0], l1 = alast[r1];
+      const float dl0 = ex2(l0), dl1 = ex2(l1);
+      const uint32_t sreg = tl + kColSU + 64u * (uint32_t)su;
+      {
+        float u[32];
+        tmem_ld16x256_x8(sreg + kLaneTile1, u);
+        tmem_wait_ld();
+        // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const float d = (x & 2) ? dl1 : dl0;
+          Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
         }
-        continue;
       }
+      a2r0 += l0;
+      a2r1 += l1;
+      if (partial) {
+        // this chunk's Qh' = Qh 2^(A from the segment start) -> its workspace tile (fp16,
+        // the 128-byte-swizzle MMA layout), the A operand of the second phase; read from
+        // the staged Qh before P is signalled (P V's completion frees the stage)
+        const float* eseg = alast + 64;  // gate row 1
+        uint8_t* dst = reinterpret_cast<uint8_t*>(fp.qhp + ((size_t)seq * fp.Nc + c) * 4096);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) Ls[e] = 0.f;
-      a2r0 = a2r1 = 0.f;
-      {  // zero start state for this round's first chunk (its tile's last reader, the
-         // O = Qh S of chunk n-3, completed before chunk n-1's scores were issued)
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        uint4* sz = reinterpret_cast<uint4*>(smem + kOffS + (n % 3) * kTile);
-        for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
-        fence_proxy_async_smem();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->sready[n % 3]);
+        for (int cb = 0; cb < 8; ++cb) {
+          const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
+          const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
+          const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
+          *reinterpret_cast<uint32_t*>(dst + r0 * 128 + o) =
+              h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
+          *reinterpret_cast<uint32_t*>(dst + r1 * 128 + o) =
+              h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
+        }
       }
-      for (int c = sp.c0; c < sp.c1; ++c, ++n) {
-        const int bb = n & 1, st = n % kStages;
-        const bool last_chunk = (c + 1 == sp.c1);
-        if (!wg_wait(wg, wtid, &ms->su_full[bb], ph_of(n), ms, hdr, 0x400, slot)) { alive = false; break; }
-        tc_fence_after();
-        const bool fbk = ms->fb[st] != 0;
-        const float* alast = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes + 3 * kTile);
-        const float l0 = alast[r0], l1 = alast[r1];
-        const float dl0 = ex2(l0), dl1 = ex2(l1);
-        {
-          float u[32];
-          tmem_ld16x256_x8(tl + kColSU + 64u * bb + kLaneTile1, u);
-          tmem_wait_ld();
-          // state rows r0 / r1: S <- 2^a (S + U')   (CUDA-core chunks: S <- 2^a S + U)
+      // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
+      // the A operand of P V.  A rows are read from the lanes of the output rows, so P
+      // goes to the lane tile of the chunk's output region (tile 1: over U', already
+      // loaded).  Register 2c+q of the 16x128b shape is row r0 + 8q, column 4c + lane%4,
+      // i.e. the score pair (8c + cq, 8c + cq + 1) of that row.
+      const uint32_t pdst = sreg + ((n & 1) ? kLaneTile1 : 0u);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float d = (x & 2) ? dl1 : dl0;
-            Ls[x] = fbk ? fmaf(d, Ls[x], u[x]) : d * (Ls[x] + u[x]);
-          }
-        }
-        a2r0 += l0;
-        a2r1 += l1;
-        if (hold) {
-          // (read from the staged Qh before P is signalled: P V's completion frees the stage)
-          // held Qh' = Qh 2^(A from the segment start) of this chunk -> tensor memory, in the
-          // lane tile of its held output (16x128b: register 2c+q is row r0 + 8q, channels
-          // 8c + cq, 8c + cq + 1)
-          const int g = c - sp.c0;
-          const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
-          const float* eseg = reinterpret_cast<const float*>(qt + 3 * kTile) + 64;  // gate row 1
-          uint32_t hw[16];
-#pragma unroll
-          for (int cb = 0; cb < 8; ++cb) {
-            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
-            const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
-            const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
-            hw[2 * cb] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
-            hw[2 * cb + 1] = h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
-          }
-          tmem_st16x128_x8(tl + kColHQ + (kSetCols / 2) * (uint32_t)(r & 1) + 32u * (uint32_t)(g >> 1) +
-                               ((g & 1) ? kLaneTile1 : 0u),
-                           hw);
-        } else if (segm && seg > 0) {
-          // segmented: this chunk's Qh' = Qh 2^(A from the segment start) -> its workspace
-          // tile (fp16, the 128-byte-swizzle MMA layout), the A operand of the second phase
-          const uint8_t* qt = smem + kOffStage + st * kStageBytes;
-          const float* eseg = reinterpret_cast<const float*>(qt + 3 * kTile) + 64;  // gate row 1
-          uint8_t* dst = reinterpret_cast<uint8_t*>(fp.qhp + ((size_t)seq * fp.Nc + c) * 4096);
-#pragma unroll
-          for (int cb = 0; cb < 8; ++cb) {
-            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
-            const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
-            const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
-            *reinterpret_cast<uint32_t*>(dst + r0 * 128 + o) =
-                h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
-            *reinterpret_cast<uint32_t*>(dst + r1 * 128 + o) =
-                h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
-          }
-        }
-        // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
-        // the A operand of P V.  A rows are read from the lanes of the output rows, so P
-        // goes to the lane tile of the chunk's output region (tile 1: over U', already
-        // loaded).  Register 2c+q of the 16x128b shape is row r0 + 8q, column 4c + lane%4,
-        // i.e. the score pair (8c + cq, 8c + cq + 1) of that row.
-        const uint32_t pdst = tl + kColSU + 64u * bb + (((hold ? (c - sp.c0) : n) & 1) ? kLaneTile1 : 0u);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {  // score columns 32hf .. 32hf+31 -> P columns 16hf .. 16hf+15
+      for (int hf = 0; hf < 2; ++hf) {  // score columns 32hf .. 32hf+31 -> P columns 16hf .. 16hf+15
         float sc[16];
-        tmem_ld16x256_x4(tl + kColSU + 64u * bb + 32u * hf, sc);
+        tmem_ld16x256_x4(sreg + 32u * hf, sc);
         tmem_wait_ld();
         uint32_t pw[8];
 #pragma unroll
@@ -1025,75 +977,74 @@ __global__ void __launch_bounds__(kThreads, 1)
           pw[2 * cl + 1] = pack_h2(x2, x3);
         }
         tmem_st16x128_x4(pdst + 16u * hf, pw);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->pready[bb]);
-        if (!last_chunk) {
-          // the next chunk's start state (three tiles: the one written here was last read
-          // by O = Qh S of chunk n-2, complete since chunk n's scores were issued)
-          uint8_t* srow0 = smem + kOffS + ((n + 1) % 3) * kTile + r0 * 128;
-          uint8_t* srow1 = srow0 + 8 * 128;
-#pragma unroll
-          for (int cb = 0; cb < 8; ++cb) {
-            const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;
-            sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
-            sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
-          }
-          fence_proxy_async_smem();
-        }
-        wg_sync(wg);
-        if (wtid == 0 && !last_chunk) mbar_arrive(&ms->sready[(n + 1) % 3]);
       }
-      if (!alive) break;
-      // the Qh' tiles written above are read back by bulk copy (async proxy)
-      if (segm && seg > 0) asm volatile("fence.proxy.async.global;" ::: "memory");
-      if (xcta) {
-        // segment summary of this round: U_seg = local end state, its log2 decay
+      tmem_wait_st();
+      tc_fence_before();
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->pready[su]);
+      if (!last_chunk) {
+        // the next chunk's start state, into state tile (n+1) % 3 once O = Qh S of chunk
+        // n-2, its last reader, has completed
+        const int t = (n + 1) % 3;
+        if (!wg_wait(wg, wtid, &ms->sfree[t], ph_rel<3>(n + 1), ms, hdr, 0x401, slot)) { alive = false; break; }
+        uint8_t* srow0 = smem + kOffS + t * kTile + r0 * 128;
+        uint8_t* srow1 = srow0 + 8 * 128;
 #pragma unroll
         for (int cb = 0; cb < 8; ++cb) {
-          __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb], Ls[4 * cb + 1]));
-          __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+          const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;
+          sts32(srow0 + o, pack_h2(Ls[4 * cb], Ls[4 * cb + 1]));
+          sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
         }
-        if ((lane & 3) == 0) {
-          mine[4096 + r0] = a2r0;
-          mine[4096 + r1] = a2r1;
-        }
-        __threadfence();
+        fence_proxy_async_smem();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->agg_pub[r & 1]);
+        if (wtid == 0) mbar_arrive(&ms->sready[t]);
       }
     }
+    if (segm && alive) {
+      // the Qh' tiles written above are read back by bulk copy (async proxy)
+      if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
+      // segment summary: U_seg = local end state, its log2 decay
+      float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * (4096 + 64);
+#pragma unroll
+      for (int cb = 0; cb < 8; ++cb) {
+        __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb], Ls[4 * cb + 1]));
+        __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+      }
+      if ((lane & 3) == 0) {
+        mine[4096 + r0] = a2r0;
+        mine[4096 + r1] = a2r1;
+      }
+      __threadfence();
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->agg_pub);
+      if (partial) second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
+    }
   } else if (warp < 16) {
-    // ===================================================================== WG_C: epilogue, HOLD round end
+    // ===================================================================== WG_C: epilogue, scan
     const int wg = 3, wtid = tid - 3 * kWG, wq = warp & 3;
     const int trow = wq * 16 + (lane & 15);
     const int tsel = lane >> 4;  // lane tile: chunk 2m (0) or 2m+1 (1) of an output pair
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
-    bool alive_c = true;
-    if (!hold) {
-      // STREAM: the whole sequence; SEGMENTED: this segment's run, whose outputs (but
-      // segment 0's) are partial -- fp16 rows of the workspace, corrected in phase two
-      const Span sp0 = round_span(fp, 0, seg);
-      const int cnt = sp0.c1 - sp0.c0;
-      const bool partial = segm && seg > 0;
+    bool alive = true;
+    {
+      // this CTA's chunks; in a segment s > 0 the outputs are partial: fp16 rows of the
+      // workspace, completed in the second phase
       const int pairs = (cnt + 1) / 2;
       for (int pr = 0; pr < pairs; ++pr) {
-        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_of(pr), ms, hdr, 0x500, slot)) { alive_c = false; break; }
+        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_use<2>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
         const int ci = 2 * pr + tsel;
-        const long long s = (long long)(sp0.c0 + ci) * kChunk + (fp.rev ? 63 - trow : trow);
+        const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - trow : trow);
         const bool valid = ci < cnt && s < L;
+        const uint32_t src = tl + kColO + 64u * (uint32_t)(pr & 1);
         if (partial) {
-          uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp0.c0 + ci) * 4096) + trow * 128
+          uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp.c0 + ci) * 4096) + trow * 128
                               : nullptr;
-          epilogue_rows<__half>(tl + kColO + 64u * (uint32_t)(pr & 1), od, wstage, lane, nonfinite);
+          epilogue_rows<__half>(src, od, wstage, lane, nonfinite);
         } else {
-          epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)(pr & 1), out_row<Tout>(p, b, h, valid, s), wstage, lane,
-                              nonfinite);
+          epilogue_rows<Tout>(src, out_row<Tout>(p, b, h, valid, s), wstage, lane, nonfinite);
         }
         tc_fence_before();
         wg_sync(wg);
@@ -1102,15 +1053,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the O_local rows written above are read back by bulk copy (async proxy)
       if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-    if (xcta && alive_c) {
-      // Round-end scan of the segment summaries.  This CTA owns state entries
-      // [4 f0, 4 f1) (float4 units f, F of them).  Threads split into nB blocks of bs
-      // consecutive segments x FP float4 columns (nB * FP <= 128): a thread loads its
-      // block's summaries for its f all at once (consecutive threads read consecutive
-      // float4s), composes them sequentially, and the block compositions are exchanged
-      // through shared memory; each thread then walks its segments again from its
-      // block's carry-in, writing each segment's start state (fp16, MMA layout).  The
-      // carry (state entering the round, fp32) lives in the workspace between rounds.
+    if (segm && alive) {
+      // Scan of the segment summaries.  This CTA owns state entries [4 f0, 4 f1) (float4
+      // units f, F of them).  Threads split into nB blocks of bs consecutive segments x FP
+      // float4 columns (nB * FP <= 128): a thread loads its block's summaries for its f
+      // all at once (consecutive threads read consecutive float4s), composes them
+      // sequentially, and the block compositions are exchanged through shared memory;
+      // each thread then walks its segments again from its block's carry-in, writing
+      // each segment's start state (fp16, MMA layout).
       const int ns = fp.n_s;
       const int f0 = (int)((long long)seg * 1024 / ns), f1 = (int)((long long)(seg + 1) * 1024 / ns);
       const int F = f1 - f0;
@@ -1122,25 +1072,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bi = wtid / FP, fi = wtid % FP;
       const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
       unsigned int* ctr = fp.counters + (size_t)seq * 2;
-      const float* aggs0 = fp.agg + (size_t)seq * 2 * ns * (4096 + 64);
+      const float* aggs = fp.agg + (size_t)seq * ns * (4096 + 64);
       uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
-      float4* carry = reinterpret_cast<float4*>(fp.carry + (size_t)seq * 4096);
       float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
       float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
-      const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
-      const uint32_t s_base = smem_u32(smem);
-      for (int r = 0; r < rounds; ++r) {
-        const int sig = r & 1;
-        const Span sp = round_span(fp, r, seg);
-        const float* aggs = aggs0 + (size_t)sig * ns * (4096 + 64);
-        if (!wg_wait(wg, wtid, &ms->agg_pub[sig], ph_of(r), ms, hdr, 0x600, slot)) break;
-        const unsigned int target = (unsigned int)(r + 1) * (unsigned int)ns;
-        bool ok0 = true;
+      const unsigned int target = (unsigned int)ns;
+      bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
+      if (ok0) {
         if (wtid == 0) {
           red_release_add(ctr, 1u);
           ok0 = wait_counter(ctr, target, ms, hdr, 0x601);
         }
-        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
+        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
+      }
+      if (ok0) {
         for (int base = f0; base < f1; base += FP) {
           const int f = base + fi;
           const bool act = bi < nB && f < f1;
@@ -1148,7 +1093,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4 u[kScanBlock];
           float dd[kScanBlock];
           float4 X = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (act && r > 0) X = __ldcg(carry + f);
 #pragma unroll
           for (int j = 0; j < kScanBlock; ++j) {
             const int sg = s_lo + j;
@@ -1192,100 +1136,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 fmaf(dd[j], X.w, u[j].w));
               }
             }
-            if (s_hi == ns) __stcg(carry + f, X);  // the last block's end state enters the next round
           }
           if (nB > 1) wg_sync(wg);  // the exchange slots are reused by the next column pass
         }
         __threadfence();
         wg_sync(wg);
-        ok0 = true;
         if (wtid == 0) {
           red_release_add(ctr + 1, 1u);
           ok0 = wait_counter(ctr + 1, target, ms, hdr, 0x602);
         }
-        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
-        {  // my segment's start state -> shared memory (already in the MMA layout)
-          const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
-          uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
-          for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
-        }
+        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
+      }
+      if (ok0 && partial) {
+        // this segment's start state -> shared memory (already in the MMA layout), then
+        // the second phase on all four warpgroups
+        const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
+        uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
+        for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
         fence_proxy_async_smem();
         wg_sync(wg);
-        if (segm) {
-          // ---- second phase: outputs of segment s > 0 = O_local + Qh' S_start.  Chunk
-          // pairs: Qh' and O_local tiles (2 x 8 KB each, consecutive in the workspace) come
-          // back by bulk copy into the free staging buffers; one M = 128 MMA per pair
-          // puts chunk 2m's rows in lanes 0-63 and chunk 2m+1's in lanes 64-127.
-          if (seg > 0) {
-            const int cnt = sp.c1 - sp.c0, npairs = (cnt + 1) / 2;
-            const uint32_t id_128 = idesc_f16(0, 128, 64, 0, 1);
-            auto issue_loads = [&](int m2) {
-              const int sl = m2 & 3;
-              uint8_t* sbuf = smem + kOffStage + sl * kStageBytes;
-              const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
-              mbar_arrive_expect_tx(&ms->p2_full[sl], (uint32_t)(2 * nb * 8192));
-              bulk_load(sbuf, fp.qhp + ((size_t)seq * fp.Nc + c) * 4096, (uint32_t)(nb * 8192), &ms->p2_full[sl]);
-              bulk_load(sbuf + 16384, fp.olc + ((size_t)seq * fp.Nc + c) * 4096, (uint32_t)(nb * 8192), &ms->p2_full[sl]);
-            };
-            if (wtid == 0)
-              for (int m2 = 0; m2 < npairs && m2 < 4; ++m2) issue_loads(m2);
-            for (int m2 = 0; m2 < npairs; ++m2) {
-              const int sl = m2 & 3;
-              const uint32_t par = (uint32_t)(m2 >> 2) & 1u;
-              if (!wg_wait(wg, wtid, &ms->p2_full[sl], par, ms, hdr, 0x605, slot)) break;
-              if (wtid == 0) {
-                tc_fence_after();
-                const uint32_t a0 = s_base + kOffStage + sl * kStageBytes;
-                for (int k = 0; k < 4; ++k)
-                  mma_f16(tmem + 64u * sl, sw128_desc(a0 + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_128, k > 0);
-                mma_commit(&ms->p2_mma[sl]);
-              }
-              if (!wg_wait(wg, wtid, &ms->p2_mma[sl], par, ms, hdr, 0x606, slot)) break;
-              tc_fence_after();
-              const int ci = 2 * m2 + (wq >> 1), row = 32 * (wq & 1) + lane;
-              const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
-              const uint8_t* olc_rows = smem + kOffStage + sl * kStageBytes + 16384 + (wq >> 1) * 8192 + 32 * (wq & 1) * 128;
-              epilogue_rows_add<Tout>(tl + 64u * sl, out_row<Tout>(p, b, h, ci < cnt && s < L, s), olc_rows, wstage, lane,
-                                      nonfinite);
-              tc_fence_before();
-              wg_sync(wg);  // the pair's buffers are read out
-              if (wtid == 0 && m2 + 4 < npairs) issue_loads(m2 + 4);
-            }
-          }
-          continue;
-        }
-        const int G = sp.c1 - sp.c0;
-        ok0 = true;
-        if (wtid == 0) {
-          // held outputs of this round += (Q 2^(A_seg)) S_segment_start, once their own
-          // MMAs have completed
-          if (G > 0) ok0 = wait_bar(&ms->round_done[sig], ph_of(r), ms, hdr, 0x604);
-          if (ok0) {
-            tc_fence_after();
-            for (int g = 0; g < G; ++g) {
-              const uint32_t d_o = tmem + kColO + kSetCols * sig + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
-              const uint32_t a_h = tmem + kColHQ + (kSetCols / 2) * sig + 32u * (uint32_t)(g >> 1) +
-                                   ((g & 1) ? kLaneTile1 : 0u);  // held Qh', same lanes as the output
-              for (int k = 0; k < 4; ++k)
-                mma_f16_ta(d_o, a_h + 8 * k, sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
-            }
-            mma_commit(&ms->corr_done[sig]);
-          }
-        }
-        if (!wg_agree(wg, wtid, ok0, ms, slot)) break;
-        if (!wg_wait(wg, wtid, &ms->corr_done[sig], ph_of(r), ms, hdr, 0x603, slot)) break;
-        tc_fence_after();
-        // epilogue of the held chunks: pair m holds chunks 2m (lane tile 0) and 2m+1 (lane
-        // tile 1)
-        for (int m2 = 0; m2 < (G + 1) / 2; ++m2) {
-          const int gi = 2 * m2 + tsel;
-          const long long s = (long long)(sp.c0 + gi) * kChunk + (fp.rev ? 63 - trow : trow);
-          epilogue_rows<Tout>(tl + kColO + kSetCols * sig + 64u * (uint32_t)m2, out_row<Tout>(p, b, h, gi < G && s < L, s),
-                              wstage, lane, nonfinite);
-        }
-        tc_fence_before();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->set_free[sig]);
+        if (wtid == 0) mbar_arrive(&ms->p2_go);
+        second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
       }
     }
   }
@@ -1298,7 +1169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
   // last CTA out resets this call's counters: the workspace is ready for the next call
-  if (xcta && tid == 0) {
+  if (segm && tid == 0) {
     __threadfence();
     const unsigned int done = atomicAdd(&hdr->ticket, 1u);
     if (done == (unsigned int)fp.grid - 1) {
@@ -1352,35 +1223,25 @@ bool make_chunk_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
 }
 
 struct Plan {
-  int mode, n_seq, n_s, rounds, grid;
+  int mode, n_seq, n_s, grid;
 };
 
 // Length-aware plan: many sequences -> one CTA each (STREAM); few sequences -> each is
-// split over n_s CTAs with about kHeldPerSet chunks per CTA per round (HOLD).
+// split into n_s segments, one CTA each, so that the launch fills the SMs (SEGMENTED).
 Plan make_plan(const Problem& p, int sms) {
   Plan pl;
   pl.n_seq = p.B * p.heads;
   const int Nc = p.n_chunks();
-  const int cap = sms < (int)kMaxHoldSegments ? sms : (int)kMaxHoldSegments;
+  const int cap = sms < (int)kMaxSegCtas ? sms : (int)kMaxSegCtas;
   if (pl.n_seq * 2 > cap || Nc <= 1) {
     pl.mode = 0;
     pl.n_s = 1;
-    pl.rounds = 1;
     pl.grid = pl.n_seq;
   } else {
     pl.mode = 1;
     pl.n_s = cap / pl.n_seq;
     if (pl.n_s > Nc) pl.n_s = Nc;
-    const int per_round = pl.n_s * kHeldPerSet;
-    pl.rounds = (Nc + per_round - 1) / per_round;
     pl.grid = pl.n_seq * pl.n_s;
-    // GTR_FUSED_MODE=2: one contiguous run per segment, corrected in a second phase
-    if (const char* e = getenv("GTR_FUSED_MODE")) {
-      if (e[0] == '2') {
-        pl.mode = 2;
-        pl.rounds = 1;
-      }
-    }
   }
   return pl;
 }
@@ -1398,9 +1259,10 @@ int device_sms() {
   return sms[dev];
 }
 
-size_t hold_segments(const Problem& p) {
+// Segment summaries and start states the workspace holds room for (0: STREAM only).
+size_t seg_capacity(const Problem& p) {
   const size_t n_seq = (size_t)p.B * p.heads;
-  return n_seq * 2 <= kMaxHoldSegments ? n_seq * (kMaxHoldSegments / n_seq) : 0;
+  return n_seq * 2 <= kMaxSegCtas ? n_seq * (kMaxSegCtas / n_seq) : 0;
 }
 
 template <typename Tin, typename Tout>
@@ -1418,7 +1280,6 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   if (force_mode == 0) {
     pl.mode = 0;
     pl.n_s = 1;
-    pl.rounds = 1;
     pl.grid = pl.n_seq;
   }
   FusedParams fp;
@@ -1428,12 +1289,10 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.counters = w.counters;
   fp.agg = w.agg;
   fp.sstart = w.sstart;
-  fp.carry = w.carry;
   fp.qhp = w.qhp;
   fp.olc = w.olc;
   fp.n_seq = pl.n_seq;
   fp.n_s = pl.n_s;
-  fp.rounds = pl.rounds;
   fp.Nc = p.n_chunks();
   fp.mode = pl.mode;
   fp.grid = pl.grid;
@@ -1464,7 +1323,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = pl.mode != 0 ? 1 : 0;  // the CTAs of a sequence wait on one another
+  attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;  // the CTAs of a sequence wait on one another
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;
@@ -1473,23 +1332,21 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
 
 }  // namespace
 
-// Per-chunk tiles of the segmented mode's second phase (Qh' and O_local, fp16): only when
-// sequences are split over CTAs.
+// Per-chunk tiles of the second phase (Qh' and O_local, fp16): only when sequences may
+// be split over CTAs.
 size_t segmented_tile_bytes(const Problem& p) {
-  return hold_segments(p) ? (size_t)p.B * p.heads * p.n_chunks() * 4096 * sizeof(uint16_t) : 0;
+  return seg_capacity(p) ? (size_t)p.B * p.heads * p.n_chunks() * 4096 * sizeof(uint16_t) : 0;
 }
 
 size_t fused_workspace_bytes(const Problem& p) {
-  const size_t segs = hold_segments(p);
-  const size_t carry_seqs = segs ? (size_t)p.B * p.heads : 0;
-  size_t b = sizeof(WsHeader) + kCounterBytes + 2 * segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t) +
-             carry_seqs * 4096 * sizeof(float);
+  const size_t segs = seg_capacity(p);
+  size_t b = sizeof(WsHeader) + kCounterBytes + segs * (4096 + 64) * sizeof(float) + segs * 4096 * sizeof(uint16_t);
   b = (b + 1023) & ~size_t(1023);  // 1 KB-aligned tiles for the bulk copies
   return b + 2 * segmented_tile_bytes(p);
 }
 
 FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
-  const size_t segs = hold_segments(p);
+  const size_t segs = seg_capacity(p);
   FusedWorkspace w;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   w.hdr = reinterpret_cast<WsHeader*>(base);
@@ -1497,11 +1354,9 @@ FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
   w.counters = reinterpret_cast<unsigned int*>(base);
   base += kCounterBytes;
   w.agg = reinterpret_cast<float*>(base);
-  base += 2 * segs * (4096 + 64) * sizeof(float);
+  base += segs * (4096 + 64) * sizeof(float);
   w.sstart = reinterpret_cast<uint16_t*>(base);
   base += segs * 4096 * sizeof(uint16_t);
-  w.carry = reinterpret_cast<float*>(base);
-  base += (hold_segments(p) ? (size_t)p.B * p.heads : 0) * 4096 * sizeof(float);
   const size_t used = (size_t)(base - reinterpret_cast<uint8_t*>(ws));
   base = reinterpret_cast<uint8_t*>(ws) + ((used + 1023) & ~size_t(1023));
   const size_t tiles = segmented_tile_bytes(p);
