@@ -30,7 +30,7 @@
 // Qh' S_start(s) to O_local, one M = 128 MMA per chunk pair, spread over all four
 // of its warpgroups.
 //
-// Warp roles (608 threads):
+// Warp roles (640 threads):
 //   warps 0-7   WG_A  two warpgroups, one per half of the key channels: cumulative
 //               gates, Qh / Kh in place, CUDA-core scores
 //   warps 8-11  WG_B  score masking, fp32 state update, Qh' (16-lane tensor-memory
@@ -38,7 +38,8 @@
 //   warps 12-15 WG_C  epilogue; SEGMENTED: summary scan
 //   warps 16-17 producer: TMA boxes, or cp.async row copies (direction remap,
 //               128-byte-swizzled placement, zero fill past the sequence end)
-//   warp 18     tcgen05 MMA issuer and tensor-memory owner
+//   warp 18     tcgen05 MMA issuer of the scores and U' (in chunk order), tensor-memory owner
+//   warp 19     tcgen05 MMA issuer of the outputs O = Qh S, O += P V (in chunk order)
 //   SEGMENTED second phase: warpgroups 0-3 (warps 0-15) each take every fourth pair
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -58,9 +59,11 @@ using namespace sm100;
 
 constexpr int kStages = 4;          // staging depth (chunks in flight)
 constexpr int kSU = 4;              // score / U' regions in tensor memory (chunks in flight)
-constexpr int kThreads = 608;
-constexpr int kProducerThreads = 64;
-constexpr int kMmaWarp = 18;
+constexpr int kThreads = 640;
+constexpr int kProducerThreads = 32;  // cp.async copies (warp 16)
+constexpr int kQhWarp = 17;           // Qh' tiles of segments s > 0
+constexpr int kMmaWarp = 18;  // stage 1 (scores, U'); tensor-memory owner
+constexpr int kOutWarp = 19;  // stages 2a / 2b (outputs)
 constexpr int kWG = 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -70,11 +73,12 @@ constexpr int kTile = 8192;
 constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
 constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V, G
 constexpr int kOffStage = 0;
-constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [3] chunk-start states
-constexpr int kOffSst = kOffS + 3 * kTile;                 // segment start state
-constexpr int kOffStg = kOffSst + kTile;                   // output staging, 4 warps x 32 rows x 128 B
+constexpr int kNS = 5;                                     // chunk-start state tiles
+constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [kNS] chunk-start states
+constexpr int kOffSst = kOffS;                             // segment start state (after the chunks: over state tile 0)
+constexpr int kOffStg = kOffS + kNS * kTile;               // output staging, 4 warps x 32 rows x 128 B
 constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
-constexpr int kMiscBytes = 2048;
+constexpr int kMiscBytes = 4096;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 // second phase, pair slot q (one per warpgroup) in staging buffer q: Qh' of the pair
 // (16 KB, the A operand; then the warps' fp32 output staging) and O_local (16 KB)
@@ -122,16 +126,17 @@ struct Misc {
   // MMA warp, so a two-deep ring could complete a phase twice before it is observed
   uint64_t opready[kStages];
   uint64_t su_full[kSU], su_free[kSU], pready[kSU];  // per score / U' region
-  uint64_t sready[3], sfree[3];                      // per chunk-start state tile
+  uint64_t sready[kNS];                              // per chunk-start state tile
+  uint64_t qdone[kStages];                           // Qh' of the staged chunk copied out
   uint64_t o_full[2], o_free[2];                     // per output pair
-  uint64_t agg_pub, p2_go, mma_final;
+  uint64_t agg_pub, p2_go, mma_final[2];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
   uint32_t tmem_base;
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
-  int fbh[2][2];         // chunk parity x channel half -> CUDA-core scores needed
   int fb[kStages];       // stage -> scores from the CUDA cores
-  alignas(16) float red[2][4][32];  // WG_A cumsum: per channel half and warp, channel totals
+  alignas(16) float red[2][2][4][32];  // WG_A cumsum: per warpgroup, channel half and warp, channel totals
+  alignas(16) float eseg[64];          // Qh' warp: 2^(decay from the segment start) per channel
   int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
 };
 // The in-chunk log2 decay per channel (a) of a staged chunk is kept in row 0 of its
@@ -162,6 +167,24 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr
   while (true) {
     if (*(volatile int*)&ms->abort) return false;
     if (mbar_wait_sleep(bar, parity, 1000000u)) return true;
+    if (globaltimer() - t0 > 1000000000ull) {
+      record_error(hdr, GTR_ERR_TIMEOUT, where);
+      *(volatile int*)&ms->abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait by polling (no suspension), for the MMA-issuing threads: they react to a
+// completed phase at once.
+__device__ bool wait_spin(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+  for (int i = 0; i < 64; ++i)
+    if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test(bar, parity)) return true;
+    if (*(volatile int*)&ms->abort) return false;
     if (globaltimer() - t0 > 1000000000ull) {
       record_error(hdr, GTR_ERR_TIMEOUT, where);
       *(volatile int*)&ms->abort = 1;
@@ -208,6 +231,20 @@ __device__ bool wg_wait(int wg, int wtid, uint64_t* bar, uint32_t parity, Misc* 
   slot ^= 1;
   if (go) (void)mbar_try_wait(bar, parity);
   return go;
+}
+
+// AND of a predicate over the 128 threads of warpgroup wg (named barrier wg + 1).
+__device__ __forceinline__ bool wg_all(int wg, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(wg + 1)
+      : "memory");
+  return r != 0;
 }
 
 __device__ bool wg_agree(int wg, int wtid, bool ok0, Misc* ms, int& slot) {
@@ -393,6 +430,16 @@ __device__ __forceinline__ uint32_t ph_rel(int n) { return ((uint32_t)(n / depth
 // by bulk copy into staging buffer q; one M = 128 MMA puts chunk 2m's rows in lanes
 // 0-63 and chunk 2m+1's in lanes 64-127 of tensor-memory slot q; warp wq of the group
 // takes lanes 32wq .. 32wq+31 (chunk 2m + wq/2, rows 32(wq%2) ..).
+// Bulk copies of pair m2's Qh' and O_local tiles into staging buffer q (second phase).
+__device__ __forceinline__ void p2_load(const FusedParams& fp, Misc* ms, uint8_t* smem, int seq, Span sp, int q, int m2) {
+  const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
+  const size_t t0 = ((size_t)seq * fp.Nc + c) * 4096;
+  uint8_t* sbuf = smem + kOffStage + q * kStageBytes;
+  mbar_arrive_expect_tx(&ms->p2_full[q], (uint32_t)(2 * nb * kTile));
+  bulk_load(sbuf, fp.qhp + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
+  bulk_load(sbuf + kP2Olc, fp.olc + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
+}
+
 template <typename Tout>
 __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem, uint32_t tmem, int q,
                              int wtid, int lane, int seq, int b, int h, Span sp, int& slot, float& nf) {
@@ -407,13 +454,7 @@ __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uin
   const uint32_t dq = tmem + 64u * (uint32_t)q;
   int u = 0;
   for (int m2 = q; m2 < npairs; m2 += 4, ++u) {
-    const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
-    if (wtid == 0) {
-      const size_t t0 = ((size_t)seq * fp.Nc + c) * 4096;
-      mbar_arrive_expect_tx(&ms->p2_full[q], (uint32_t)(2 * nb * kTile));
-      bulk_load(sbuf, fp.qhp + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
-      bulk_load(sbuf + kP2Olc, fp.olc + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
-    }
+    if (wtid == 0 && u > 0) p2_load(fp, ms, smem, seq, sp, q, m2);  // (the first pair's load is issued early)
     if (!wg_wait(q, wtid, &ms->p2_full[q], (uint32_t)u & 1u, ms, hdr, 0x710u + q, slot)) return;
     if (wtid == 0) {
       tc_fence_after();
@@ -436,7 +477,7 @@ __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uin
   }
 }
 
-template <typename Tin, typename Tout>
+template <typename Tin, typename Tout, bool kRev>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_gla_kernel(const __grid_constant__ FusedParams fp) {
   extern __shared__ uint8_t smem_raw[];
@@ -461,18 +502,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&ms->full[i], fp.tma ? 1 : kProducerThreads);
       mbar_init(&ms->empty[i], 1);
-      mbar_init(&ms->opready[i], 2);  // one arrival per channel half
+      mbar_init(&ms->opready[i], 4);  // every warp of the WG_A warpgroup that builds the chunk
+      mbar_init(&ms->qdone[i], 1);
       ms->fb[i] = 0;
     }
     for (int i = 0; i < kSU; ++i) {
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
-      mbar_init(&ms->pready[i], 1);
+      mbar_init(&ms->pready[i], 4);  // every WG_B warp
     }
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&ms->sready[i], 1);
-      mbar_init(&ms->sfree[i], 1);
-    }
+    for (int i = 0; i < kNS; ++i) mbar_init(&ms->sready[i], 4);  // every WG_B warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
@@ -481,9 +520,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->p2_full[i], 1);
       mbar_init(&ms->p2_mma[i], 1);
     }
-    mbar_init(&ms->agg_pub, 1);
+    mbar_init(&ms->agg_pub, partial ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
     mbar_init(&ms->p2_go, 1);
-    mbar_init(&ms->mma_final, 1);
+    mbar_init(&ms->mma_final[0], 1);
+    mbar_init(&ms->mma_final[1], 1);
     ms->abort = 0;
     for (int i = 0; i < 4; ++i) ms->go[i][0] = ms->go[i][1] = 0;
     fence_mbar_init();
@@ -497,18 +537,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
 
-  if (warp == 16 || warp == 17) {
+  if (warp == 16) {
     // ===================================================================== producer
     // Staged chunk row r holds scan position c*64 + r, or c*64 + 63 - r for the reversed
     // directions (right-to-left, bottom-to-top), where a chunk is stored in memory order.
-    const int pt = tid - 16 * 32;  // 0..63
+    // A staging buffer is refilled once the P V of its previous chunk has completed and,
+    // in a segment s > 0, that chunk's Qh' has been copied out.
+    auto stage_free = [&](int n, int st) -> bool {
+      if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) return false;
+      return !partial || wait_bar(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
+    };
     if (fp.tma) {
       // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
       // plain); rows past the sequence end arrive zero-filled.
-      if (pt == 0) {
+      if (lane == 0) {
         for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
           const int st = n % kStages;
-          if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) break;
+          if (!stage_free(n, st)) break;
           uint8_t* sb = smem + kOffStage + st * kStageBytes;
           mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);
           const long long s0 = (long long)c * kChunk;
@@ -536,35 +581,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      // Per chunk, thread t first resolves the grid cell of scan position c*64 + t (the
-      // direction remap) into a shared table; then the 64 threads copy the tiles with
-      // whole 128-byte rows per group of 8 threads (Q, K, V: placed in the 128-byte-swizzle
-      // layout) and 256-byte gate rows per group of 16, so each warp-wide copy touches
-      // only 4 (2) full lines.  Rows past the sequence end are zero-filled (source size 0).
+      // Per chunk, lane t first resolves the grid cells of scan positions c*64 + t and
+      // c*64 + 32 + t (the direction remap) into a shared table; then the warp copies the
+      // tiles with whole 128-byte rows per group of 8 lanes (Q, K, V: placed in the
+      // 128-byte-swizzle layout) and 256-byte gate rows per group of 16, so each copy
+      // instruction touches only 4 (2) full lines.  Rows past the sequence end are
+      // zero-filled (source size 0).
       const uint8_t* gq = reinterpret_cast<const uint8_t*>(p.q);
       const uint8_t* gk = reinterpret_cast<const uint8_t*>(p.k);
       const uint8_t* gv = reinterpret_cast<const uint8_t*>(p.v);
       const uint8_t* gg = reinterpret_cast<const uint8_t*>(p.log_gamma);
-      const int j8 = pt & 7, rq = pt >> 3;     // 16-byte column, row within a group of 8
-      const int j16 = pt & 15, rg = pt >> 4;   // gate rows: 16-byte column, row within 4
-      const int srow = fp.rev ? 63 - pt : pt;  // staged row of scan position c*64 + pt
+      const int j8 = lane & 7, rq = lane >> 3;     // 16-byte column, row within a group of 4
+      const int j16 = lane & 15, rg = lane >> 4;   // gate rows: 16-byte column, row within 2
       for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
         const int st = n % kStages;
         int* rows = ms->rowoff[n & 1];
-        {
-          const long long s = (long long)c * kChunk + pt;
-          rows[srow] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
-        }
-        int ok = 0;
-        if (lane == 0) ok = wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100);
-        bool stop = !__shfl_sync(0xffffffffu, ok, 0);
-        asm volatile("bar.sync 5, 64;" ::: "memory");  // the row table is complete
-        if (*(volatile int*)&ms->abort) stop = true;
-        if (stop) break;
-        const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int row = 8 * it + rq;
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int pt = lane + 32 * hlf;
+          const long long s = (long long)c * kChunk + pt;
+          rows[kRev ? 63 - pt : pt] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
+        }
+        __syncwarp();
+        int ok = 0;
+        if (lane == 0) ok = stage_free(n, st) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // (the row table is complete, too)
+        const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+          const int row = 4 * it + rq;
           const int cell = rows[row];
           const uint32_t nb = cell >= 0 ? 16u : 0u;
           const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
@@ -573,9 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async16(dst + kTile, gk + src, nb);
           cp_async16(dst + 2 * kTile, gv + src, nb);
         }
-#pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const int row = 4 * it + rg;
+#pragma unroll 4
+        for (int it = 0; it < 32; ++it) {
+          const int row = 2 * it + rg;
           const int cell = rows[row];
           const uint32_t nb = cell >= 0 ? 16u : 0u;
           cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
@@ -586,273 +631,300 @@ __global__ void __launch_bounds__(kThreads, 1)
       // copies already issued must land before this CTA's shared memory is released
       asm volatile("cp.async.wait_all;" ::: "memory");
     }
+  } else if (warp == kQhWarp) {
+    // ===================================================================== Qh' tiles
+    // Segment s > 0: per chunk, Qh' = Qh 2^(A from the segment start) -> the chunk's
+    // workspace tile, fp16 in the staged 128-byte-swizzle layout (the A operand of the
+    // second phase).  Lane l keeps the decay from the segment start of channels 2l, 2l+1
+    // (the sum of the earlier chunks' decays, row 0 of their gate tiles) and takes the
+    // 16-byte pieces l, l+32, ... of the tile, so every store instruction writes 512
+    // contiguous bytes.
+    if (partial) {
+      bool ok = true;
+      float a2s0 = 0.f, a2s1 = 0.f;
+      const float* eseg = ms->eseg;
+      for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
+        const int st = n % kStages;
+        if (!wait_bar(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x110)) { ok = false; break; }
+        const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
+        {
+          *reinterpret_cast<float2*>(&ms->eseg[2 * lane]) = make_float2(ex2(a2s0), ex2(a2s1));
+          const float2 a2 = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(qt + 3 * kTile) + 2 * lane);
+          a2s0 += a2.x;
+          a2s1 += a2.y;
+          __syncwarp();
+        }
+        uint8_t* dst = reinterpret_cast<uint8_t*>(fp.qhp + ((size_t)seq * fp.Nc + c) * 4096);
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int idx = lane + 32 * i, r = idx >> 3, jp = idx & 7, jl = jp ^ (r & 7);
+          uint4 v = *reinterpret_cast<const uint4*>(qt + r * 128 + 16 * jp);  // channels 8 jl .. 8 jl + 7
+          const float4 e0 = *reinterpret_cast<const float4*>(eseg + 8 * jl);
+          const float4 e1 = *reinterpret_cast<const float4*>(eseg + 8 * jl + 4);
+          v.x = h2_bits(__hmul2(bits_h2(v.x), __floats2half2_rn(e0.x, e0.y)));
+          v.y = h2_bits(__hmul2(bits_h2(v.y), __floats2half2_rn(e0.z, e0.w)));
+          v.z = h2_bits(__hmul2(bits_h2(v.z), __floats2half2_rn(e1.x, e1.y)));
+          v.w = h2_bits(__hmul2(bits_h2(v.w), __floats2half2_rn(e1.z, e1.w)));
+          *reinterpret_cast<uint4*>(dst + r * 128 + 16 * jp) = v;
+        }
+        // the tile is read back by bulk copy (async proxy); the staged chunk is released
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms->qdone[st]);
+      }
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&ms->agg_pub);
+    }
   } else if (warp == kMmaWarp) {
-    // ===================================================================== MMA issuer
-    // Event-driven over the CTA's chunks: whichever of stage 1 (scores, U'), stage 2a
-    // (O = Qh S) and stage 2b (O += P V) has its inputs ready is issued, so a slow
-    // operand build never holds back the products of earlier chunks (and with them the
-    // release of their staging buffers).  Stage 1 runs up to kSU chunks ahead of 2b.
+    // ===================================================================== MMA issuer, stage 1
+    // Scores = Qh Kh^T (tensor-core chunks) and U' = Kh^T V, in chunk order, up to kSU
+    // chunks ahead of the outputs.
     if (lane == 0) {
       const uint32_t id_qk = idesc_f16(0, 64, 64, 0, 0);  // A K-major, B K-major
       const uint32_t id_kv = idesc_f16(0, 64, 64, 1, 1);  // A MN-major, B MN-major
-      const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);  // A K-major, B MN-major
       const uint32_t s_base = smem_u32(smem);
-      // output region of chunk m: pair (m/2) % 2, lane tile m % 2
-      auto out_region = [&](int m) -> uint32_t {
-        return tmem + kColO + 64u * (uint32_t)((m >> 1) & 1) + ((m & 1) ? kLaneTile1 : 0u);
-      };
-      int n1 = 0, n2a = 0, n2b = 0;
-      uint64_t t_last = globaltimer();
-      while (n2b < cnt) {
-        bool prog = false;
-        if (n2b < n2a && mbar_test(&ms->pready[n2b % kSU], ph_use<kSU>(n2b))) {
-          // stage 2b of chunk m: O += P V with P in tensor memory; the chunk's staging
-          // buffer and score region are free afterwards
-          const int m = n2b, st = m % kStages, su = m % kSU;
-          const uint32_t a_v = s_base + kOffStage + st * kStageBytes + 2 * kTile;
-          // P sits in the lane tile of the chunk's output (A and D rows share lanes)
-          const uint32_t a_p = tmem + kColSU + 64u * su + ((m & 1) ? kLaneTile1 : 0u);
-          const uint32_t d_o = out_region(m);
-          tc_fence_after();
+      for (int n = 0; n < cnt; ++n) {
+        const int st = n % kStages;
+        if (!wait_spin(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x200)) break;
+        if (!wait_spin(&ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x201)) break;
+        const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
+        const uint32_t a_k = a_q + kTile;                            // Kh
+        const uint32_t a_v = a_q + 2 * kTile;
+        tc_fence_after();
+        const uint32_t su = tmem + kColSU + 64u * (uint32_t)(n % kSU);
+        if (!*(volatile int*)&ms->fb[st]) {
           for (int k = 0; k < 4; ++k)
-            mma_f16_ta(d_o, a_p + 8 * k, sw128_desc(a_v + 2048 * k), id_qs, 1);
-          mma_commit(&ms->su_free[su]);
-          mma_commit(&ms->empty[st]);
-          if ((m & 1) || m + 1 == cnt) mma_commit(&ms->o_full[(m >> 1) & 1]);
-          ++n2b;
-          prog = true;
+            mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
         }
-        if (n2a < n1) {
-          // stage 2a of chunk m: O = Qh S (S = the chunk-start state tile); an output
-          // pair's region is reused once the epilogue of the pair two back is done
-          const int m = n2a, st = m % kStages;
-          bool rdy = mbar_test(&ms->sready[m % 3], ph_use<3>(m));
-          if (!(m & 1)) rdy = rdy && mbar_test(&ms->o_free[(m >> 1) & 1], ph_rel<2>(m >> 1));
-          if (rdy) {
-            const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
-            const uint32_t a_s = s_base + kOffS + (m % 3) * kTile;
-            tc_fence_after();
-            for (int k = 0; k < 4; ++k)
-              mma_f16(out_region(m), sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-            mma_commit(&ms->sfree[m % 3]);
-            ++n2a;
-            prog = true;
-          }
-        }
-        if (n1 < cnt && mbar_test(&ms->opready[n1 % kStages], ph_use<kStages>(n1)) &&
-            mbar_test(&ms->su_free[n1 % kSU], ph_rel<kSU>(n1))) {
-          // stage 1 of chunk n: scores = Qh Kh^T (tensor-core chunks), U' = Kh^T V
-          const int n = n1, st = n % kStages;
-          const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
-          const uint32_t a_k = a_q + kTile;                            // Kh
-          const uint32_t a_v = a_q + 2 * kTile;
-          tc_fence_after();
-          const uint32_t su = tmem + kColSU + 64u * (uint32_t)(n % kSU);
-          if (!*(volatile int*)&ms->fb[st]) {
-            for (int k = 0; k < 4; ++k)
-              mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
-          }
-          for (int k = 0; k < 4; ++k)
-            mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
-          mma_commit(&ms->su_full[n % kSU]);
-          ++n1;
-          prog = true;
-        }
-        if (prog) {
-          t_last = globaltimer();
-        } else {
-          if (*(volatile int*)&ms->abort) break;
-          if (globaltimer() - t_last > 1000000000ull) {
-            record_error(hdr, GTR_ERR_TIMEOUT, 0x207);
-            *(volatile int*)&ms->abort = 1;
-            break;
-          }
-          // sleep in hardware on the oldest pending step's barrier (woken when it
-          // completes, at most half a microsecond); the loop then re-polls every step
-          if (n2b < n2a)
-            (void)mbar_wait_sleep(&ms->pready[n2b % kSU], ph_use<kSU>(n2b), 500u);
-          else if (n2a < n1)
-            (void)mbar_wait_sleep(&ms->sready[n2a % 3], ph_use<3>(n2a), 500u);
-          else
-            (void)mbar_wait_sleep(&ms->opready[n1 % kStages], ph_use<kStages>(n1), 500u);
-        }
+        for (int k = 0; k < 4; ++k)
+          mma_f16(su + kLaneTile1, sw128_desc(a_k + 2048 * k), sw128_desc(a_v + 2048 * k), id_kv, k > 0);
+        mma_commit(&ms->su_full[n % kSU]);
       }
       // every MMA issued here has completed before tensor memory is freed
-      mma_commit(&ms->mma_final);
+      mma_commit(&ms->mma_final[0]);
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&ms->mma_final, 0) && globaltimer() - t0 < 1000000000ull) {
+      while (!mbar_try_wait(&ms->mma_final[0], 0) && globaltimer() - t0 < 1000000000ull) {
+      }
+    }
+  } else if (warp == kOutWarp) {
+    // ===================================================================== MMA issuer, stage 2
+    // Per chunk m in order: O = Qh S (2a, once Qh is built, the chunk-start state is
+    // written and, for the first chunk of a pair, the pair's output region is free), then
+    // O += P V (2b, with P in tensor memory), which frees the chunk's staging buffer and
+    // score region.
+    if (lane == 0) {
+      const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);  // A K-major, B MN-major
+      const uint32_t s_base = smem_u32(smem);
+      for (int m = 0; m < cnt; ++m) {
+        const int st = m % kStages, su = m % kSU;
+        // output region of chunk m: pair (m/2) % 2, lane tile m % 2
+        const uint32_t d_o = tmem + kColO + 64u * (uint32_t)((m >> 1) & 1) + ((m & 1) ? kLaneTile1 : 0u);
+        // Qh built (the stage-1 issuer waits on the same phase; neither can lap it, as the
+        // stage is refilled only after this chunk's P V), chunk-start state written
+        if (!wait_spin(&ms->opready[st], ph_use<kStages>(m), ms, hdr, 0x205)) break;
+        if (!wait_spin(&ms->sready[m % kNS], ph_use<kNS>(m), ms, hdr, 0x202)) break;
+        if (!(m & 1) && !wait_spin(&ms->o_free[(m >> 1) & 1], ph_rel<2>(m >> 1), ms, hdr, 0x203)) break;
+        const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
+        const uint32_t a_s = s_base + kOffS + (m % kNS) * kTile;
+        tc_fence_after();
+        for (int k = 0; k < 4; ++k)
+          mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
+        if (!wait_spin(&ms->pready[su], ph_use<kSU>(m), ms, hdr, 0x204)) break;
+        // P sits in the lane tile of the chunk's output (A and D rows share lanes)
+        const uint32_t a_v = a_q + 2 * kTile;
+        const uint32_t a_p = tmem + kColSU + 64u * su + ((m & 1) ? kLaneTile1 : 0u);
+        tc_fence_after();
+        for (int k = 0; k < 4; ++k)
+          mma_f16_ta(d_o, a_p + 8 * k, sw128_desc(a_v + 2048 * k), id_qs, 1);
+        mma_commit(&ms->su_free[su]);
+        mma_commit(&ms->empty[st]);
+        if ((m & 1) || m + 1 == cnt) mma_commit(&ms->o_full[(m >> 1) & 1]);
+      }
+      mma_commit(&ms->mma_final[1]);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&ms->mma_final[1], 0) && globaltimer() - t0 < 1000000000ull) {
       }
     }
   } else if (warp < 8) {
     // ===================================================================== WG_A: operand tiles
-    // Two warpgroups share every chunk: warpgroup hh takes channels 32hh .. 32hh+31, its
-    // warp w4 the rows 16w4 .. 16w4+15, a thread 4 rows x 4 channels.
+    // The two warpgroups take alternate chunks (warpgroup hh: chunks n = hh, hh+2, ...),
+    // each in two passes over the key-channel halves: its warp w4 takes rows 16w4 ..
+    // 16w4+15, a thread 4 rows x 4 channels per pass.
     const int hh = warp >> 2, w4 = warp & 3;
     const int wg = hh, wtid = tid - kWG * hh;
-    const int cc = lane & 7;                  // channels ch0 .. ch0+3
-    const int ch0 = 32 * hh + 4 * cc;
+    const int cc = lane & 7;                     // channels 32p + 4cc .. 32p + 4cc + 3 in pass p
     const int row0 = 16 * w4 + 4 * (lane >> 3);  // rows row0 .. row0+3
-    const bool rev = fp.rev != 0;
+    constexpr bool rev = kRev;
     int slot = 0;
     bool alive = true;
-    float a2s[4] = {0.f, 0.f, 0.f, 0.f};  // log2 decay from the segment start, channels ch0..ch0+3
-    for (int n = 0; n < cnt; ++n) {
-      const int bb = n & 1, st = n % kStages;
+    for (int n = hh; n < cnt; n += 2) {
+      const int st = n % kStages;
       if (!wg_wait(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
         alive = false;
         break;
       }
       uint8_t* sb = smem + kOffStage + st * kStageBytes;
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
-      // ---- in-chunk cumulative log2-gates in scan order: my 4 rows, a scan over the
-      // warp's 4 row blocks, then over the 4 warps (staged rows run backwards in scan
-      // order when the chunk is reversed)
-      float A[4][4];
-      float run[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+      // ---- in-chunk cumulative log2-gates in scan order: my 4 rows (written back over
+      // the gates, still without the offset of the rows before them), a scan over the
+      // warp's 4 row blocks, then over the 4 warps through shared memory (staged rows run
+      // backwards in scan order when the chunk is reversed)
+      float run[2][4], incl[2][4];
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+        const int ch0 = 32 * ps + 4 * cc;
         float gv[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * 64 + ch0);
           gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
         }
-        if (!rev) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+        for (int e = 0; e < 4; ++e) run[ps][e] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              run[e] = fmaf(gv[i][e], kLog2e, run[e]);
-              A[i][e] = run[e];
-            }
-        } else {
+        for (int k = 0; k < 4; ++k) {
+          const int i = rev ? 3 - k : k;
 #pragma unroll
-          for (int i = 3; i >= 0; --i)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              run[e] = fmaf(gv[i][e], kLog2e, run[e]);
-              A[i][e] = run[e];
-            }
+          for (int e = 0; e < 4; ++e) {
+            run[ps][e] = fmaf(gv[i][e], kLog2e, run[ps][e]);
+            gv[i][e] = run[ps][e];
+          }
         }
-      }
-      float incl[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        incl[e] = run[e];
-        if (!rev) {
-          float x = __shfl_up_sync(0xffffffffu, incl[e], 8);
-          if (lane >= 8) incl[e] += x;
-          x = __shfl_up_sync(0xffffffffu, incl[e], 16);
-          if (lane >= 16) incl[e] += x;
-        } else {
-          float x = __shfl_down_sync(0xffffffffu, incl[e], 8);
-          if (lane < 24) incl[e] += x;
-          x = __shfl_down_sync(0xffffffffu, incl[e], 16);
-          if (lane < 16) incl[e] += x;
-        }
-      }
-      float* redh = &ms->red[hh][0][0];  // [4 warps][32 channels] of this channel half
-      if (rev ? lane < 8 : lane >= 24)
-        *reinterpret_cast<float4*>(redh + w4 * 32 + 4 * cc) = make_float4(incl[0], incl[1], incl[2], incl[3]);
-      wg_sync(wg);
-      float off[4], last[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        off[e] = incl[e] - run[e];
-        last[e] = 0.f;
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float4 t4 = *reinterpret_cast<const float4*>(redh + w * 32 + 4 * cc);
-        const float t[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (rev ? w > w4 : w < w4) off[e] += t[e];
-          last[e] += t[e];
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) A[i][e] += off[e];
-      // CUDA-core decision over all 64 channels: each warp covers its half's 32 channels,
-      // the two halves meet at a 256-thread barrier
-      bool exp_unsafe = false;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (-last[e] > fp.max_exp2) exp_unsafe = true;
-      const bool half_unsafe = __any_sync(0xffffffffu, exp_unsafe);
-      if (wtid == 0) ms->fbh[bb][hh] = half_unsafe ? 1 : 0;
-      asm volatile("bar.sync 6, 256;" ::: "memory");
-      const bool fbx = (*(volatile int*)&ms->fbh[bb][0] | *(volatile int*)&ms->fbh[bb][1]) != 0;
-      if (fbx) {
-        // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
-        // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i);
-        // warpgroup hh fills score columns 32hh .. 32hh+31 of its warps' rows.  A goes to
-        // the gate tile so that every thread can read every row and channel.
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(A[i][0], A[i][1], A[i][2], A[i][3]);
-        if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
-        asm volatile("bar.sync 6, 256;" ::: "memory");  // A of both channel halves is in place
-        tc_fence_after();
-        const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
-        float sv[16];
-        for (int x = 0; x < 16; ++x) {
-          const int i = r0 + 8 * ((x & 3) >> 1);
-          const int j = 32 * hh + 8 * (x >> 2) + cq + (x & 1);
-          float acc = 0.f;
-          if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
-            for (int k = 0; k < 64; k += 2) {
-              const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
-              const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
-              acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
-              acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
-            }
+          *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(gv[i][0], gv[i][1], gv[i][2], gv[i][3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = run[ps][e];
+          if (!rev) {
+            float x = __shfl_up_sync(0xffffffffu, v, 8);
+            if (lane >= 8) v += x;
+            x = __shfl_up_sync(0xffffffffu, v, 16);
+            if (lane >= 16) v += x;
+          } else {
+            float x = __shfl_down_sync(0xffffffffu, v, 8);
+            if (lane < 24) v += x;
+            x = __shfl_down_sync(0xffffffffu, v, 16);
+            if (lane < 16) v += x;
           }
-          sv[x] = acc * 0.125f;
+          incl[ps][e] = v;
         }
-        tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU) + 32u * hh, sv);
+        if (rev ? lane < 8 : lane >= 24)
+          *reinterpret_cast<float4*>(&ms->red[hh][ps][w4][4 * cc]) =
+              make_float4(incl[ps][0], incl[ps][1], incl[ps][2], incl[ps][3]);
+      }
+      wg_sync(wg);
+      // offsets of my rows (the rows of earlier lanes and warps) and the chunk decay a
+      float off[2][4], last[2][4];
+      bool exp_unsafe = false;
+#pragma unroll
+      for (int ps = 0; ps < 2; ++ps) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          off[ps][e] = incl[ps][e] - run[ps][e];
+          last[ps][e] = 0.f;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 t4 = *reinterpret_cast<const float4*>(&ms->red[hh][ps][w][4 * cc]);
+          const float t[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (rev ? w > w4 : w < w4) off[ps][e] += t[e];
+            last[ps][e] += t[e];
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (-last[ps][e] > fp.max_exp2) exp_unsafe = true;
+      }
+      // CUDA-core decision: the lanes of every warp hold the decays of all 64 channels
+      const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
+      if (fbx) {
+        // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
+        // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i).
+        // The full A goes to the gate tile so that every thread can read every row and
+        // channel.
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float4* gp = reinterpret_cast<float4*>(G + (row0 + i) * 64 + 32 * ps + 4 * cc);
+            const float4 a4 = *gp;
+            *gp = make_float4(a4.x + off[ps][0], a4.y + off[ps][1], a4.z + off[ps][2], a4.w + off[ps][3]);
+          }
+        if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
+        tc_fence_after();  // (the wait's barrier also publishes the full A)
+        const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
+        for (int ps = 0; ps < 2; ++ps) {
+          float sv[16];
+          for (int x = 0; x < 16; ++x) {
+            const int i = r0 + 8 * ((x & 3) >> 1);
+            const int j = 32 * ps + 8 * (x >> 2) + cq + (x & 1);
+            float acc = 0.f;
+            if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
+              for (int k = 0; k < 64; k += 2) {
+                const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
+                const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
+                acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
+                acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
+              }
+            }
+            sv[x] = acc * 0.125f;
+          }
+          tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU) + 32u * ps, sv);
+        }
         tmem_wait_st();
         tc_fence_before();
-        asm volatile("bar.sync 6, 256;" ::: "memory");  // raw q / k reads done before the overwrite
+        wg_sync(wg);  // raw q / k reads done before the overwrite
+#pragma unroll
+        for (int ps = 0; ps < 2; ++ps)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) off[ps][e] = 0.f;  // the gate tile holds the full A now
       }
       // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
       const __half2 eighth = __float2half2_rn(0.125f);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = row0 + i;
-        // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
-        const uint32_t off8 = row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
-        uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
-        uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
-        uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
-        uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
+      for (int ps = 0; ps < 2; ++ps) {
+        const int ch0 = 32 * ps + 4 * cc;
 #pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {
-          const float A0 = A[i][2 * e2], A1 = A[i][2 * e2 + 1];
-          const float xk0 = fbx ? last[2 * e2] - A0 : -A0;
-          const float xk1 = fbx ? last[2 * e2 + 1] - A1 : -A1;
-          __half2 qh, kh;
-          if constexpr (std::is_same<Tin, __half>::value) {
-            qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
-            kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
-          } else {
-            const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
-            qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
-            kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+        for (int i = 0; i < 4; ++i) {
+          const int row = row0 + i;
+          const float4 a4 = *reinterpret_cast<const float4*>(G + row * 64 + ch0);
+          const float Ar[4] = {a4.x + off[ps][0], a4.y + off[ps][1], a4.z + off[ps][2], a4.w + off[ps][3]};
+          // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
+          const uint32_t off8 =
+              row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
+          uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
+          uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
+          uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
+          uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const float A0 = Ar[2 * e2], A1 = Ar[2 * e2 + 1];
+            const float xk0 = fbx ? last[ps][2 * e2] - A0 : -A0;
+            const float xk1 = fbx ? last[ps][2 * e2 + 1] - A1 : -A1;
+            __half2 qh, kh;
+            if constexpr (std::is_same<Tin, __half>::value) {
+              qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
+              kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
+            } else {
+              const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
+              qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
+              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+            }
+            qw[e2] = h2_bits(qh);
+            kw[e2] = h2_bits(kh);
           }
-          qw[e2] = h2_bits(qh);
-          kw[e2] = h2_bits(kh);
+          *reinterpret_cast<uint2*>(sb + off8) = qraw;
+          *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
         }
-        *reinterpret_cast<uint2*>(sb + off8) = qraw;
-        *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
       }
       if constexpr (!std::is_same<Tin, __half>::value) {
-        // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range);
-        // the two warpgroups take alternate 16-byte chunks
+        // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
         uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
 #pragma unroll
-        for (int i = tid; i < kTile / 16; i += 2 * kWG) {
+        for (int i = wtid; i < kTile / 16; i += kWG) {
           uint4 x = vt[i];
           uint32_t* w = reinterpret_cast<uint32_t*>(&x);
 #pragma unroll
@@ -864,28 +936,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (w4 == 0 && lane < 8) {
-        // gate row 0 now holds the chunk's decay a per channel, row 1 the factor
-        // 2^(decay from the segment start to this chunk) of Qh'
-        *reinterpret_cast<float4*>(G + ch0) = make_float4(last[0], last[1], last[2], last[3]);
-        *reinterpret_cast<float4*>(G + 64 + ch0) = make_float4(ex2(a2s[0]), ex2(a2s[1]), ex2(a2s[2]), ex2(a2s[3]));
-      }
+        // gate row 0 (read by this thread only, above) now holds the chunk's decay a per
+        // channel
 #pragma unroll
-      for (int e = 0; e < 4; ++e) a2s[e] += last[e];
-      if (tid == 0) ms->fb[st] = fbx ? 1 : 0;
+        for (int ps = 0; ps < 2; ++ps)
+          *reinterpret_cast<float4*>(G + 32 * ps + 4 * cc) = make_float4(last[ps][0], last[ps][1], last[ps][2], last[ps][3]);
+      }
+      if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
       fence_proxy_async_smem();
-      wg_sync(wg);
-      if (wtid == 0) mbar_arrive(&ms->opready[st]);  // one arrival per channel half
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->opready[st]);  // every warp, once its writes are done
     }
     if (partial && alive) second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
 
   } else if (warp < 12) {
     // ===================================================================== WG_B: masking, state
     // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
-    // r0 + 8(q>>1), column 8c + cq + (q&1) of the warp's 16-row slice.
+    // r0 + 8(q>>1), column 8c + cq + (q&1) of the warp's 16-row slice.  No named barrier
+    // inside the chunk loop: every thread waits on the mbarriers itself (bounded), every
+    // warp arrives on the ones it feeds.
     const int wg = 2, wtid = tid - 2 * kWG, wq = warp & 3;
     const int r0 = 16 * wq + (lane >> 2), r1 = r0 + 8, cq = 2 * (lane & 3);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);  // this warp's lane quarter
-    const bool rev = fp.rev != 0;
+    constexpr bool rev = kRev;
     float Ls[32];                  // fp32 state entries (rows r0 / r1 = key channels)
     float a2r0 = 0.f, a2r1 = 0.f;  // log2 segment decay of rows r0 / r1
     int slot = 0;
@@ -897,17 +970,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4* sz = reinterpret_cast<uint4*>(smem + kOffS);
       for (int i = wtid; i < kTile / 16; i += kWG) sz[i] = z;
       fence_proxy_async_smem();
-      wg_sync(wg);
-      if (wtid == 0) mbar_arrive(&ms->sready[0]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->sready[0]);
     }
     for (int n = 0; n < cnt; ++n) {
-      const int c = sp.c0 + n, st = n % kStages, su = n % kSU;
-      const bool last_chunk = n + 1 == cnt;
-      if (!wg_wait(wg, wtid, &ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400, slot)) { alive = false; break; }
+      const int st = n % kStages, su = n % kSU;
+      if (!wait_bar(&ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400)) { alive = false; break; }
       tc_fence_after();
       const bool fbk = ms->fb[st] != 0;
-      const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
-      const float* alast = reinterpret_cast<const float*>(qt + 3 * kTile);
+      const float* alast = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes + 3 * kTile);
       const float l0 = alast[r0], l1 = alast[r1];
       const float dl0 = ex2(l0), dl1 = ex2(l1);
       const uint32_t sreg = tl + kColSU + 64u * (uint32_t)su;
@@ -924,23 +995,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       a2r0 += l0;
       a2r1 += l1;
-      if (partial) {
-        // this chunk's Qh' = Qh 2^(A from the segment start) -> its workspace tile (fp16,
-        // the 128-byte-swizzle MMA layout), the A operand of the second phase; read from
-        // the staged Qh before P is signalled (P V's completion frees the stage)
-        const float* eseg = alast + 64;  // gate row 1
-        uint8_t* dst = reinterpret_cast<uint8_t*>(fp.qhp + ((size_t)seq * fp.Nc + c) * 4096);
-#pragma unroll
-        for (int cb = 0; cb < 8; ++cb) {
-          const uint32_t o = (((uint32_t)cb ^ ((uint32_t)r0 & 7u)) << 4) + cq * 2;  // r1 & 7 == r0 & 7
-          const float2 ef = *reinterpret_cast<const float2*>(eseg + 8 * cb + cq);
-          const __half2 e2 = __floats2half2_rn(ef.x, ef.y);
-          *reinterpret_cast<uint32_t*>(dst + r0 * 128 + o) =
-              h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r0 * 128 + o)), e2));
-          *reinterpret_cast<uint32_t*>(dst + r1 * 128 + o) =
-              h2_bits(__hmul2(bits_h2(*reinterpret_cast<const uint32_t*>(qt + r1 * 128 + o)), e2));
-        }
-      }
       // masked scores -> fp16 P over the first 32 columns of the chunk's score region,
       // the A operand of P V.  A rows are read from the lanes of the output rows, so P
       // goes to the lane tile of the chunk's output region (tile 1: over U', already
@@ -980,14 +1034,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      wg_sync(wg);
-      if (wtid == 0) mbar_arrive(&ms->pready[su]);
-      if (!last_chunk) {
-        // the next chunk's start state, into state tile (n+1) % 3 once O = Qh S of chunk
-        // n-2, its last reader, has completed
-        const int t = (n + 1) % 3;
-        if (!wg_wait(wg, wtid, &ms->sfree[t], ph_rel<3>(n + 1), ms, hdr, 0x401, slot)) { alive = false; break; }
-        uint8_t* srow0 = smem + kOffS + t * kTile + r0 * 128;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->pready[su]);
+      if (n + 1 < cnt) {
+        // the next chunk's start state, into state tile (n+1) % kNS.  Its last reader,
+        // O = Qh S of chunk n+1-kNS, has completed: the P V of that chunk, issued after
+        // it by the same thread, released the score region chunk n's scores went to.
+        uint8_t* srow0 = smem + kOffS + ((n + 1) % kNS) * kTile + r0 * 128;
         uint8_t* srow1 = srow0 + 8 * 128;
 #pragma unroll
         for (int cb = 0; cb < 8; ++cb) {
@@ -996,13 +1049,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           sts32(srow1 + o, pack_h2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
         }
         fence_proxy_async_smem();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->sready[t]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms->sready[(n + 1) % kNS]);
       }
     }
+    // every thread leaves the loop (the waits are bounded): agree on the outcome
+    alive = wg_all(wg, alive);
     if (segm && alive) {
-      // the Qh' tiles written above are read back by bulk copy (async proxy)
-      if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
       // segment summary: U_seg = local end state, its log2 decay
       float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * (4096 + 64);
 #pragma unroll
@@ -1036,7 +1089,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_use<2>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
         const int ci = 2 * pr + tsel;
-        const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - trow : trow);
+        const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
         const bool valid = ci < cnt && s < L;
         const uint32_t src = tl + kColO + 64u * (uint32_t)(pr & 1);
         if (partial) {
@@ -1080,6 +1133,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
       if (ok0) {
         if (wtid == 0) {
+          // the second phase's first four pairs start loading now (every MMA of this
+          // CTA has completed, so all staging buffers are free; the Qh' and O_local
+          // tiles are written and fenced)
+          if (partial)
+            for (int q = 0; q < 4 && 2 * q < cnt; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
           red_release_add(ctr, 1u);
           ok0 = wait_counter(ctr, target, ms, hdr, 0x601);
         }
@@ -1267,14 +1325,15 @@ size_t seg_capacity(const Problem& p) {
 
 template <typename Tin, typename Tout>
 gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
-  auto kern = fused_gla_kernel<Tin, Tout>;
-  static std::atomic<unsigned long long> configured{0};
+  const bool rev = p.direction == GTR_R2L || p.direction == GTR_B2T;
+  auto kern = rev ? fused_gla_kernel<Tin, Tout, true> : fused_gla_kernel<Tin, Tout, false>;
+  static std::atomic<unsigned long long> configured[2];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
-  if (!(configured.load() & (1ull << dev))) {
+  if (!(configured[rev].load() & (1ull << dev))) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
       return GTR_ERR_CUDA;
-    configured.fetch_or(1ull << dev);
+    configured[rev].fetch_or(1ull << dev);
   }
   Plan pl = make_plan(p, device_sms());
   if (force_mode == 0) {
