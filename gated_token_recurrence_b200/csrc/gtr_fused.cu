@@ -430,6 +430,34 @@ __device__ __forceinline__ uint32_t ph_rel(int n) { return ((uint32_t)(n / depth
 // by bulk copy into staging buffer q; one M = 128 MMA puts chunk 2m's rows in lanes
 // 0-63 and chunk 2m+1's in lanes 64-127 of tensor-memory slot q; warp wq of the group
 // takes lanes 32wq .. 32wq+31 (chunk 2m + wq/2, rows 32(wq%2) ..).
+// Scores of a chunk whose gates decay too fast for the factorisation, on the CUDA cores:
+// d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i), from the raw q / k
+// tiles and the full A in the gate tile, into the 16 rows of warp w4 of the chunk's score
+// region (16x256b shape: register 4c+q is row r0 + 8(q>>1), column 8c + cq + (q&1)).
+// Out of line: the chunk loops stay small for the instruction cache.
+template <typename Tin, bool kRev>
+__device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G, uint32_t taddr, int w4, int lane) {
+  const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
+  for (int ps = 0; ps < 2; ++ps) {
+    float sv[16];
+    for (int x = 0; x < 16; ++x) {
+      const int i = r0 + 8 * ((x & 3) >> 1);
+      const int j = 32 * ps + 8 * (x >> 2) + cq + (x & 1);
+      float acc = 0.f;
+      if (kRev ? j >= i : j <= i) {  // scan(j) <= scan(i)
+        for (int k = 0; k < 64; k += 2) {
+          const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
+          const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
+          acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
+          acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
+        }
+      }
+      sv[x] = acc * 0.125f;
+    }
+    tmem_st16x256_x4(taddr + 32u * ps, sv);
+  }
+}
+
 // Bulk copies of pair m2's Qh' and O_local tiles into staging buffer q (second phase).
 __device__ __forceinline__ void p2_load(const FusedParams& fp, Misc* ms, uint8_t* smem, int seq, Span sp, int q, int m2) {
   const int c = sp.c0 + 2 * m2, nb = min(2, sp.c1 - c);
@@ -855,25 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
         tc_fence_after();  // (the wait's barrier also publishes the full A)
-        const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
-        for (int ps = 0; ps < 2; ++ps) {
-          float sv[16];
-          for (int x = 0; x < 16; ++x) {
-            const int i = r0 + 8 * ((x & 3) >> 1);
-            const int j = 32 * ps + 8 * (x >> 2) + cq + (x & 1);
-            float acc = 0.f;
-            if (rev ? j >= i : j <= i) {  // scan(j) <= scan(i)
-              for (int k = 0; k < 64; k += 2) {
-                const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
-                const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
-                acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
-                acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
-              }
-            }
-            sv[x] = acc * 0.125f;
-          }
-          tmem_st16x256_x4(tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU) + 32u * ps, sv);
-        }
+        cuda_core_scores<Tin, rev>(sb, G, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU), w4,
+                                   lane);
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);  // raw q / k reads done before the overwrite
@@ -884,14 +895,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
       const __half2 eighth = __float2half2_rn(0.125f);
-#pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
+#pragma unroll 1
+      for (int ps = 0; ps < 2; ++ps) {  // (rolled: the loop body stays small for the instruction cache)
         const int ch0 = 32 * ps + 4 * cc;
+        float offp[4], lastp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          offp[e] = ps ? off[1][e] : off[0][e];
+          lastp[e] = ps ? last[1][e] : last[0][e];
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = row0 + i;
           const float4 a4 = *reinterpret_cast<const float4*>(G + row * 64 + ch0);
-          const float Ar[4] = {a4.x + off[ps][0], a4.y + off[ps][1], a4.z + off[ps][2], a4.w + off[ps][3]};
+          const float Ar[4] = {a4.x + offp[0], a4.y + offp[1], a4.z + offp[2], a4.w + offp[3]};
           // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
           const uint32_t off8 =
               row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
@@ -902,8 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const float A0 = Ar[2 * e2], A1 = Ar[2 * e2 + 1];
-            const float xk0 = fbx ? last[ps][2 * e2] - A0 : -A0;
-            const float xk1 = fbx ? last[ps][2 * e2 + 1] - A1 : -A1;
+            const float xk0 = fbx ? lastp[2 * e2] - A0 : -A0;
+            const float xk1 = fbx ? lastp[2 * e2 + 1] - A1 : -A1;
             __half2 qh, kh;
             if constexpr (std::is_same<Tin, __half>::value) {
               qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
