@@ -1316,6 +1316,11 @@ Plan make_plan(const Problem& p, int sms) {
     pl.mode = 1;
     pl.n_s = cap / pl.n_seq;
     if (pl.n_s > Nc) pl.n_s = Nc;
+    // the longest segment sets the time: with k = ceil(Nc / n_s) chunks in it, take the
+    // fewest segments that still hold at most k each (less contention, a shorter scan).
+    // Runs of one or two chunks keep every CTA: most segments are then a single chunk.
+    const int k = (Nc + pl.n_s - 1) / pl.n_s;
+    if (k >= 3) pl.n_s = (Nc + k - 1) / k;
     pl.grid = pl.n_seq * pl.n_s;
   }
   return pl;
