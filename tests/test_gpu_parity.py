@@ -296,11 +296,11 @@ def test_back_to_back_calls_leave_no_device_error(name):
 
 
 @pytest.mark.parametrize("name", ["2048", "stack"])
-def test_multi_round_calls_in_alternating_directions_match_the_oracle(name):
-    """Workloads whose sequences span several rounds of the held mode (2048^2 also has
-    segments with no chunks in its last round): calls in alternating directions, every
-    output checked against the oracle.  A segment summary overwritten before every CTA
-    had scanned it shows up as wrong outputs from that segment on, in some calls only."""
+def test_segmented_calls_in_alternating_directions_match_the_oracle(name):
+    """Workloads split into segments (one CTA each; 2048^2: 24 segments of 10-11 chunks,
+    the stack: 3 of 20): calls in alternating directions, every output checked against
+    the oracle.  A segment summary, start state or second-phase tile read before its
+    writer was done shows up as wrong outputs from that segment on, in some calls only."""
     w = WORKLOADS[name]
     q, k, v, lg = make_inputs(w, 83)
     dev = torch.device("cuda:0")
