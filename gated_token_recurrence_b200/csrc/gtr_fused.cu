@@ -77,8 +77,9 @@ constexpr int kNS = 5;                                     // chunk-start state 
 constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [kNS] chunk-start states
 constexpr int kOffSst = kOffS;                             // segment start state (after the chunks: over state tile 0)
 constexpr int kOffStg = kOffS + kNS * kTile;               // output staging, 4 warps x 32 rows x 128 B
-constexpr int kOffMisc = kOffStg + 4 * 32 * 128;
-constexpr int kMiscBytes = 4096;
+constexpr int kStgBytes = 4 * 32 * 128 + 1024;             // (CLUSTER: the summary slices received, <= 16464 B)
+constexpr int kOffMisc = kOffStg + kStgBytes;
+constexpr int kMiscBytes = 8192;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 // second phase, pair slot q (one per warpgroup) in staging buffer q: Qh' of the pair
 // (16 KB, the A operand; then the warps' fp32 output staging) and O_local (16 KB)
@@ -88,9 +89,13 @@ static_assert(2 * kP2Olc <= kStageBytes, "a chunk pair's second-phase tiles fit 
 // tensor memory columns
 constexpr uint32_t kColSU = 0;     // [kSU] x 64: scores (lane tile 0; masked fp16 P over their first
                                    // 32 columns) and U' (lane tile 1)
-constexpr uint32_t kColO = kColSU + 64u * kSU;  // [2] x 64 output pairs (chunk 2m lane tile 0, 2m+1 tile 1)
+constexpr int kOPairs = 4;         // output pairs in tensor memory (a ring; CLUSTER: all of a CTA's chunks)
+constexpr uint32_t kColO = kColSU + 64u * kSU;  // [kOPairs] x 64 output pairs (chunk 2m lane tile 0, 2m+1 tile 1)
 constexpr uint32_t kLaneTile1 = 16u << 16;
-static_assert(kColO + 128 <= kTmemCols, "tensor memory budget");
+constexpr int kClusterChunks = 2 * kOPairs;  // CLUSTER: chunks per CTA (outputs held in tensor memory)
+constexpr int kMaxCluster = 16;              // CLUSTER: CTAs per sequence (non-portable cluster size)
+static_assert(kColO + 64 * kOPairs <= kTmemCols, "tensor memory budget");
+static_assert(kClusterChunks * kTile + 3 * 16384 <= kOffS, "a CTA's Qh' tiles and three epilogue staging areas fit the idle staging buffers");
 static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) reuse the score regions");
 
 // Segment counters sit at a fixed place right after the workspace header, whatever
@@ -112,7 +117,7 @@ struct alignas(64) FusedParams {
   uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
   uint16_t* qhp;           // [n_seq][Nc][64*64] Qh' per chunk, fp16, MMA layout
   uint16_t* olc;           // [n_seq][Nc][64][64] outputs from a zero segment start, fp16
-  int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED
+  int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED, 2 = CLUSTER
   int grid;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
   int tma;                 // 1: every chunk is one TMA box per tensor; 0: cp.async row copies
@@ -128,13 +133,14 @@ struct Misc {
   uint64_t su_full[kSU], su_free[kSU], pready[kSU];  // per score / U' region
   uint64_t sready[kNS];                              // per chunk-start state tile
   uint64_t qdone[kStages];                           // Qh' of the staged chunk copied out
-  uint64_t o_full[2], o_free[2];                     // per output pair
-  uint64_t agg_pub, p2_go, mma_final[2];
+  uint64_t o_full[kOPairs], o_free[kOPairs];         // per output pair
+  uint64_t agg_pub, p2_go, mma_final[2], corr_done[kOPairs];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
   uint32_t tmem_base;
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
+  alignas(16) float drecv[kMaxCluster][64];  // CLUSTER: every segment's log2 decay per key channel
   alignas(16) float red[2][2][4][32];  // WG_A cumsum: per warpgroup, channel half and warp, channel totals
   alignas(16) float eseg[64];          // Qh' warp: 2^(decay from the segment start) per channel
   int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
@@ -412,7 +418,7 @@ struct Span {
 // Chunk run of segment s: one contiguous, balanced run per segment (STREAM: the whole
 // sequence).  With n_s <= Nc every segment holds at least one chunk.
 __device__ __forceinline__ Span seg_span(const FusedParams& fp, int s) {
-  if (fp.mode == 0) return Span{0, fp.Nc};
+  if (fp.mode == 0) return Span{0, fp.Nc};  // (SEGMENTED and CLUSTER: balanced runs)
   return Span{(int)((long long)s * fp.Nc / fp.n_s), (int)((long long)(s + 1) * fp.Nc / fp.n_s)};
 }
 
@@ -517,14 +523,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   WsHeader* hdr = fp.hdr;
 
   const bool segm = fp.mode == 1;          // the CTAs of a sequence exchange segment summaries
-  const int seq = segm ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
-  const int seg = segm ? (int)blockIdx.x % fp.n_s : 0;
+  const bool clus = fp.mode == 2;          // ... through distributed shared memory, outputs held on chip
+  const int seq = (segm || clus) ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
+  const int seg = (segm || clus) ? (int)blockIdx.x % fp.n_s : 0;
   const bool partial = segm && seg > 0;    // outputs completed in the second phase
+  const bool qhw = (segm || clus) && seg > 0;  // Qh' tiles go to the workspace (the Qh' warp)
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
   const Span sp = seg_span(fp, seg);
   const int cnt = sp.c1 - sp.c0;           // chunks of this CTA
   float nonfinite = 0.f;
+  bool cwaited = false;                    // CLUSTER: this thread has passed the start barrier
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -540,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->pready[i], 4);  // every WG_B warp
     }
     for (int i = 0; i < kNS; ++i) mbar_init(&ms->sready[i], 4);  // every WG_B warp
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kOPairs; ++i) {
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
     }
@@ -548,8 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->p2_full[i], 1);
       mbar_init(&ms->p2_mma[i], 1);
     }
-    mbar_init(&ms->agg_pub, partial ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
+    mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
     mbar_init(&ms->p2_go, 1);
+    for (int i = 0; i < kOPairs; ++i) mbar_init(&ms->corr_done[i], 1);
     mbar_init(&ms->mma_final[0], 1);
     mbar_init(&ms->mma_final[1], 1);
     ms->abort = 0;
@@ -564,6 +574,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
+  // CLUSTER: a CTA's shared memory is written by the others only once every CTA of the
+  // cluster has started (the matching wait comes before the first remote access)
+  if (clus) cluster_arrive_relaxed();
 
   if (warp == 16) {
     // ===================================================================== producer
@@ -573,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // in a segment s > 0, that chunk's Qh' has been copied out.
     auto stage_free = [&](int n, int st) -> bool {
       if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) return false;
-      return !partial || wait_bar(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
+      return !qhw || wait_bar(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
     };
     if (fp.tma) {
       // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
@@ -667,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (the sum of the earlier chunks' decays, row 0 of their gate tiles) and takes the
     // 16-byte pieces l, l+32, ... of the tile, so every store instruction writes 512
     // contiguous bytes.
-    if (partial) {
+    if (qhw) {
       bool ok = true;
       float a2s0 = 0.f, a2s1 = 0.f;
       const float* eseg = ms->eseg;
@@ -695,11 +708,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           v.w = h2_bits(__hmul2(bits_h2(v.w), __floats2half2_rn(e1.z, e1.w)));
           *reinterpret_cast<uint4*>(dst + r * 128 + 16 * jp) = v;
         }
-        // the tile is read back by bulk copy (async proxy); the staged chunk is released
-        asm volatile("fence.proxy.async.global;" ::: "memory");
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ms->qdone[st]);
+        if (lane == 0) mbar_arrive(&ms->qdone[st]);  // the staged chunk is released
       }
+      // the tiles are read back by bulk copy (async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
       __syncwarp();
       if (lane == 0 && ok) mbar_arrive(&ms->agg_pub);
     }
@@ -746,12 +759,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int m = 0; m < cnt; ++m) {
         const int st = m % kStages, su = m % kSU;
         // output region of chunk m: pair (m/2) % 2, lane tile m % 2
-        const uint32_t d_o = tmem + kColO + 64u * (uint32_t)((m >> 1) & 1) + ((m & 1) ? kLaneTile1 : 0u);
+        const uint32_t d_o = tmem + kColO + 64u * (uint32_t)((m >> 1) % kOPairs) + ((m & 1) ? kLaneTile1 : 0u);
         // Qh built (the stage-1 issuer waits on the same phase; neither can lap it, as the
         // stage is refilled only after this chunk's P V), chunk-start state written
         if (!wait_spin(&ms->opready[st], ph_use<kStages>(m), ms, hdr, 0x205)) break;
         if (!wait_spin(&ms->sready[m % kNS], ph_use<kNS>(m), ms, hdr, 0x202)) break;
-        if (!(m & 1) && !wait_spin(&ms->o_free[(m >> 1) & 1], ph_rel<2>(m >> 1), ms, hdr, 0x203)) break;
+        if (!(m & 1) && !wait_spin(&ms->o_free[(m >> 1) % kOPairs], ph_rel<kOPairs>(m >> 1), ms, hdr, 0x203)) break;
         const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
         const uint32_t a_s = s_base + kOffS + (m % kNS) * kTile;
         tc_fence_after();
@@ -766,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16_ta(d_o, a_p + 8 * k, sw128_desc(a_v + 2048 * k), id_qs, 1);
         mma_commit(&ms->su_free[su]);
         mma_commit(&ms->empty[st]);
-        if ((m & 1) || m + 1 == cnt) mma_commit(&ms->o_full[(m >> 1) & 1]);
+        if ((m & 1) || m + 1 == cnt) mma_commit(&ms->o_full[(m >> 1) % kOPairs]);
       }
       mma_commit(&ms->mma_final[1]);
       const uint64_t t0 = globaltimer();
@@ -1072,6 +1085,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // every thread leaves the loop (the waits are bounded): agree on the outcome
     alive = wg_all(wg, alive);
+    if (clus && alive) {
+      // the segment summary goes straight to the CTAs that scan it: entry pair (key kk,
+      // values v0, v0+1) is unit u = 32 kk + v0/2, owned by rank r = ((u+1) n_s - 1) / 2048
+      // (units [r 2048/n_s, (r+1) 2048/n_s)), and lands in the owner's receive area (its
+      // idle output staging) at [this segment][u - first unit of r]; the log2 decays go to
+      // every CTA of the cluster
+      cluster_wait();  // (every CTA has started)
+      cwaited = true;
+      const int ns = fp.n_s;
+      const uint32_t recv = smem_u32(smem + kOffStg);
+#pragma unroll
+      for (int cb = 0; cb < 8; ++cb) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int kk = hr ? r1 : r0;
+          const int u = kk * 32 + ((8 * cb + cq) >> 1);
+          const int r = ((u + 1) * ns - 1) / 2048;
+          const int ub = r * 2048 / ns, nu = (r + 1) * 2048 / ns - ub;
+          st_cluster_f32x2(cluster_map(recv + (uint32_t)((seg * nu + (u - ub)) * 8), (uint32_t)r),
+                           make_float2(Ls[4 * cb + 2 * hr], Ls[4 * cb + 2 * hr + 1]));
+        }
+      }
+      if ((lane & 3) == 0)
+        for (int j = 0; j < ns; ++j) {
+          st_cluster_f32(cluster_map(smem_u32(&ms->drecv[seg][r0]), (uint32_t)j), a2r0);
+          st_cluster_f32(cluster_map(smem_u32(&ms->drecv[seg][r1]), (uint32_t)j), a2r1);
+        }
+      wg_sync(wg);
+      if (wtid == 0) mbar_arrive(&ms->agg_pub);
+    }
     if (segm && alive) {
       // segment summary: U_seg = local end state, its log2 decay
       float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * (4096 + 64);
@@ -1098,17 +1141,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
     bool alive = true;
-    {
+    if (clus) {
+      // the outputs stay in tensor memory until the start state is known: wait for their
+      // last MMAs; then (segments s > 0) the chunks' Qh' tiles start loading into the idle
+      // staging buffers
+      for (int pr = 0; pr < (cnt + 1) / 2 && alive; ++pr)
+        alive = wg_wait(wg, wtid, &ms->o_full[pr], 0u, ms, hdr, 0x520, slot);
+      if (alive && seg > 0 && wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x521, slot) && wtid == 0) {
+        mbar_arrive_expect_tx(&ms->p2_full[0], (uint32_t)(cnt * kTile));
+        for (int g = 0; g < cnt; g += 2) {
+          const int nb = min(2, cnt - g);
+          bulk_load(smem + kOffStage + g * kTile, fp.qhp + ((size_t)seq * fp.Nc + sp.c0 + g) * 4096,
+                    (uint32_t)(nb * kTile), &ms->p2_full[0]);
+        }
+      }
+    } else {
       // this CTA's chunks; in a segment s > 0 the outputs are partial: fp16 rows of the
       // workspace, completed in the second phase
       const int pairs = (cnt + 1) / 2;
       for (int pr = 0; pr < pairs; ++pr) {
-        if (!wg_wait(wg, wtid, &ms->o_full[pr & 1], ph_use<2>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
+        if (!wg_wait(wg, wtid, &ms->o_full[pr % kOPairs], ph_use<kOPairs>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
         const int ci = 2 * pr + tsel;
         const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
         const bool valid = ci < cnt && s < L;
-        const uint32_t src = tl + kColO + 64u * (uint32_t)(pr & 1);
+        const uint32_t src = tl + kColO + 64u * (uint32_t)(pr % kOPairs);
         if (partial) {
           uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp.c0 + ci) * 4096) + trow * 128
                               : nullptr;
@@ -1118,7 +1175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->o_free[pr & 1]);
+        if (wtid == 0) mbar_arrive(&ms->o_free[pr % kOPairs]);
       }
       // the O_local rows written above are read back by bulk copy (async proxy)
       if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -1236,6 +1293,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (clus) {
+    // ===================================================================== CLUSTER combine
+    // The n_s CTAs of a sequence form one cluster.  Every thread of every CTA meets at the
+    // cluster barrier (all waits before it are bounded): the summaries are delivered and
+    // every MMA of the cluster has completed.  CTA rank r then composes its units over the
+    // n_s segments from its receive area and writes each segment's start state (fp16, MMA
+    // layout) into that segment's CTA; after a second barrier every CTA holds its own.
+    if (!cwaited) cluster_wait();
+    __syncwarp();
+    cluster_sync_all();
+    if (tid < 4 * kWG) {
+      const int ns = fp.n_s;
+      const int u0 = seg * 2048 / ns, u1 = (seg + 1) * 2048 / ns, nu = u1 - u0;
+      for (int u = u0 + tid; u < u1; u += 4 * kWG) {  // (more than one unit a thread below 4 CTAs)
+        const int kk = u >> 5, v0 = 2 * (u & 31);  // key channel, value pair
+        const float2* rv = reinterpret_cast<const float2*>(smem + kOffStg) + (u - u0);
+        const uint32_t a_s = smem_u32(smem + kOffSst) + (uint32_t)kk * 128u +
+                             ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (uint32_t)(v0 & 7) * 2u;
+        float2 X = make_float2(0.f, 0.f);
+        for (int j = 0; j < ns; ++j) {
+          st_cluster_u32(cluster_map(a_s, (uint32_t)j), pack_h2(X.x, X.y));
+          const float2 uj = rv[j * nu];
+          const float d = ex2(ms->drecv[j][kk]);
+          X = make_float2(fmaf(d, X.x, uj.x), fmaf(d, X.y, uj.y));
+        }
+      }
+    }
+    asm volatile("fence.proxy.async;" ::: "memory");  // the start states are read by the MMA (async proxy)
+    __syncwarp();
+    cluster_sync_all();
+    if (tid < 4 * kWG) {
+      // outputs += Qh' S_start (segments s > 0; issued by one thread, one commit per pair),
+      // then the epilogue of the held pairs: warpgroup q (warps 4q .. 4q+3) takes pair q
+      const int q = warp >> 2, wtid = tid - kWG * q, wq = warp & 3;
+      const int trow = wq * 16 + (lane & 15), tsel = lane >> 4;
+      const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+      // staging: warpgroup 3 over the receive area (read out), the others past the Qh' tiles
+      uint8_t* wstage = (q == 3 ? smem + kOffStg : smem + kOffStage + kClusterChunks * kTile + q * 4 * 32 * 128) +
+                        wq * 32 * 128;
+      const int npairs = (cnt + 1) / 2;
+      int slot = 0;
+      if (seg > 0 && q == 3 && wtid == 0 && wait_bar(&ms->p2_full[0], 0u, ms, hdr, 0x530)) {
+        const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
+        const uint32_t s_base = smem_u32(smem);
+        tc_fence_after();
+        for (int g = 0; g < cnt; ++g) {
+          const uint32_t d_o = tmem + kColO + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
+          const uint32_t a_q = s_base + kOffStage + g * kTile;  // the chunk's Qh'
+          for (int k = 0; k < 4; ++k)
+            mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
+          if ((g & 1) || g + 1 == cnt) mma_commit(&ms->corr_done[g >> 1]);
+        }
+      }
+      for (int pr = q; pr < npairs; pr += 4) {
+        if (seg > 0 && !wg_wait(q, wtid, &ms->corr_done[pr], 0u, ms, hdr, 0x531, slot)) break;
+        tc_fence_after();
+        const int ci = 2 * pr + tsel;
+        const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
+        epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(p, b, h, ci < cnt && s < L, s), wstage,
+                            lane, nonfinite);
+      }
+    }
+  }
+
   if (__any_sync(0xffffffffu, nonfinite != nonfinite) && lane == 0) record_error(hdr, GTR_ERR_RANGE, 0x500u + warp);
 
   // ---- teardown
@@ -1345,6 +1466,39 @@ size_t seg_capacity(const Problem& p) {
   return n_seq * 2 <= kMaxSegCtas ? n_seq * (kMaxSegCtas / n_seq) : 0;
 }
 
+// Clusters of `cs` CTAs of this kernel the device can hold at once (cached per device,
+// direction kind and size).
+template <typename K>
+int max_active_clusters(K kern, int dev, bool rev, int cs) {
+  static int cache[64][2][kMaxCluster + 1];
+  static std::once_flag once;
+  static std::mutex mu;
+  std::call_once(once, [] {
+    for (auto& a : cache)
+      for (auto& b : a)
+        for (int& c : b) c = -1;
+  });
+  std::lock_guard<std::mutex> lock(mu);
+  int& c = cache[dev][rev ? 1 : 0][cs];
+  if (c < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    c = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess ? n : 0;
+    (void)cudaGetLastError();  // a refused size only means no cluster mode
+  }
+  return c;
+}
+
 template <typename Tin, typename Tout>
 gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
   const bool rev = p.direction == GTR_R2L || p.direction == GTR_B2T;
@@ -1353,11 +1507,32 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
   if (!(configured[rev].load() & (1ull << dev))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return GTR_ERR_CUDA;
     configured[rev].fetch_or(1ull << dev);
   }
   Plan pl = make_plan(p, device_sms());
+  if (pl.mode == 1 && force_mode < 0) {
+    // short sequences: one cluster per sequence (the largest size the device holds for
+    // every sequence at once), at most kClusterChunks chunks per CTA; then the fewest
+    // CTAs that keep the longest run
+    const int Nc = p.n_chunks();
+    int best_k = kClusterChunks + 1;
+    for (int cs = kMaxCluster; cs >= 2; --cs) {
+      if (max_active_clusters(kern, dev, rev, cs) < pl.n_seq) continue;
+      const int k = (Nc + cs - 1) / cs;
+      if (k < best_k) best_k = k;
+    }
+    if (best_k <= kClusterChunks) {
+      const int cs = (Nc + best_k - 1) / best_k;
+      if (cs >= 2 && max_active_clusters(kern, dev, rev, cs) >= pl.n_seq) {
+        pl.mode = 2;
+        pl.n_s = cs;
+        pl.grid = pl.n_seq * cs;
+      }
+    }
+  }
   if (force_mode == 0) {
     pl.mode = 0;
     pl.n_s = 1;
@@ -1403,8 +1578,15 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;  // the CTAs of a sequence wait on one another
+  if (pl.mode == 2) {  // one cluster per sequence
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.n_s;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;  // the CTAs of a sequence wait on one another
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;

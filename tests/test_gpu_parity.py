@@ -313,3 +313,16 @@ def test_segmented_calls_in_alternating_directions_match_the_oracle(name):
             err = rel_err(out, refs[d])
             assert err <= TOL[w.dtype], f"{name} rep={rep} dir={d}: max err / rms = {err:.3e}"
     assert gtr.read_error() == 0
+
+
+# ------------------------------------------------------------------ cluster sizes
+@pytest.mark.parametrize("shape", [(1, 1, 8, 16), (1, 1, 8, 24), (1, 2, 9, 16), (2, 2, 5, 13), (1, 1, 32, 96)])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_short_sequences_over_clusters_of_every_size(shape, dtype):
+    """Short sequences are split over one thread-block cluster each (2 to 16 CTAs, one to
+    eight chunks a CTA): with fewer than four CTAs a scanning thread owns several state
+    entries, and a ragged last chunk leaves rows past the sequence end in its segment."""
+    B, heads, H, W = shape
+    w = Workload("cl", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=0.5)
+    for d in range(4):
+        check(w, d, seed=31 + d, path="fused")
