@@ -535,35 +535,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   float nonfinite = 0.f;
   bool cwaited = false;                    // CLUSTER: this thread has passed the start barrier
 
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
+  // The next launch may start its prologue now (programmatic dependent launch): it waits
+  // for this grid to complete before it touches global memory.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  static_assert(kStages <= 8 && kSU <= 8 && kNS <= 8 && kOPairs <= 8, "barrier arrays fit lanes 0-7");
+  if (warp == 0) {  // lane i initialises entry i of every barrier array (a few inits a lane)
+    const int i = lane;
+    if (i < kStages) {
       mbar_init(&ms->full[i], fp.tma ? 1 : kProducerThreads);
       mbar_init(&ms->empty[i], 1);
       mbar_init(&ms->opready[i], 4);  // every warp of the WG_A warpgroup that builds the chunk
       mbar_init(&ms->qdone[i], 1);
       ms->fb[i] = 0;
     }
-    for (int i = 0; i < kSU; ++i) {
+    if (i < kSU) {
       mbar_init(&ms->su_full[i], 1);
       mbar_init(&ms->su_free[i], 1);
       mbar_init(&ms->pready[i], 4);  // every WG_B warp
     }
-    for (int i = 0; i < kNS; ++i) mbar_init(&ms->sready[i], 4);  // every WG_B warp
-    for (int i = 0; i < kOPairs; ++i) {
+    if (i < kNS) mbar_init(&ms->sready[i], 4);  // every WG_B warp
+    if (i < kOPairs) {
       mbar_init(&ms->o_full[i], 1);
       mbar_init(&ms->o_free[i], 1);
+      mbar_init(&ms->corr_done[i], 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    if (i < 4) {
       mbar_init(&ms->p2_full[i], 1);
       mbar_init(&ms->p2_mma[i], 1);
+      ms->go[i][0] = ms->go[i][1] = 0;
     }
-    mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
-    mbar_init(&ms->p2_go, 1);
-    for (int i = 0; i < kOPairs; ++i) mbar_init(&ms->corr_done[i], 1);
-    mbar_init(&ms->mma_final[0], 1);
-    mbar_init(&ms->mma_final[1], 1);
-    ms->abort = 0;
-    for (int i = 0; i < 4; ++i) ms->go[i][0] = ms->go[i][1] = 0;
+    if (i == 8) mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
+    if (i == 9) mbar_init(&ms->p2_go, 1);
+    if (i == 10) mbar_init(&ms->mma_final[0], 1);
+    if (i == 11) mbar_init(&ms->mma_final[1], 1);
+    if (i == 12) ms->abort = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -574,6 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
+  // every global access of this grid comes after the previous grid in the stream has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // CLUSTER: a CTA's shared memory is written by the others only once every CTA of the
   // cluster has started (the matching wait comes before the first remote access)
   if (clus) cluster_arrive_relaxed();
@@ -1577,18 +1584,26 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int na = 0;
   if (pl.mode == 2) {  // one cluster per sequence
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.n_s;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-  } else {
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = pl.mode == 1 ? 1 : 0;  // the CTAs of a sequence wait on one another
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = pl.n_s;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pl.mode == 1) {  // the CTAs of a sequence wait on one another
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  } else {  // the prologue may overlap the previous launch's tail
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
   }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;
   return GTR_OK;
 }
