@@ -77,7 +77,7 @@ constexpr int kNS = 5;                                     // chunk-start state 
 constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [kNS] chunk-start states
 constexpr int kOffSst = kOffS;                             // segment start state (after the chunks: over state tile 0)
 constexpr int kOffStg = kOffS + kNS * kTile;               // output staging, 4 warps x 32 rows x 128 B
-constexpr int kStgBytes = 4 * 32 * 128 + 1024;             // (CLUSTER: the summary slices received, <= 16464 B)
+constexpr int kStgBytes = 4 * 32 * 128;                    // (CLUSTER: first the segment summary, fp32)
 constexpr int kOffMisc = kOffStg + kStgBytes;
 constexpr int kMiscBytes = 8192;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
@@ -140,7 +140,7 @@ struct Misc {
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
-  alignas(16) float drecv[kMaxCluster][64];  // CLUSTER: every segment's log2 decay per key channel
+  alignas(16) float dseg[64];  // CLUSTER: this segment's log2 decay per key channel (read by the cluster)
   alignas(16) float red[2][2][4][32];  // WG_A cumsum: per warpgroup, channel half and warp, channel totals
   alignas(16) float eseg[64];          // Qh' warp: 2^(decay from the segment start) per channel
   int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
@@ -1093,32 +1093,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every thread leaves the loop (the waits are bounded): agree on the outcome
     alive = wg_all(wg, alive);
     if (clus && alive) {
-      // the segment summary goes straight to the CTAs that scan it: entry pair (key kk,
-      // values v0, v0+1) is unit u = 32 kk + v0/2, owned by rank r = ((u+1) n_s - 1) / 2048
-      // (units [r 2048/n_s, (r+1) 2048/n_s)), and lands in the owner's receive area (its
-      // idle output staging) at [this segment][u - first unit of r]; the log2 decays go to
-      // every CTA of the cluster
-      cluster_wait();  // (every CTA has started)
-      cwaited = true;
-      const int ns = fp.n_s;
-      const uint32_t recv = smem_u32(smem + kOffStg);
+      // segment summary for the cluster's scan, read by the other CTAs after the cluster
+      // barrier: U_seg (fp32, row-major) over the output staging area (idle: the outputs
+      // are held), the log2 decay per key channel in the misc area
+      float* U = reinterpret_cast<float*>(smem + kOffStg);
 #pragma unroll
       for (int cb = 0; cb < 8; ++cb) {
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int kk = hr ? r1 : r0;
-          const int u = kk * 32 + ((8 * cb + cq) >> 1);
-          const int r = ((u + 1) * ns - 1) / 2048;
-          const int ub = r * 2048 / ns, nu = (r + 1) * 2048 / ns - ub;
-          st_cluster_f32x2(cluster_map(recv + (uint32_t)((seg * nu + (u - ub)) * 8), (uint32_t)r),
-                           make_float2(Ls[4 * cb + 2 * hr], Ls[4 * cb + 2 * hr + 1]));
-        }
+        *reinterpret_cast<float2*>(U + r0 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb], Ls[4 * cb + 1]);
+        *reinterpret_cast<float2*>(U + r1 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]);
       }
-      if ((lane & 3) == 0)
-        for (int j = 0; j < ns; ++j) {
-          st_cluster_f32(cluster_map(smem_u32(&ms->drecv[seg][r0]), (uint32_t)j), a2r0);
-          st_cluster_f32(cluster_map(smem_u32(&ms->drecv[seg][r1]), (uint32_t)j), a2r1);
-        }
+      if ((lane & 3) == 0) {
+        ms->dseg[r0] = a2r0;
+        ms->dseg[r1] = a2r1;
+      }
       wg_sync(wg);
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
     }
@@ -1312,18 +1299,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_sync_all();
     if (tid < 4 * kWG) {
       const int ns = fp.n_s;
-      const int u0 = seg * 2048 / ns, u1 = (seg + 1) * 2048 / ns, nu = u1 - u0;
+      const int u0 = seg * 2048 / ns, u1 = (seg + 1) * 2048 / ns;
       for (int u = u0 + tid; u < u1; u += 4 * kWG) {  // (more than one unit a thread below 4 CTAs)
         const int kk = u >> 5, v0 = 2 * (u & 31);  // key channel, value pair
-        const float2* rv = reinterpret_cast<const float2*>(smem + kOffStg) + (u - u0);
+        const uint32_t a_u = smem_u32(smem + kOffStg) + (uint32_t)(kk * 64 + v0) * 4u;
+        const uint32_t a_d = smem_u32(&ms->dseg[kk]);
         const uint32_t a_s = smem_u32(smem + kOffSst) + (uint32_t)kk * 128u +
                              ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (uint32_t)(v0 & 7) * 2u;
+        // every segment's summary entries first (the remote loads overlap), then the
+        // sequential composition
+        float2 uj[kMaxCluster];
+        float dj[kMaxCluster];
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+          if (j < ns) {
+            uj[j] = ld_cluster_f32x2(cluster_map(a_u, (uint32_t)j));
+            dj[j] = ld_cluster_f32(cluster_map(a_d, (uint32_t)j));
+          }
+        }
         float2 X = make_float2(0.f, 0.f);
-        for (int j = 0; j < ns; ++j) {
-          st_cluster_u32(cluster_map(a_s, (uint32_t)j), pack_h2(X.x, X.y));
-          const float2 uj = rv[j * nu];
-          const float d = ex2(ms->drecv[j][kk]);
-          X = make_float2(fmaf(d, X.x, uj.x), fmaf(d, X.y, uj.y));
+#pragma unroll
+        for (int j = 0; j < kMaxCluster; ++j) {
+          if (j < ns) {
+            st_cluster_u32(cluster_map(a_s, (uint32_t)j), pack_h2(X.x, X.y));
+            const float d = ex2(dj[j]);
+            X = make_float2(fmaf(d, X.x, uj[j].x), fmaf(d, X.y, uj[j].y));
+          }
         }
       }
     }
