@@ -150,6 +150,7 @@ struct Misc {
 // in row 1; the summary scan exchanges its block transfers through the segment-start-
 // state tile, which is idle at that point.
 static_assert(sizeof(Misc) <= kMiscBytes, "misc area too small");
+static_assert(sizeof(Misc::red) >= kStages * 64 * sizeof(float), "the in-place Qh' factors fit the cumsum exchange");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -527,11 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int seq = (segm || clus) ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
   const int seg = (segm || clus) ? (int)blockIdx.x % fp.n_s : 0;
   const bool partial = segm && seg > 0;    // outputs completed in the second phase
-  const bool qhw = (segm || clus) && seg > 0;  // Qh' tiles go to the workspace (the Qh' warp)
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
   const Span sp = seg_span(fp, seg);
   const int cnt = sp.c1 - sp.c0;           // chunks of this CTA
+  // CLUSTER with at most kStages chunks a CTA: the staging buffers are never refilled, so
+  // each chunk's Qh stays in its own and becomes Qh' in place at the end
+  const bool inplace = clus && cnt <= kStages;
+  const bool qhw = (segm || clus) && seg > 0 && !inplace;  // Qh' tiles go to the workspace (the Qh' warp)
   float nonfinite = 0.f;
   bool cwaited = false;                    // CLUSTER: this thread has passed the start barrier
 
@@ -1141,7 +1145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // staging buffers
       for (int pr = 0; pr < (cnt + 1) / 2 && alive; ++pr)
         alive = wg_wait(wg, wtid, &ms->o_full[pr], 0u, ms, hdr, 0x520, slot);
-      if (alive && seg > 0 && wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x521, slot) && wtid == 0) {
+      if (alive && qhw && wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x521, slot) && wtid == 0) {
         mbar_arrive_expect_tx(&ms->p2_full[0], (uint32_t)(cnt * kTile));
         for (int g = 0; g < cnt; g += 2) {
           const int nb = min(2, cnt - g);
@@ -1328,7 +1332,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    asm volatile("fence.proxy.async;" ::: "memory");  // the start states are read by the MMA (async proxy)
+    if (inplace && seg > 0 && tid < 4 * kWG) {
+      // Qh' = Qh 2^(decay from the segment start) in place: per chunk and channel the factor
+      // sums row 0 (the decay a) of the earlier chunks' gate tiles, then every 16-byte piece
+      // of the tiles is scaled
+      float* fac = &ms->red[0][0][0][0];  // [cnt][64] (the cumsum exchange is idle now)
+      if (tid < cnt * 64) {
+        const int g = tid >> 6, ch = tid & 63;
+        float a2 = 0.f;
+        for (int j = 0; j < g; ++j)
+          a2 += reinterpret_cast<const float*>(smem + kOffStage + j * kStageBytes + 3 * kTile)[ch];
+        fac[tid] = ex2(a2);
+      }
+      asm volatile("bar.sync 7, 512;" ::: "memory");
+      for (int i = tid; i < cnt * 512; i += 4 * kWG) {
+        const int g = i >> 9, pi = i & 511, r = pi >> 3, jp = pi & 7, jl = jp ^ (r & 7);
+        uint4* ptr = reinterpret_cast<uint4*>(smem + kOffStage + g * kStageBytes + r * 128 + 16 * jp);
+        const float4 f0 = *reinterpret_cast<const float4*>(fac + g * 64 + 8 * jl);
+        const float4 f1 = *reinterpret_cast<const float4*>(fac + g * 64 + 8 * jl + 4);
+        uint4 v = *ptr;
+        v.x = h2_bits(__hmul2(bits_h2(v.x), __floats2half2_rn(f0.x, f0.y)));
+        v.y = h2_bits(__hmul2(bits_h2(v.y), __floats2half2_rn(f0.z, f0.w)));
+        v.z = h2_bits(__hmul2(bits_h2(v.z), __floats2half2_rn(f1.x, f1.y)));
+        v.w = h2_bits(__hmul2(bits_h2(v.w), __floats2half2_rn(f1.z, f1.w)));
+        *ptr = v;
+      }
+    }
+    // the start states and the in-place Qh' are read by the MMA (async proxy)
+    asm volatile("fence.proxy.async;" ::: "memory");
     __syncwarp();
     cluster_sync_all();
     if (tid < 4 * kWG) {
@@ -1337,18 +1368,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q = warp >> 2, wtid = tid - kWG * q, wq = warp & 3;
       const int trow = wq * 16 + (lane & 15), tsel = lane >> 4;
       const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-      // staging: warpgroup 3 over the receive area (read out), the others past the Qh' tiles
-      uint8_t* wstage = (q == 3 ? smem + kOffStg : smem + kOffStage + kClusterChunks * kTile + q * 4 * 32 * 128) +
+      // staging: warpgroup 3 over the summary area (read out), the others past the Qh' tiles
+      // (in place: over the K and V tiles of stages 0-2)
+      uint8_t* wstage = (q == 3 ? smem + kOffStg
+                                : (inplace ? smem + kOffStage + q * kStageBytes + kTile
+                                           : smem + kOffStage + kClusterChunks * kTile + q * 4 * 32 * 128)) +
                         wq * 32 * 128;
       const int npairs = (cnt + 1) / 2;
       int slot = 0;
-      if (seg > 0 && q == 3 && wtid == 0 && wait_bar(&ms->p2_full[0], 0u, ms, hdr, 0x530)) {
+      if (seg > 0 && q == 3 && wtid == 0 && (inplace || wait_bar(&ms->p2_full[0], 0u, ms, hdr, 0x530))) {
         const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
         const uint32_t s_base = smem_u32(smem);
         tc_fence_after();
         for (int g = 0; g < cnt; ++g) {
           const uint32_t d_o = tmem + kColO + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
-          const uint32_t a_q = s_base + kOffStage + g * kTile;  // the chunk's Qh'
+          const uint32_t a_q = s_base + kOffStage + g * (inplace ? kStageBytes : kTile);  // the chunk's Qh'
           for (int k = 0; k < 4; ++k)
             mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
           if ((g & 1) || g + 1 == cnt) mma_commit(&ms->corr_done[g >> 1]);
