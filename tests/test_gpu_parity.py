@@ -326,3 +326,47 @@ def test_short_sequences_over_clusters_of_every_size(shape, dtype):
     w = Workload("cl", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=0.5)
     for d in range(4):
         check(w, d, seed=31 + d, path="fused")
+
+
+# ------------------------------------------------------------------ launches back to back
+def test_graph_of_calls_in_every_plan_matches_the_oracle():
+    """One CUDA graph holding calls of every plan back to back -- cluster, segmented
+    (cooperative), one CTA per sequence, and the split path -- each with its own
+    workspace: a launch that overlaps its prologue with the previous one must still see
+    that one's results (and leave its workspace ready), replay after replay."""
+    cases = [
+        (Workload("cl", B=1, heads=6, H=40, W=40, dtype="f16", scale=0.5), 1, "auto"),    # cluster
+        (Workload("sg", B=1, heads=2, H=128, W=112, dtype="f16", scale=0.5), 3, "auto"),  # segmented
+        (Workload("st", B=13, heads=6, H=8, W=16, dtype="bf16"), 2, "auto"),              # one CTA each
+        (Workload("cl2", B=2, heads=2, H=5, W=13, dtype="bf16"), 0, "auto"),              # small clusters
+        (Workload("sp", B=1, heads=2, H=16, W=16, dtype="f32"), 1, "split"),
+    ]
+    dev = torch.device("cuda:0")
+    runs = []
+    for w, d, path in cases:
+        q, k, v, lg = make_inputs(w, 57)
+        ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, d)
+        tq, tk, tv, tg = (t.to(dev) for t in (q, k, v, lg))
+        in_dtype = {"f32": 0, "f16": 1, "bf16": 2}[w.dtype]
+        ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, in_dtype=in_dtype, path=path, device=dev)
+        out = gtr.gla_fwd(tq, tk, tv, tg, grid=(w.H, w.W), direction=d, path=path, workspace=ws)
+        runs.append((w, d, path, tq, tk, tv, tg, ws, out, ref))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(2):
+            for w, d, path, tq, tk, tv, tg, ws, out, ref in runs:
+                gtr.gla_fwd(tq, tk, tv, tg, grid=(w.H, w.W), direction=d, path=path, workspace=ws, out=out,
+                            stream=stream)
+    for rep in range(3):
+        for _, _, _, _, _, _, _, _, out, _ in runs:
+            out.fill_(float("nan"))
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        for w, d, path, _, _, _, _, ws, out, ref in runs:
+            err = rel_err(out, ref)
+            assert err <= TOL[w.dtype], f"{w.name} rep={rep}: max err / rms = {err:.3e}"
+            assert gtr.read_error(ws) == 0, f"{w.name} rep={rep}: device error"
+    del g
