@@ -105,6 +105,23 @@ constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
 constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
+// floor(n / d) for 0 <= n < 2^31 by one wide multiply and a shift: with l = ceil(log2 d)
+// and m = ceil(2^(31+l) / d) (m < 2^32), floor(n m / 2^(31+l)) = floor(n / d) for every
+// such n (Granlund and Montgomery, "Division by Invariant Integers using Multiplication",
+// PLDI 1994, Theorem 4.2 with N = 31).  The scan remap divides by the grid width or
+// height for every staged row and every stored output row.
+struct FastDiv {
+  uint32_t m, sh;  // multiplier and total shift 31 + l
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  return FastDiv{(uint32_t)(((1ull << (31 + l)) + d - 1) / d), 31 + l};
+}
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
+  return (uint32_t)(((unsigned long long)n * f.m) >> f.sh);
+}
+
 struct alignas(64) FusedParams {
   // TMA tensor maps for Q, K, V (16-bit, 128-byte swizzle) and the log-gates (fp32):
   // row view [B][L][heads][64] (4-D) or column view [B][H][W][heads][64] (5-D), boxes of
@@ -120,9 +137,28 @@ struct alignas(64) FusedParams {
   int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED, 2 = CLUSTER
   int grid;
   float max_exp2;          // largest in-chunk log2-decay the score factorisation takes
-  int tma;                 // 1: every chunk is one TMA box per tensor; 0: cp.async row copies
+  int tma;                 // 1: one TMA box per tensor; 2: 4-row TMA gathers; 0: cp.async row copies
   int rev;                 // 1: chunks are staged in reverse scan order (right-to-left, bottom-to-top)
+  FastDiv divW, divH;      // the grid width and height as invariant divisors
 };
+
+// Scan position s (< L < 2^31) -> token index y*W + x: the direction remap (rows top to
+// bottom, left to right or right to left; columns left to right, top to bottom or bottom
+// to top), with the division by W or H done by multiplication.
+__device__ __forceinline__ uint32_t scan_token(const FusedParams& fp, uint32_t s) {
+  const uint32_t W = (uint32_t)fp.p.W, H = (uint32_t)fp.p.H;
+  uint32_t x, y;
+  if (fp.p.direction <= GTR_R2L) {
+    y = fast_div(s, fp.divW);
+    x = s - y * W;
+    if (fp.p.direction == GTR_R2L) x = W - 1 - x;
+  } else {
+    x = fast_div(s, fp.divH);
+    y = s - x * H;
+    if (fp.p.direction == GTR_B2T) y = H - 1 - y;
+  }
+  return y * W + x;
+}
 static_assert(alignof(FusedParams) >= 64, "tensor maps need 64-byte alignment");
 
 struct Misc {
@@ -358,10 +394,10 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, u
 
 // Grid-cell destination of output row s of (b, h), or nullptr when not `valid`.
 template <typename Tout>
-__device__ __forceinline__ uint8_t* out_row(const Problem& p, int b, int h, bool valid, long long s) {
+__device__ __forceinline__ uint8_t* out_row(const FusedParams& fp, int b, int h, bool valid, long long s) {
   if (!valid) return nullptr;
-  const long long m = ((long long)b * p.L() + scan_to_token(s, p.direction, p.H, p.W)) * p.heads + h;
-  return reinterpret_cast<uint8_t*>(reinterpret_cast<Tout*>(p.out) + m * 64);
+  const long long m = ((long long)b * fp.p.L() + scan_token(fp, (uint32_t)s)) * fp.p.heads + h;
+  return reinterpret_cast<uint8_t*>(reinterpret_cast<Tout*>(fp.p.out) + m * 64);
 }
 
 // Segmented mode, second phase: the 32 rows of one warp hold the correction Qh' S_start
@@ -504,7 +540,7 @@ __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uin
     const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
     const uint8_t* olc_rows = sbuf + kP2Olc + (wq >> 1) * kTile + 32 * (wq & 1) * 128;
     // fp32 staging over the pair's Qh' (its MMA has completed)
-    epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp.p, b, h, ci < cnt && s < L, s),
+    epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp, b, h, ci < cnt && s < L, s),
                             olc_rows, sbuf + wq * 4096, lane, nf);
     tc_fence_before();
     fence_proxy_async_smem();  // generic accesses of the buffer before the next pair's copies
@@ -512,7 +548,7 @@ __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uin
   }
 }
 
-template <typename Tin, typename Tout, bool kRev>
+template <typename Tin, typename Tout, bool kRev, bool kBox>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_gla_kernel(const __grid_constant__ FusedParams fp) {
   extern __shared__ uint8_t smem_raw[];
@@ -599,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) return false;
       return !qhw || wait_bar(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
     };
-    if (fp.tma) {
+    if constexpr (kBox) {
       // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
       // plain); rows past the sequence end arrive zero-filled.
       if (lane == 0) {
@@ -632,6 +668,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+    } else if (fp.tma == 2) {
+      // Chunks that are not one box (right-to-left rows or columns not a multiple of 64
+      // long): lane t resolves the rows of scan positions c*64 + t and c*64 + 32 + t (the
+      // direction remap) in the 2-D row views [B*L*heads][64] into a shared table; then
+      // each lane issues two 4-row TMA gathers (lanes 8i .. 8i+7: tensor i of Q, K, V, G),
+      // which land in the same tile layouts as the boxes.  Rows past the sequence end point
+      // past the view and arrive zero-filled.
+      const int oob = (int)((long long)p.B * L * p.heads);  // first row past the views
+      const int rbase = (int)((long long)b * L * p.heads + h);
+      const int t = lane >> 3, g0 = 2 * (lane & 7);
+      const void* tmap = t == 0 ? (const void*)&fp.tq : t == 1 ? (const void*)&fp.tk
+                                                               : t == 2 ? (const void*)&fp.tv : (const void*)&fp.tg;
+      for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
+        const int st = n % kStages;
+        int* rows = ms->rowoff[n & 1];
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int pt = lane + 32 * hlf;
+          const long long s = (long long)c * kChunk + pt;
+          rows[kRev ? 63 - pt : pt] = s < L ? rbase + (int)scan_token(fp, (uint32_t)s) * p.heads : oob;
+        }
+        int ok = 0;
+        if (lane == 0) {
+          ok = stage_free(n, st) ? 1 : 0;
+          if (ok) mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);  // the arrival comes first
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        __syncwarp();  // (the row table is complete)
+        uint8_t* sb = smem + kOffStage + st * kStageBytes;
+        uint8_t* tile = t < 3 ? sb + t * kTile : sb + 3 * kTile;
+        const int rowb = t < 3 ? 128 : 256;
+#pragma unroll
+        for (int gi = g0; gi < g0 + 2; ++gi)
+          tma_gather4(tile + gi * 4 * rowb, tmap, &ms->full[st], 0, rows[4 * gi], rows[4 * gi + 1], rows[4 * gi + 2],
+                      rows[4 * gi + 3]);
+      }
     } else {
       // Per chunk, lane t first resolves the grid cells of scan positions c*64 + t and
       // c*64 + 32 + t (the direction remap) into a shared table; then the warp copies the
@@ -652,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hlf = 0; hlf < 2; ++hlf) {
           const int pt = lane + 32 * hlf;
           const long long s = (long long)c * kChunk + pt;
-          rows[kRev ? 63 - pt : pt] = s < L ? (int)((long long)b * L + scan_to_token(s, p.direction, p.H, p.W)) : -1;
+          rows[kRev ? 63 - pt : pt] = s < L ? (int)((long long)b * L + scan_token(fp, (uint32_t)s)) : -1;
         }
         __syncwarp();
         int ok = 0;
@@ -1169,7 +1241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               : nullptr;
           epilogue_rows<__half>(src, od, wstage, lane, nonfinite);
         } else {
-          epilogue_rows<Tout>(src, out_row<Tout>(p, b, h, valid, s), wstage, lane, nonfinite);
+          epilogue_rows<Tout>(src, out_row<Tout>(fp, b, h, valid, s), wstage, lane, nonfinite);
         }
         tc_fence_before();
         wg_sync(wg);
@@ -1393,7 +1465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int ci = 2 * pr + tsel;
         const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
-        epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(p, b, h, ci < cnt && s < L, s), wstage,
+        epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(fp, b, h, ci < cnt && s < L, s), wstage,
                             lane, nonfinite);
       }
     }
@@ -1460,6 +1532,22 @@ bool make_chunk_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a [rows][64] view (one token-head a row) whose box is one row: the
+// source of 4-row TMA gathers.
+bool make_row_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, long long rows,
+                  bool swizzle) {
+  auto enc = get_encode();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) || rows >= (1ll << 31)) return false;
+  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(64 * esize)};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 struct Plan {
   int mode, n_seq, n_s, grid;
 };
@@ -1509,10 +1597,10 @@ size_t seg_capacity(const Problem& p) {
 }
 
 // Clusters of `cs` CTAs of this kernel the device can hold at once (cached per device,
-// direction kind and size).
+// kernel kind and size).
 template <typename K>
-int max_active_clusters(K kern, int dev, bool rev, int cs) {
-  static int cache[64][2][kMaxCluster + 1];
+int max_active_clusters(K kern, int dev, int kind, int cs) {
+  static int cache[64][4][kMaxCluster + 1];
   static std::once_flag once;
   static std::mutex mu;
   std::call_once(once, [] {
@@ -1521,7 +1609,7 @@ int max_active_clusters(K kern, int dev, bool rev, int cs) {
         for (int& c : b) c = -1;
   });
   std::lock_guard<std::mutex> lock(mu);
-  int& c = cache[dev][rev ? 1 : 0][cs];
+  int& c = cache[dev][kind][cs];
   if (c < 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs);
@@ -1544,59 +1632,8 @@ int max_active_clusters(K kern, int dev, bool rev, int cs) {
 template <typename Tin, typename Tout>
 gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
   const bool rev = p.direction == GTR_R2L || p.direction == GTR_B2T;
-  auto kern = rev ? fused_gla_kernel<Tin, Tout, true> : fused_gla_kernel<Tin, Tout, false>;
-  static std::atomic<unsigned long long> configured[2];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
-  if (!(configured[rev].load() & (1ull << dev))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-      return GTR_ERR_CUDA;
-    configured[rev].fetch_or(1ull << dev);
-  }
-  Plan pl = make_plan(p, device_sms());
-  if (pl.mode == 1 && force_mode < 0) {
-    // short sequences: one cluster per sequence (the largest size the device holds for
-    // every sequence at once), at most kClusterChunks chunks per CTA; then the fewest
-    // CTAs that keep the longest run
-    const int Nc = p.n_chunks();
-    int best_k = kClusterChunks + 1;
-    for (int cs = kMaxCluster; cs >= 2; --cs) {
-      if (max_active_clusters(kern, dev, rev, cs) < pl.n_seq) continue;
-      const int k = (Nc + cs - 1) / cs;
-      if (k < best_k) best_k = k;
-    }
-    if (best_k <= kClusterChunks) {
-      const int cs = (Nc + best_k - 1) / best_k;
-      if (cs >= 2 && max_active_clusters(kern, dev, rev, cs) >= pl.n_seq) {
-        pl.mode = 2;
-        pl.n_s = cs;
-        pl.grid = pl.n_seq * cs;
-      }
-    }
-  }
-  if (force_mode == 0) {
-    pl.mode = 0;
-    pl.n_s = 1;
-    pl.grid = pl.n_seq;
-  }
   FusedParams fp;
   fp.p = p;
-  const FusedWorkspace w = fused_workspace_carve(ws, p);
-  fp.hdr = w.hdr;
-  fp.counters = w.counters;
-  fp.agg = w.agg;
-  fp.sstart = w.sstart;
-  fp.qhp = w.qhp;
-  fp.olc = w.olc;
-  fp.n_seq = pl.n_seq;
-  fp.n_s = pl.n_s;
-  fp.Nc = p.n_chunks();
-  fp.mode = pl.mode;
-  fp.grid = pl.grid;
-  // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the
-  // fp16 rounding of the small Qh values keep their precision
-  fp.max_exp2 = 11.5f;
   // chunks are staged in reverse scan order for the reversed directions; a chunk is one
   // TMA box per tensor when its 64 scan positions are consecutive cells of one row view
   // (left-to-right always; right-to-left when rows hold whole chunks) or of one column
@@ -1613,7 +1650,73 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
                    make_chunk_map(&fp.tg, p.log_gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, column, false)
                ? 1
                : 0;
+  fp.divW = make_fastdiv((uint32_t)p.W);
+  fp.divH = make_fastdiv((uint32_t)p.H);
+  if (!fp.tma) {  // other chunks: 4-row gathers from [B*L*heads][64] row views
+    const long long rows = (long long)p.B * p.L() * p.heads;
+    fp.tma = make_row_map(&fp.tq, p.q, dt16, 2, rows, true) && make_row_map(&fp.tk, p.k, dt16, 2, rows, true) &&
+                     make_row_map(&fp.tv, p.v, dt16, 2, rows, true) &&
+                     make_row_map(&fp.tg, p.log_gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, false)
+                 ? 2
+                 : 0;
+  }
 
+  // one kernel per direction kind and producer: the one-box producer's kernel carries
+  // none of the row-table code
+  const bool box = fp.tma == 1;
+  const int kind = (rev ? 2 : 0) + (box ? 1 : 0);
+  auto kern = rev ? (box ? fused_gla_kernel<Tin, Tout, true, true> : fused_gla_kernel<Tin, Tout, true, false>)
+                  : (box ? fused_gla_kernel<Tin, Tout, false, true> : fused_gla_kernel<Tin, Tout, false, false>);
+  static std::atomic<unsigned long long> configured[4];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
+  if (!(configured[kind].load() & (1ull << dev))) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return GTR_ERR_CUDA;
+    configured[kind].fetch_or(1ull << dev);
+  }
+  Plan pl = make_plan(p, device_sms());
+  if (pl.mode == 1 && force_mode < 0) {
+    // short sequences: one cluster per sequence (the largest size the device holds for
+    // every sequence at once), at most kClusterChunks chunks per CTA; then the fewest
+    // CTAs that keep the longest run
+    const int Nc = p.n_chunks();
+    int best_k = kClusterChunks + 1;
+    for (int cs = kMaxCluster; cs >= 2; --cs) {
+      if (max_active_clusters(kern, dev, kind, cs) < pl.n_seq) continue;
+      const int k = (Nc + cs - 1) / cs;
+      if (k < best_k) best_k = k;
+    }
+    if (best_k <= kClusterChunks) {
+      const int cs = (Nc + best_k - 1) / best_k;
+      if (cs >= 2 && max_active_clusters(kern, dev, kind, cs) >= pl.n_seq) {
+        pl.mode = 2;
+        pl.n_s = cs;
+        pl.grid = pl.n_seq * cs;
+      }
+    }
+  }
+  if (force_mode == 0) {
+    pl.mode = 0;
+    pl.n_s = 1;
+    pl.grid = pl.n_seq;
+  }
+  const FusedWorkspace w = fused_workspace_carve(ws, p);
+  fp.hdr = w.hdr;
+  fp.counters = w.counters;
+  fp.agg = w.agg;
+  fp.sstart = w.sstart;
+  fp.qhp = w.qhp;
+  fp.olc = w.olc;
+  fp.n_seq = pl.n_seq;
+  fp.n_s = pl.n_s;
+  fp.Nc = p.n_chunks();
+  fp.mode = pl.mode;
+  fp.grid = pl.grid;
+  // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the
+  // fp16 rounding of the small Qh values keep their precision
+  fp.max_exp2 = 11.5f;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.grid);
   cfg.blockDim = dim3(kThreads);
