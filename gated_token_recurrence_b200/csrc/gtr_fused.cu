@@ -512,8 +512,9 @@ __device__ __forceinline__ void p2_load(const FusedParams& fp, Misc* ms, uint8_t
 }
 
 template <typename Tout>
-__device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem, uint32_t tmem, int q,
-                             int wtid, int lane, int seq, int b, int h, Span sp, int& slot, float& nf) {
+__device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
+                                                  uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
+                                                  Span sp, int& slot, float& nf) {
   const int wq = (wtid >> 5) & 3;
   if (!wg_wait(q, wtid, &ms->p2_go, 0u, ms, hdr, 0x700u + q, slot)) return;
   const long long L = fp.p.L();
@@ -548,7 +549,34 @@ __device__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uin
   }
 }
 
-template <typename Tin, typename Tout, bool kRev, bool kBox>
+// How the second phase joins the kernel, per output type, by the measured time of segmented
+// launches: fp16 outputs inline, bf16 outputs as the compiler decides, fp32 outputs (twice
+// the staging traffic and registers) as a call, which keeps the kernel's own register
+// allocation from spilling.
+template <typename Tout>
+__device__ __noinline__ void second_phase_call(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
+                                               uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
+                                               Span sp, int& slot, float& nf) {
+  second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+}
+template <typename Tout>
+__device__ void second_phase_auto(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem, uint32_t tmem,
+                                  int q, int wtid, int lane, int seq, int b, int h, Span sp, int& slot, float& nf) {
+  second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+}
+template <typename Tout>
+__device__ __forceinline__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
+                                             uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h, Span sp,
+                                             int& slot, float& nf) {
+  if constexpr (sizeof(Tout) == 4)
+    second_phase_call<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+  else if constexpr (std::is_same<Tout, __half>::value)
+    second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+  else
+    second_phase_auto<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+}
+
+template <typename Tin, typename Tout, bool kRev, bool kBox, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_gla_kernel(const __grid_constant__ FusedParams fp) {
   extern __shared__ uint8_t smem_raw[];
@@ -559,8 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Problem& p = fp.p;
   WsHeader* hdr = fp.hdr;
 
-  const bool segm = fp.mode == 1;          // the CTAs of a sequence exchange segment summaries
-  const bool clus = fp.mode == 2;          // ... through distributed shared memory, outputs held on chip
+  // kMode: the plan's mode (0 STREAM, 1 SEGMENTED, 2 CLUSTER) fixed at compile time, or -1:
+  // read at run time (segmented launches take this kernel: ptxas spills fewer bytes in it
+  // than in the one specialised for mode 1)
+  const bool segm = kMode < 0 ? fp.mode == 1 : kMode == 1;  // the CTAs of a sequence exchange segment summaries
+  const bool clus = kMode < 0 ? fp.mode == 2 : kMode == 2;  // ... through distributed shared memory
   const int seq = (segm || clus) ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
   const int seg = (segm || clus) ? (int)blockIdx.x % fp.n_s : 0;
   const bool partial = segm && seg > 0;    // outputs completed in the second phase
@@ -1629,6 +1660,12 @@ int max_active_clusters(K kern, int dev, int kind, int cs) {
   return c;
 }
 
+template <typename Tin, typename Tout, int kMode>
+void (*pick_kernel(bool rev, bool box))(FusedParams) {
+  return rev ? (box ? fused_gla_kernel<Tin, Tout, true, true, kMode> : fused_gla_kernel<Tin, Tout, true, false, kMode>)
+             : (box ? fused_gla_kernel<Tin, Tout, false, true, kMode> : fused_gla_kernel<Tin, Tout, false, false, kMode>);
+}
+
 template <typename Tin, typename Tout>
 gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
   const bool rev = p.direction == GTR_R2L || p.direction == GTR_B2T;
@@ -1661,19 +1698,21 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
                  : 0;
   }
 
-  // one kernel per direction kind and producer: the one-box producer's kernel carries
-  // none of the row-table code
+  // one kernel per direction kind, producer and mode: each carries only the code its
+  // plan runs (the one-box producer's kernels none of the row-table code)
   const bool box = fp.tma == 1;
   const int kind = (rev ? 2 : 0) + (box ? 1 : 0);
-  auto kern = rev ? (box ? fused_gla_kernel<Tin, Tout, true, true> : fused_gla_kernel<Tin, Tout, true, false>)
-                  : (box ? fused_gla_kernel<Tin, Tout, false, true> : fused_gla_kernel<Tin, Tout, false, false>);
+  using Kern = void (*)(FusedParams);
+  const Kern kerns[3] = {pick_kernel<Tin, Tout, 0>(rev, box), pick_kernel<Tin, Tout, -1>(rev, box),
+                         pick_kernel<Tin, Tout, 2>(rev, box)};
   static std::atomic<unsigned long long> configured[4];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
   if (!(configured[kind].load() & (1ull << dev))) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-      return GTR_ERR_CUDA;
+    for (Kern k : kerns)
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return GTR_ERR_CUDA;
     configured[kind].fetch_or(1ull << dev);
   }
   Plan pl = make_plan(p, device_sms());
@@ -1684,13 +1723,13 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
     const int Nc = p.n_chunks();
     int best_k = kClusterChunks + 1;
     for (int cs = kMaxCluster; cs >= 2; --cs) {
-      if (max_active_clusters(kern, dev, kind, cs) < pl.n_seq) continue;
+      if (max_active_clusters(kerns[2], dev, kind, cs) < pl.n_seq) continue;
       const int k = (Nc + cs - 1) / cs;
       if (k < best_k) best_k = k;
     }
     if (best_k <= kClusterChunks) {
       const int cs = (Nc + best_k - 1) / best_k;
-      if (cs >= 2 && max_active_clusters(kern, dev, kind, cs) >= pl.n_seq) {
+      if (cs >= 2 && max_active_clusters(kerns[2], dev, kind, cs) >= pl.n_seq) {
         pl.mode = 2;
         pl.n_s = cs;
         pl.grid = pl.n_seq * cs;
@@ -1742,7 +1781,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, kern, fp) != cudaSuccess) return GTR_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kerns[pl.mode], fp) != cudaSuccess) return GTR_ERR_CUDA;
   return GTR_OK;
 }
 
