@@ -40,8 +40,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FLOPS_PER_TOKEN_HEAD = 24704  # chunkwise, causal: 4*dk*dv + (C+1)(dk+dv)
 
 
-KERNEL_SOURCES = ("gtr_fused.cu", "gtr_sm100.cuh", "gtr_common.cuh")
-TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "fused_gla_kernel_dram_traffic.md")
+KERNEL_SOURCES = ("gtr_fused_kernel.cuh", "gtr_sm100.cuh", "gtr_common.cuh")
+TRAFFIC_DATA = os.path.join(ROOT, "profiles", "fused_gla_kernel_dram_traffic.json")
 
 
 def kernel_fingerprint() -> str:
@@ -55,23 +55,20 @@ def kernel_fingerprint() -> str:
 
 
 def measured_traffic(workload: str):
-    """DRAM bytes per launch (read + write) that an ncu capture recorded for this workload
-    in profiles/fused_gla_kernel_dram_traffic.md -- only when the capture was taken on the
-    current kernel sources (same fingerprint); None otherwise."""
+    """(read, write) DRAM bytes per launch that an ncu capture recorded for this workload
+    (profiles/fused_gla_kernel_dram_traffic.json) -- only when the capture was taken on the
+    current kernel sources (same fingerprint); (None, None) otherwise.  The write figure
+    undercounts the outputs: they reach DRAM by write-back after the kernel ends."""
     try:
-        with open(TRAFFIC_TABLE) as f:
-            lines = f.read().splitlines()
-    except OSError:
-        return None
+        with open(TRAFFIC_DATA) as f:
+            rows = json.load(f)["launches"]
+    except (OSError, ValueError, KeyError):
+        return None, None
     fp = kernel_fingerprint()
-    for line in lines:
-        cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) >= 4 and cells[0] == workload and cells[1] == fp:
-            try:
-                return int(cells[2]) + int(cells[3])
-            except ValueError:
-                return None
-    return None
+    for row in rows:
+        if row.get("workload") == workload and row.get("source") == fp:
+            return int(row["dram_read_bytes"]), int(row["dram_write_bytes"])
+    return None, None
 
 
 def peaks():
@@ -253,27 +250,38 @@ def time_graph(gtr, w, sets, steps, warmup, path, stream, dist, device, per_call
     return total, per
 
 
+def host_cores() -> int:
+    """Cores this process may run on (the oracle's OpenMP threads)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def cpu_oracle_sample(w, seconds=10.0):
-    """Time the fp64 oracle on whole (batch, head) slices of the workload for ~`seconds`."""
+    """The fp64 oracle as it stands: whole calls of the workload (every batch and head) on
+    all host cores, repeated for about `seconds`, plus one whole call on one core."""
     import oracle
     d = w.directions[0]
     q, k, v, lg = make_inputs(w, w.seed(d))
-    sl = (slice(0, 1), slice(None), slice(0, 1), slice(None))
-    qs, ks, vs, gs = (t[sl].contiguous() for t in (q, k, v, lg))
-    oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)  # build + warm
-    threads = oracle.max_threads()
+    cores = host_cores()
+    oracle.gla_fwd(q, k, v, lg, w.H, w.W, d, threads=cores)  # build + warm
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+        oracle.gla_fwd(q, k, v, lg, w.H, w.W, d, threads=cores)
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds or n >= 1000:
             break
-    tokens = n * w.L  # one head of one image per call
-    return {"value": tokens / el / w.heads, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} oracle calls on one (batch, head) slice of the {w.name} workload "
-                      f"(L={w.L}, d_k=d_v={w.d_k}, fp64), {el:.1f} s; token-heads/s divided by "
-                      f"{w.heads} heads to give image tokens/s"}
+    full_call_s = el / n
+    t1 = time.perf_counter()
+    oracle.gla_fwd(q, k, v, lg, w.H, w.W, d, threads=1)
+    one_core_s = time.perf_counter() - t1
+    return {"value": w.B * w.L / full_call_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "full_call_s": full_call_s, "one_core_s": one_core_s,
+            "sample": f"{n} whole oracle calls of the {w.name} workload (B={w.B}, {w.heads} heads, "
+                      f"L={w.L}, d_k=d_v={w.d_k}, fp64, direction {d}) on {cores} cores in {el:.1f} s, "
+                      f"and one whole call on 1 core ({one_core_s:.2f} s)"}
 
 
 def sweep(gtr, names, path, device, stream, hbm):
@@ -303,25 +311,24 @@ def run_reference(args):
     import oracle
     d = w.directions[0]
     q, k, v, lg = make_inputs(w, w.seed(d))
-    sl = (slice(0, 1), slice(None), slice(0, 1), slice(None))
-    qs, ks, vs, gs = (t[sl].contiguous() for t in (q, k, v, lg))
+    cores = host_cores()
     for _ in range(args.warmup):
-        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+        oracle.gla_fwd(q, k, v, lg, w.H, w.W, d, threads=cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.gla_fwd(qs, ks, vs, gs, w.H, w.W, d)
+        oracle.gla_fwd(q, k, v, lg, w.H, w.W, d, threads=cores)
     el = time.perf_counter() - t0
-    value = args.steps * w.L / el / w.heads
-    sample = (f"each step: the fp64 oracle on one (batch, head) slice of the {w.name} workload "
-              f"(L={w.L}), token-heads/s divided by {w.heads} heads")
+    value = args.steps * w.B * w.L / el
+    sample = (f"each step: one whole fp64 oracle call of the {w.name} workload (B={w.B}, "
+              f"{w.heads} heads, L={w.L}, direction {d}) on {cores} cores")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "grid": [w.H, w.W], "heads": w.heads,
                        "d_k": w.d_k, "d_v": w.d_v, "seq_len": w.L, "in_dtype": w.dtype},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(),
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample, "full_call_s": el / args.steps},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -391,6 +398,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(w, seconds=args.cpu_seconds)
 
+    traffic = measured_traffic(w.name) if path_name == "fused" else (None, None)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -406,7 +414,9 @@ def run_ours(args):
                        "l2": f"inputs and outputs rotate over {len(sets)} buffer sets "
                              f"({len(sets) * w.algorithmic_bytes() / 2**20:.0f} MiB > L2)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": measured_traffic(w.name) if path_name == "fused" else None,
+                         "frac": achieved / hbm,
+                         "traffic": (traffic[0] + traffic[1]) if traffic[0] is not None else None,
+                         "traffic_read": traffic[0], "traffic_write": traffic[1],
                          "peak_kind": peak_kind,
                          "kernel": f"gtr_gla_fwd call ({launches} launch"
                                    f"{'es' if launches != 1 else ''}, {path_name} path)",

@@ -31,7 +31,7 @@ STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "G
 EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
             "gtr_gla_workspace_bytes", "gtr_gla_fwd_ex", "gtr_gla_fwd_host",
             "gtr_gla_read_error", "gtr_gla_plan", "gtr_gla_workspace_init", "gtr_status_string",
-            "gtr_version")
+            "gtr_version", "gtr_gla_fwd_noalloc")
 
 
 class GTRError(RuntimeError):
@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         getattr(lib, name).argtypes = fwd_args + [vp]
     lib.gtr_gla_fwd_ex.argtypes = fwd_args + [i, i, i, vp, sz, vp]
     lib.gtr_gla_fwd_host.argtypes = fwd_args + [i, i, vp]
+    lib.gtr_gla_fwd_noalloc.argtypes = fwd_args + [i, i, vp]
     lib.gtr_gla_workspace_bytes.argtypes = [i] * 8
     lib.gtr_gla_workspace_bytes.restype = sz
     lib.gtr_gla_read_error.argtypes = [vp, vp]
@@ -63,7 +64,7 @@ def _load() -> ctypes.CDLL:
     lib.gtr_version.argtypes = []
     for name in ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
                  "gtr_gla_fwd_ex", "gtr_gla_fwd_host", "gtr_gla_read_error", "gtr_gla_plan",
-                 "gtr_gla_workspace_init", "gtr_version"):
+                 "gtr_gla_workspace_init", "gtr_version", "gtr_gla_fwd_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 

@@ -61,10 +61,12 @@ Problem make_problem(const void* q, const void* k, const void* v, const float* g
 // fp32 inputs (exact FFMA arithmetic) and sequences shorter than one chunk take the
 // split path.  For a single partial chunk the fp16 rounding of the gate-scaled
 // operands is no longer averaged over many tokens (a cancelling dot product can
-// dominate the output), and the split path is just as fast there.
+// dominate the output), so such sequences run on the split path even when a fused
+// path is requested: every path then meets the same accuracy bound.
 int choose_path(const Problem& p, int requested) {
+  if (p.L() < kChunk) return GTR_PATH_SPLIT;
   if (requested != GTR_PATH_AUTO) return requested;
-  if (p.in_dtype == GTR_F32 || p.L() < kChunk) return GTR_PATH_SPLIT;
+  if (p.in_dtype == GTR_F32) return GTR_PATH_SPLIT;
   return GTR_PATH_FUSED;
 }
 
@@ -163,6 +165,14 @@ gtr_status_t fwd_internal_ws(const Problem& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+gtr_status_t validate_call(const void* q, const void* k, const void* v, const float* log_gamma, void* out,
+                           int B, int heads, int grid_H, int grid_W, int d_k, int d_v, int direction,
+                           int in_dtype, int out_dtype) {
+  const gtr_status_t st = check_shape(B, heads, grid_H, grid_W, d_k, d_v, direction, in_dtype, out_dtype);
+  return st != GTR_OK ? st : check_ptrs(q, k, v, log_gamma, out);
+}
+
 }  // namespace gtr
 
 using namespace gtr;
@@ -209,7 +219,7 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_H, int grid_W, int d_k
   if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED_SEQUENTIAL) return 0;
   const Problem p = make_problem(nullptr, nullptr, nullptr, nullptr, nullptr, B, heads, grid_H,
                                  grid_W, d_k, d_v, GTR_L2R, in_dtype, out_dtype);
-  if (path != GTR_PATH_AUTO) return path_workspace_bytes(p, path);
+  if (path != GTR_PATH_AUTO) return path_workspace_bytes(p, choose_path(p, path));
   size_t m = 0;
   for (int pth = GTR_PATH_SPLIT; pth <= GTR_PATH_FUSED_SEQUENTIAL; ++pth) {
     const size_t b = path_workspace_bytes(p, pth);

@@ -28,6 +28,9 @@ static_assert(sizeof(WsHeader) == 256, "workspace header must stay 256 bytes");
 // arrays start after this prefix, so calls of different paths can share a workspace.
 constexpr size_t kWsCounterBytes = 2048;
 constexpr size_t kWsPrefixBytes = sizeof(WsHeader) + kWsCounterBytes;
+// Split path scratch per (batch, head, chunk) unit: the chunk summary U and the chunk-start
+// state S (64 x 64 fp32 each) and the chunk log-decays (64 fp32).
+constexpr size_t kSplitUnitBytes = (2 * kD * kD + kD) * sizeof(float);
 
 struct Problem {
   const void* q;

@@ -105,6 +105,8 @@ static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) re
 constexpr size_t kMaxSegCtas = 256;  // CTAs of one launch in SEGMENTED mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
 constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
+// per-segment summary: U_seg [64][64] fp32, the log2 decay [64], the start-state factor, padding
+constexpr size_t kAggStride = 4096 + 128;
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 // floor(n / d) for 0 <= n < 2^31 by one wide multiply and a shift: with l = ceil(log2 d)
@@ -174,7 +176,18 @@ struct Misc {
   uint64_t o_full[kOPairs], o_free[kOPairs];         // per output pair
   uint64_t agg_pub, p2_go, mma_final[2], corr_done[kOPairs];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
+  uint64_t scale_ready;            // the input scale factors below are set (WG_A, first chunk)
   uint32_t tmem_base;
+  // Power-of-two input scale of this CTA, taken from its first chunk (1 unless that chunk's
+  // largest |q|, |k| or |v| is tiny): q, k, v enter the fp16 operands multiplied by
+  // sc_in[0..2] = 2^alpha, 2^beta, 2^gamma, so everything the CTA accumulates carries the
+  // factor 2^(alpha+beta+gamma) (outputs) or 2^(beta+gamma) (the state).
+  float sc_in[3];
+  float sc_out;   // 2^-(alpha+beta+gamma): outputs back to the inputs' scale
+  float sc_spub;  // 2^-(beta+gamma): this CTA's state back to the inputs' scale (published summaries)
+  float sc_sin;   // 2^(beta+gamma): a state in the inputs' scale into this CTA's scale (start states)
+  unsigned int smax[4][3];  // WG_A0: per-warp largest |q|, |k|, |v| bit patterns of the first chunk
+  float segfac[kMaxSegCtas];  // SEGMENTED scan: each segment's start-state factor (its CTA's 2^(beta+gamma))
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
@@ -332,9 +345,10 @@ __device__ __forceinline__ int stage_chunk(int R, int j) {
 // whole rows per 8 (fp32) or 4 (16-bit) lanes, so every 16-byte global store covers
 // 4 or 8 full row segments.  `rowdst` is this lane's destination row (nullptr: not
 // stored).  `nf` collects x * 0 over the values: it turns NaN once any is not finite.
+// Every value is multiplied by `osc` (a power of two: the CTA's input scale undone).
 template <typename Tout>
 __device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, uint8_t* wstage, int lane,
-                                              float& nf) {
+                                              float& nf, float osc) {
   constexpr int kRowB = 32 * (int)sizeof(Tout);  // staged bytes per row and half
   constexpr int kLanesPerRow = kRowB / 16;       // 8 (fp32) or 4 (16-bit)
   constexpr int kRowsPerOp = 32 / kLanesPerRow;
@@ -344,6 +358,8 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, u
     float v[32];
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= osc;
     uint8_t* buf = wstage;  // one 32-row tile, reused by both halves
     if constexpr (sizeof(Tout) == 4) {
 #pragma unroll
@@ -404,10 +420,11 @@ __device__ __forceinline__ uint8_t* out_row(const FusedParams& fp, int b, int h,
 
 // Segmented mode, second phase: the 32 rows of one warp hold the correction Qh' S_start
 // (fp32, tensor memory); the row's partial output O_local (fp16, row-major 128 B rows at
-// `olc_rows` in shared memory) is added on the way out and the sum stored as Tout.
+// `olc_rows` in shared memory) is added on the way out and the sum, times `osc`, stored
+// as Tout.
 template <typename Tout>
 __device__ __forceinline__ void epilogue_rows_add(uint32_t taddr, uint8_t* rowdst, const uint8_t* olc_rows,
-                                                  uint8_t* wstage, int lane, float& nf) {
+                                                  uint8_t* wstage, int lane, float& nf, float osc) {
   constexpr int kRowB = 128;  // fp32 staging, 32 columns per half
   const unsigned long long myrow = reinterpret_cast<unsigned long long>(rowdst);
 #pragma unroll
@@ -428,7 +445,8 @@ __device__ __forceinline__ void epilogue_rows_add(uint32_t taddr, uint8_t* rowds
       const float4 c = *reinterpret_cast<const float4*>(wstage + stage_chunk<kRowB>(R, jj));
       const uint2 ol = *reinterpret_cast<const uint2*>(olc_rows + R * 128 + (32 * half + 4 * jj) * 2);
       const float2 o01 = __half22float2(bits_h2(ol.x)), o23 = __half22float2(bits_h2(ol.y));
-      const float y0 = c.x + o01.x, y1 = c.y + o01.y, y2 = c.z + o23.x, y3 = c.w + o23.y;
+      const float y0 = (c.x + o01.x) * osc, y1 = (c.y + o01.y) * osc, y2 = (c.z + o23.x) * osc,
+                  y3 = (c.w + o23.y) * osc;
       if (dr) {  // (rows past the sequence end hold stale partials: neither checked nor stored)
         nf = fmaf(y0, 0.f, nf);
         nf = fmaf(y1, 0.f, nf);
@@ -475,13 +493,47 @@ __device__ __forceinline__ uint32_t ph_rel(int n) { return ((uint32_t)(n / depth
 // by bulk copy into staging buffer q; one M = 128 MMA puts chunk 2m's rows in lanes
 // 0-63 and chunk 2m+1's in lanes 64-127 of tensor-memory slot q; warp wq of the group
 // takes lanes 32wq .. 32wq+31 (chunk 2m + wq/2, rows 32(wq%2) ..).
+// Largest |x| over a 64 x 64 tile of 16-bit values, as a bit pattern with the sign dropped
+// (for non-negative fp16 and bf16 values the integer order of the patterns is their
+// numeric order), reduced over the calling warp; the warpgroup's 128 threads cover the tile.
+__device__ __forceinline__ unsigned int tile_absmax_bits(const uint8_t* tile, int wtid) {
+  unsigned int m = 0;
+  for (int i = wtid; i < kTile / 16; i += kWG) {
+    const uint4 x = *reinterpret_cast<const uint4*>(tile + 16 * i);
+    m = __vmaxu2(m, x.x & 0x7fff7fffu);
+    m = __vmaxu2(m, x.y & 0x7fff7fffu);
+    m = __vmaxu2(m, x.z & 0x7fff7fffu);
+    m = __vmaxu2(m, x.w & 0x7fff7fffu);
+  }
+  m = max(m & 0xffffu, m >> 16);
+  return __reduce_max_sync(0xffffffffu, m);
+}
+template <typename T> __device__ __forceinline__ float bits16_to_float(unsigned int b);
+template <> __device__ __forceinline__ float bits16_to_float<__half>(unsigned int b) {
+  return __half2float(__ushort_as_half((unsigned short)b));
+}
+template <> __device__ __forceinline__ float bits16_to_float<__nv_bfloat16>(unsigned int b) {
+  return __uint_as_float(b << 16);
+}
+// Exponent e >= 0 of the power of two that brings a tile maximum m into [1, 2), applied
+// only when 0 < m < 2^-6 (inputs that small would lose their precision, or vanish, in the
+// fp16 operands); at most 40, so that the undoing factors stay normal fp32 numbers.
+__device__ __forceinline__ int input_scale_exp(float m) {
+  if (!(m > 0.f) || m >= 0.015625f) return 0;
+  int ex;
+  (void)frexpf(m, &ex);  // m = f * 2^ex, f in [0.5, 1)
+  return min(1 - ex, 40);
+}
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // |e| <= 126
+
 // Scores of a chunk whose gates decay too fast for the factorisation, on the CUDA cores:
 // d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i), from the raw q / k
 // tiles and the full A in the gate tile, into the 16 rows of warp w4 of the chunk's score
 // region (16x256b shape: register 4c+q is row r0 + 8(q>>1), column 8c + cq + (q&1)).
 // Out of line: the chunk loops stay small for the instruction cache.
 template <typename Tin, bool kRev>
-__device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G, uint32_t taddr, int w4, int lane) {
+__device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G, uint32_t taddr, int w4, int lane,
+                                              float ssc) {
   const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
   for (int ps = 0; ps < 2; ++ps) {
     float sv[16];
@@ -497,7 +549,7 @@ __device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G,
           acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
         }
       }
-      sv[x] = acc * 0.125f;
+      sv[x] = acc * ssc;  // d_k^-1/2 times the CTA's q and k scale factors
     }
     tmem_st16x256_x4(taddr + 32u * ps, sv);
   }
@@ -544,7 +596,7 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
     const uint8_t* olc_rows = sbuf + kP2Olc + (wq >> 1) * kTile + 32 * (wq & 1) * 128;
     // fp32 staging over the pair's Qh' (its MMA has completed)
     epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp, b, h, ci < cnt && s < L, s),
-                            olc_rows, sbuf + wq * 4096, lane, nf);
+                            olc_rows, sbuf + wq * 4096, lane, nf, ms->sc_out);
     tc_fence_before();
     fence_proxy_async_smem();  // generic accesses of the buffer before the next pair's copies
     wg_sync(q);
@@ -642,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (i == 10) mbar_init(&ms->mma_final[0], 1);
     if (i == 11) mbar_init(&ms->mma_final[1], 1);
     if (i == 12) ms->abort = 0;
+    if (i == 13) mbar_init(&ms->scale_ready, 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -914,6 +967,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool rev = kRev;
     int slot = 0;
     bool alive = true;
+    float sq = 1.f, sk = 1.f, sv = 1.f;  // this CTA's input scale factors (set at the first chunk)
     for (int n = hh; n < cnt; n += 2) {
       const int st = n % kStages;
       if (!wg_wait(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
@@ -922,6 +976,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint8_t* sb = smem + kOffStage + st * kStageBytes;
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
+      if (n == 0) {
+        // ---- the CTA's input scale, from its first chunk (warpgroup 0, before the tiles
+        // are overwritten): powers of two, so that scaling and undoing it are exact
+        const unsigned int m0 = tile_absmax_bits(sb, wtid), m1 = tile_absmax_bits(sb + kTile, wtid),
+                           m2 = tile_absmax_bits(sb + 2 * kTile, wtid);
+        if (lane == 0) {
+          ms->smax[w4][0] = m0;
+          ms->smax[w4][1] = m1;
+          ms->smax[w4][2] = m2;
+        }
+        wg_sync(wg);
+        if (wtid == 0) {
+          int e[3];
+#pragma unroll
+          for (int t = 0; t < 3; ++t) {
+            const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
+            e[t] = input_scale_exp(bits16_to_float<Tin>(m));
+            ms->sc_in[t] = pow2f(e[t]);
+          }
+          ms->sc_out = pow2f(-(e[0] + e[1] + e[2]));
+          ms->sc_spub = pow2f(-(e[1] + e[2]));
+          ms->sc_sin = pow2f(e[1] + e[2]);
+          mbar_arrive(&ms->scale_ready);
+        }
+      }
+      if (n == hh) {  // this warpgroup's first chunk: take the scale
+        if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot)) {
+          alive = false;
+          break;
+        }
+        sq = ms->sc_in[0];
+        sk = ms->sc_in[1];
+        sv = ms->sc_in[2];
+      }
       // ---- in-chunk cumulative log2-gates in scan order: my 4 rows (written back over
       // the gates, still without the offset of the rows before them), a scan over the
       // warp's 4 row blocks, then over the 4 warps through shared memory (staged rows run
@@ -1013,7 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
         tc_fence_after();  // (the wait's barrier also publishes the full A)
         cuda_core_scores<Tin, rev>(sb, G, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU), w4,
-                                   lane);
+                                   lane, 0.125f * sq * sk);
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);  // raw q / k reads done before the overwrite
@@ -1022,8 +1110,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) off[ps][e] = 0.f;  // the gate tile holds the full A now
       }
-      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
+      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place, times
+      // the CTA's input scale factors
       const __half2 eighth = __float2half2_rn(0.125f);
+      const bool scl = sq != 1.f || sk != 1.f;
+      const float kf = 0.125f * sk;
 #pragma unroll 1
       for (int ps = 0; ps < 2; ++ps) {  // (rolled: the loop body stays small for the instruction cache)
         const int ch0 = 32 * ps + 4 * cc;
@@ -1051,13 +1142,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float xk0 = fbx ? lastp[2 * e2] - A0 : -A0;
             const float xk1 = fbx ? lastp[2 * e2 + 1] - A1 : -A1;
             __half2 qh, kh;
-            if constexpr (std::is_same<Tin, __half>::value) {
+            if (std::is_same<Tin, __half>::value && !scl) {
               qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
               kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
             } else {
               const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
-              qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
-              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+              qh = __floats2half2_rn(qv.x * sq * ex2(A0), qv.y * sq * ex2(A1));
+              kh = __floats2half2_rn(kv.x * kf * ex2(xk0), kv.y * kf * ex2(xk1));
             }
             qw[e2] = h2_bits(qh);
             kw[e2] = h2_bits(kh);
@@ -1066,8 +1157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
         }
       }
-      if constexpr (!std::is_same<Tin, __half>::value) {
-        // bf16 inputs: the V tile becomes fp16 in place (exact inside the fp16 range)
+      if (!std::is_same<Tin, __half>::value || sv != 1.f) {
+        // bf16 inputs (or a scaled fp16 V): the V tile becomes fp16 in place, times the
+        // CTA's v factor (exact inside the fp16 range)
         uint4* vt = reinterpret_cast<uint4*>(sb + 2 * kTile);
 #pragma unroll
         for (int i = wtid; i < kTile / 16; i += kWG) {
@@ -1076,7 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = In2<Tin>::unpack(w[e]);
-            w[e] = pack_h2(f.x, f.y);
+            w[e] = pack_h2(f.x * sv, f.y * sv);
           }
           vt[i] = x;
         }
@@ -1119,7 +1211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->sready[0]);
     }
-    for (int n = 0; n < cnt; ++n) {
+    // the input scale (published summaries go back to the inputs' scale)
+    if (!wait_bar(&ms->scale_ready, 0u, ms, hdr, 0x405)) alive = false;
+    for (int n = 0; n < cnt && alive; ++n) {
       const int st = n % kStages, su = n % kSU;
       if (!wait_bar(&ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400)) { alive = false; break; }
       tc_fence_after();
@@ -1206,10 +1300,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // barrier: U_seg (fp32, row-major) over the output staging area (idle: the outputs
       // are held), the log2 decay per key channel in the misc area
       float* U = reinterpret_cast<float*>(smem + kOffStg);
+      const float f = ms->sc_spub;  // in the inputs' scale
 #pragma unroll
       for (int cb = 0; cb < 8; ++cb) {
-        *reinterpret_cast<float2*>(U + r0 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb], Ls[4 * cb + 1]);
-        *reinterpret_cast<float2*>(U + r1 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]);
+        *reinterpret_cast<float2*>(U + r0 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb] * f, Ls[4 * cb + 1] * f);
+        *reinterpret_cast<float2*>(U + r1 * 64 + 8 * cb + cq) = make_float2(Ls[4 * cb + 2] * f, Ls[4 * cb + 3] * f);
       }
       if ((lane & 3) == 0) {
         ms->dseg[r0] = a2r0;
@@ -1219,17 +1314,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
     }
     if (segm && alive) {
-      // segment summary: U_seg = local end state, its log2 decay
-      float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * (4096 + 64);
+      // segment summary: U_seg = local end state (in the inputs' scale), its log2 decay, and
+      // the factor that takes a start state into this CTA's scale
+      float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * kAggStride;
+      const float f = ms->sc_spub;
 #pragma unroll
       for (int cb = 0; cb < 8; ++cb) {
-        __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb], Ls[4 * cb + 1]));
-        __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb + 2], Ls[4 * cb + 3]));
+        __stcg(reinterpret_cast<float2*>(mine + r0 * 64 + 8 * cb + cq), make_float2(Ls[4 * cb] * f, Ls[4 * cb + 1] * f));
+        __stcg(reinterpret_cast<float2*>(mine + r1 * 64 + 8 * cb + cq),
+               make_float2(Ls[4 * cb + 2] * f, Ls[4 * cb + 3] * f));
       }
       if ((lane & 3) == 0) {
         mine[4096 + r0] = a2r0;
         mine[4096 + r1] = a2r1;
       }
+      if (wtid == 0) mine[4096 + 64] = ms->sc_sin;
       __threadfence();
       wg_sync(wg);
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
@@ -1243,7 +1342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
-    bool alive = true;
+    // the input scale (the outputs are stored in the inputs' scale)
+    bool alive = wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x505, slot);
     if (clus) {
       // the outputs stay in tensor memory until the start state is known: wait for their
       // last MMAs; then (segments s > 0) the chunks' Qh' tiles start loading into the idle
@@ -1261,7 +1361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // this CTA's chunks; in a segment s > 0 the outputs are partial: fp16 rows of the
       // workspace, completed in the second phase
-      const int pairs = (cnt + 1) / 2;
+      const int pairs = alive ? (cnt + 1) / 2 : 0;
+      const float osc = ms->sc_out;
       for (int pr = 0; pr < pairs; ++pr) {
         if (!wg_wait(wg, wtid, &ms->o_full[pr % kOPairs], ph_use<kOPairs>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
@@ -1272,9 +1373,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (partial) {
           uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp.c0 + ci) * 4096) + trow * 128
                               : nullptr;
-          epilogue_rows<__half>(src, od, wstage, lane, nonfinite);
+          epilogue_rows<__half>(src, od, wstage, lane, nonfinite, 1.f);  // (kept in this CTA's scale)
         } else {
-          epilogue_rows<Tout>(src, out_row<Tout>(fp, b, h, valid, s), wstage, lane, nonfinite);
+          epilogue_rows<Tout>(src, out_row<Tout>(fp, b, h, valid, s), wstage, lane, nonfinite, osc);
         }
         tc_fence_before();
         wg_sync(wg);
@@ -1302,7 +1403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bi = wtid / FP, fi = wtid % FP;
       const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
       unsigned int* ctr = fp.counters + (size_t)seq * 2;
-      const float* aggs = fp.agg + (size_t)seq * ns * (4096 + 64);
+      const float* aggs = fp.agg + (size_t)seq * ns * kAggStride;
       uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
       float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
       float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
@@ -1321,6 +1422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok0 = wg_agree(wg, wtid, ok0, ms, slot);
       }
       if (ok0) {
+        for (int sg = wtid; sg < ns; sg += kWG) ms->segfac[sg] = __ldcg(aggs + (size_t)sg * kAggStride + 4096 + 64);
+        wg_sync(wg);
         for (int base = f0; base < f1; base += FP) {
           const int f = base + fi;
           const bool act = bi < nB && f < f1;
@@ -1332,7 +1435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < kScanBlock; ++j) {
             const int sg = s_lo + j;
             const bool on = act && sg < s_hi;
-            const float* a2p = aggs + (size_t)(on ? sg : 0) * (4096 + 64);
+            const float* a2p = aggs + (size_t)(on ? sg : 0) * kAggStride;
             u[j] = on ? __ldcg(reinterpret_cast<const float4*>(a2p) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
             dd[j] = on ? __ldcg(a2p + 4096 + kk) : 0.f;
           }
@@ -1365,7 +1468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < kScanBlock; ++j) {
               const int sg = s_lo + j;
               if (sg < s_hi) {
-                const uint2 w = make_uint2(pack_h2(X.x, X.y), pack_h2(X.z, X.w));
+                const float fs = ms->segfac[sg];  // into segment sg's CTA scale
+                const uint2 w = make_uint2(pack_h2(X.x * fs, X.y * fs), pack_h2(X.z * fs, X.w * fs));
                 __stcg(reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(sst + (size_t)sg * 4096) + soff), w);
                 X = make_float4(fmaf(dd[j], X.x, u[j].x), fmaf(dd[j], X.y, u[j].y), fmaf(dd[j], X.z, u[j].z),
                                 fmaf(dd[j], X.w, u[j].w));
@@ -1413,24 +1517,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kk = u >> 5, v0 = 2 * (u & 31);  // key channel, value pair
         const uint32_t a_u = smem_u32(smem + kOffStg) + (uint32_t)(kk * 64 + v0) * 4u;
         const uint32_t a_d = smem_u32(&ms->dseg[kk]);
+        const uint32_t a_f = smem_u32(&ms->sc_sin);
         const uint32_t a_s = smem_u32(smem + kOffSst) + (uint32_t)kk * 128u +
                              ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (uint32_t)(v0 & 7) * 2u;
         // every segment's summary entries first (the remote loads overlap), then the
         // sequential composition
         float2 uj[kMaxCluster];
-        float dj[kMaxCluster];
+        float dj[kMaxCluster], fj[kMaxCluster];  // fj: a start state into CTA j's scale
 #pragma unroll
         for (int j = 0; j < kMaxCluster; ++j) {
           if (j < ns) {
             uj[j] = ld_cluster_f32x2(cluster_map(a_u, (uint32_t)j));
             dj[j] = ld_cluster_f32(cluster_map(a_d, (uint32_t)j));
+            fj[j] = ld_cluster_f32(cluster_map(a_f, (uint32_t)j));
           }
         }
         float2 X = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < kMaxCluster; ++j) {
           if (j < ns) {
-            st_cluster_u32(cluster_map(a_s, (uint32_t)j), pack_h2(X.x, X.y));
+            st_cluster_u32(cluster_map(a_s, (uint32_t)j), pack_h2(X.x * fj[j], X.y * fj[j]));
             const float d = ex2(dj[j]);
             X = make_float2(fmaf(d, X.x, uj[j].x), fmaf(d, X.y, uj[j].y));
           }
@@ -1499,7 +1605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ci = 2 * pr + tsel;
         const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
         epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(fp, b, h, ci < cnt && s < L, s), wstage,
-                            lane, nonfinite);
+                            lane, nonfinite, ms->sc_out);
       }
     }
   }

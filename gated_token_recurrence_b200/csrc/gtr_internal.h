@@ -27,6 +27,12 @@ struct FusedWorkspace {
   uint16_t* olc;           // segmented mode: per-chunk outputs from a zero segment start (fp16)
 };
 
+// Argument validation of the device entry points (shape, enums, dtype pairing, pointers),
+// done on the host before anything is enqueued.
+gtr_status_t validate_call(const void* q, const void* k, const void* v, const float* log_gamma, void* out,
+                           int B, int heads, int grid_H, int grid_W, int d_k, int d_v, int direction,
+                           int in_dtype, int out_dtype);
+
 size_t split_workspace_bytes(const Problem& p);
 SplitWorkspace split_workspace_carve(void* ws, const Problem& p);
 gtr_status_t launch_split(const Problem& p, void* ws, cudaStream_t stream);

@@ -18,13 +18,17 @@
 #include <mutex>
 
 #include "gtr_common.cuh"
+#include "gtr_internal.h"
 
 namespace gtr {
 namespace {
 
-// 20 MiB: room for B * heads * ceil(L/64) <= 636 chunk units of the split path
-// (256 header bytes + 32,960 bytes per unit), e.g. the 1024^2 image with 8 heads.
+// 20 MiB: the split path needs the shared workspace prefix plus kSplitUnitBytes per
+// (batch, head, chunk) unit, so B * heads * ceil(L/64) <= 634 units fit (for example
+// the 1024^2 image with 8 heads: 512 units).
 constexpr size_t kNoallocScratchBytes = size_t(20) << 20;
+constexpr size_t kNoallocMaxUnits = (kNoallocScratchBytes - kWsPrefixBytes) / kSplitUnitBytes;
+static_assert(kNoallocMaxUnits == 634, "the documented unit limit matches the array size");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
@@ -58,18 +62,16 @@ extern "C" gtr_status_t gtr_gla_fwd_noalloc(const void* q, const void* k, const 
                                             const float* log_gamma, void* out, int B, int heads,
                                             int grid_H, int grid_W, int d_k, int d_v, int direction,
                                             int in_dtype, int out_dtype, gtr_stream_t stream) {
-  // Size check first, on the host: a problem whose scratch does not fit is refused
-  // before anything touches the device.
-  const size_t need = gtr_gla_workspace_bytes(B, heads, grid_H, grid_W, d_k, d_v, in_dtype,
-                                               GTR_PATH_SPLIT);
-  if (need == 0) {
-    // invalid or unsupported shape: let the ordinary validation name the reason
-    return gtr_gla_fwd_ex(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v, direction,
-                          in_dtype, out_dtype, GTR_PATH_SPLIT, nullptr, 0, stream);
-  }
-  if (need > gtr::kNoallocScratchBytes) return GTR_ERR_WORKSPACE;
+  // The same argument checks as every other entry point, then the size limit: all on
+  // the host, before anything touches the device.
+  gtr_status_t st = gtr::validate_call(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v,
+                                       direction, in_dtype, out_dtype);
+  if (st != GTR_OK) return st;
+  const long long L = (long long)grid_H * grid_W;
+  const long long units = (long long)B * heads * ((L + gtr::kChunk - 1) / gtr::kChunk);
+  if (units > (long long)gtr::kNoallocMaxUnits) return GTR_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const gtr_status_t st = gtr::scratch_address(&scratch);
+  st = gtr::scratch_address(&scratch);
   if (st != GTR_OK) return st;
   // Nothing in the scratch has to start at zero: the split path writes every
   // summary, state and log-decay it reads earlier in the same call, and it never

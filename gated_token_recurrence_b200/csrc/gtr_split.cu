@@ -278,7 +278,7 @@ gtr_status_t launch_split_typed(const Problem& p, const SplitWorkspace& ws, cuda
 
 size_t split_workspace_bytes(const Problem& p) {
   const size_t units = (size_t)p.B * p.heads * p.n_chunks();
-  return kWsPrefixBytes + units * (2 * kD * kD + kD) * sizeof(float);
+  return kWsPrefixBytes + units * kSplitUnitBytes;
 }
 
 SplitWorkspace split_workspace_carve(void* ws, const Problem& p) {

@@ -76,7 +76,10 @@ typedef enum {
                                 call's output is not valid - use GTR_PATH_SPLIT for such data */
 } gtr_status_t;
 
-/* Execution paths.  GTR_PATH_AUTO lets the length-aware dispatcher choose. */
+/* Execution paths.  GTR_PATH_AUTO lets the length-aware dispatcher choose.  Sequences
+ * shorter than one chunk (grid_H * grid_W < 64) always run on GTR_PATH_SPLIT, whichever
+ * path is requested (the fused paths' fp16 operand rounding is not averaged over enough
+ * tokens there to stay inside the accuracy bound). */
 typedef enum {
     GTR_PATH_AUTO = 0,
     GTR_PATH_SPLIT = 1, /* three launches: chunk summaries -> state scan -> chunk outputs (any dtype) */
@@ -169,9 +172,10 @@ gtr_status_t gtr_gla_fwd_host(const void *q, const void *k, const void *v,
  * 20 MiB array compiled into the library; every GPU that loads libgtr.so
  * holds that array until the process exits.  Problems whose scratch,
  * gtr_gla_workspace_bytes(..., GTR_PATH_SPLIT), exceeds 20 MiB - more than
- * 636 chunk units B * heads * ceil(L / 64) - are refused on the host with
- * GTR_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
- * (no cudaMalloc, cudaFree or allocating library routine).
+ * 634 chunk units B * heads * ceil(L / 64) - are refused on the host with
+ * GTR_ERR_WORKSPACE before anything is enqueued (after the argument checks of
+ * gtr_gla_fwd, whose codes take precedence).  The call allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine).
  *
  * The first call on each device looks up the array's device address with
  * cudaGetSymbolAddress while that device is current, and caches it; make that

@@ -83,3 +83,36 @@ def test_dispatcher_plan():
     assert gtr.plan(8, 6, 48, 80, in_dtype=gtr.BF16) == ("fused", 1)
     assert gtr.plan(1, 2, 16, 16, in_dtype=gtr.F32) == ("split", 3)
     assert gtr.status_string(6) == "GTR_ERR_RANGE"
+
+
+def test_short_sequences_take_the_split_path_whatever_is_requested():
+    """Shorter than one chunk: a requested fused path runs the split path, so the
+    workspace query for that request is the split path's size."""
+    split = gtr.workspace_bytes(1, 2, 7, 9, 64, 64, gtr.F16, "split")
+    assert gtr.workspace_bytes(1, 2, 7, 9, 64, 64, gtr.F16, "fused") == split
+    assert gtr.workspace_bytes(1, 2, 7, 9, 64, 64, gtr.F16, "fused_sequential") == split
+    assert gtr.plan(1, 2, 7, 9, in_dtype=gtr.F16) == ("split", 3)
+
+
+# ---------------------------------------------------------------- gtr_gla_fwd_noalloc (host side)
+def _noalloc(B, heads, H, W, q=256, out=256, din=gtr.F16, dout=gtr.F16, dk=64):
+    # the pointers are never dereferenced: every case below is decided on the host
+    return gtr.lib.gtr_gla_fwd_noalloc(q, 256, 256, 256, out, B, heads, H, W, dk, 64, 0, din, dout, None)
+
+
+def test_noalloc_unit_limit_matches_its_array():
+    """634 chunk units of split-path scratch fit the fixed 20 MiB array, 635 do not."""
+    array = 20 << 20
+    fits = gtr.workspace_bytes(1, 2, 64, 317, 64, 64, gtr.F16, "split")   # 2 x 317 = 634 units
+    over = gtr.workspace_bytes(1, 1, 64, 635, 64, 64, gtr.F16, "split")   # 635 units
+    assert fits <= array < over
+    assert _noalloc(1, 1, 64, 635) == 5          # GTR_ERR_WORKSPACE, nothing enqueued
+    assert _noalloc(5, 127, 1, 64) == 5          # 635 units spread over (batch, head)
+
+
+def test_noalloc_validates_arguments_before_the_size_limit():
+    """Argument errors keep their own codes on a problem that is also too large."""
+    assert _noalloc(1, 1, 64, 635, q=None) == 1                       # null pointer
+    assert _noalloc(1, 1, 64, 635, out=8) == 1                        # misaligned
+    assert _noalloc(1, 1, 64, 635, din=gtr.BF16, dout=gtr.F16) == 2   # unsupported pairing
+    assert _noalloc(1, 1, 64, 635, dk=48) == 2                        # unsupported d_k

@@ -92,24 +92,8 @@ def test_ragged_and_degenerate_shapes(shape, dtype, path):
     B, heads, H, W = shape
     w = Workload("odd", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=1.0, index=9)
     for d in range(4):
-        if H * W == 1 and path.startswith("fused"):
-            check_single_token(w, d, 9000 + 100 * H + W + d, path)
-        else:
-            check(w, d, 9000 + 100 * H + W + d, path)
-
-
-def check_single_token(w: Workload, direction: int, seed: int, path: str):
-    """One token: o = d_k^{-1/2} (q . k) v.  The tensor-core path rounds the gate-scaled q
-    and k and the score to fp16, so its error is bounded by a few fp16 ulps of the
-    dot product's absolute terms, sum_i |q_i k_i|, times |v|; a cancelling q . k makes
-    1e-2 * rms(o) smaller than that (the automatic dispatch sends such sequences to the
-    fp32 split path)."""
-    q, k, v, lg = make_inputs(w, seed)
-    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, direction)
-    out = run_gpu(w, q, k, v, lg, direction, path).double().cpu().numpy()
-    qa, ka, va = (t.double().numpy() for t in (q, k, v))
-    scale = np.abs(qa * ka).sum(axis=-1, keepdims=True) * np.abs(va) / np.sqrt(w.d_k)
-    assert (np.abs(out - ref) <= 4 * 2.0 ** -11 * scale + 1e-6).all()
+        # (sequences shorter than one chunk run on the split path whatever path is asked for)
+        check(w, d, 9000 + 100 * H + W + d, path)
 
 
 @pytest.mark.parametrize("path", ["auto"] + PATHS)
@@ -138,6 +122,26 @@ def test_no_decay_gates(path):
     assert rel_err(out, ref) <= 1e-2
 
 
+# shapes that take each plan of the fused kernel: one cluster per sequence (2 x 25 chunks),
+# several CTAs per sequence exchanging segment summaries (2 x 224 chunks), one CTA per
+# sequence (78 sequences of 2 chunks)
+PLAN_SHAPES = [(1, 2, 40, 40), (1, 2, 128, 112), (13, 6, 8, 16)]
+
+
+@pytest.mark.parametrize("path", ["auto", "fused", "fused_sequential"])
+@pytest.mark.parametrize("shape", PLAN_SHAPES)
+@pytest.mark.parametrize("dtype,exp2", [("bf16", -16), ("bf16", -24), ("f16", -12)])
+def test_tiny_magnitude_inputs_keep_their_precision(dtype, exp2, shape, path):
+    """q, k, v scaled by 2^-16 or 2^-24 (bf16) or 2^-12 (fp16, many values subnormal): the
+    products fall below the normal range of the fp16 tensor-core operands, so the fused
+    kernel brings each CTA's inputs into range by a power of two (exact) and undoes it on
+    the outputs.  The bound is the same 1e-2 * rms as for ordinary inputs."""
+    B, heads, H, W = shape
+    w = Workload("tinymag", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=2.0 ** exp2, index=9)
+    for d in range(4):
+        check(w, d, 6100 + 10 * d - exp2, path)
+
+
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.float16])
 def test_fp16_inputs_either_output_dtype(out_dtype):
     w = WORKLOADS["640"].with_(heads=2)
@@ -145,7 +149,9 @@ def test_fp16_inputs_either_output_dtype(out_dtype):
 
 
 def test_bf16_inputs_bf16_output_runs():
-    """bf16 output is allowed; its own rounding costs ~2^-9 * max|o|, so the bound is looser."""
+    """bf16 OUTPUT is an opt-in outside the 1e-2 * rms accuracy bound: rounding o to bf16
+    alone costs up to 2^-9 * max|o| (about 1.5% of rms on these workloads, where max|o| is
+    5-6 rms), so this check uses 3e-2.  The default output for bf16 inputs is fp32."""
     w = WORKLOADS["1024"].with_(heads=2, H=32)
     check(w, 0, 556, out_dtype=torch.bfloat16, tol=3e-2)
 
