@@ -104,9 +104,8 @@ static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) re
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
 constexpr size_t kMaxSegCtas = 256;  // CTAs of one launch in SEGMENTED mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
-constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
-// per-segment summary: U_seg [64][64] fp32, the log2 decay [64], the start-state factor, padding
-constexpr size_t kAggStride = 4096 + 128;
+// per-segment summary: U_seg [64][64] fp32 and the log2 decay [64]
+constexpr size_t kAggStride = 4096 + 64;
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 // floor(n / d) for 0 <= n < 2^31 by one wide multiply and a shift: with l = ceil(log2 d)
@@ -133,9 +132,8 @@ struct alignas(64) FusedParams {
   CUtensorMap tq, tk, tv, tg;
   Problem p;
   WsHeader* hdr;
-  unsigned int* counters;  // [n_seq][2], monotonic within a call, zero between calls
+  unsigned int* counters;  // SEGMENTED: [n_seq][n_s] segment flags (summary published), zero between calls
   float* agg;              // [n_seq][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
-  uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
   uint16_t* qhp;           // [n_seq][Nc][64*64] Qh' per chunk, fp16, MMA layout
   uint16_t* olc;           // [n_seq][Nc][64][64] outputs from a zero segment start, fp16
   int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED, 2 = CLUSTER
@@ -174,7 +172,7 @@ struct Misc {
   uint64_t sready[kNS];                              // per chunk-start state tile
   uint64_t qdone[kStages];                           // Qh' of the staged chunk copied out
   uint64_t o_full[kOPairs], o_free[kOPairs];         // per output pair
-  uint64_t agg_pub, p2_go, mma_final[2], corr_done[kOPairs];
+  uint64_t agg_pub, mma_final[2], corr_done[kOPairs];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
   uint64_t scale_ready;            // the input scale factors below are set (WG_A, first chunk)
   uint32_t tmem_base;
@@ -187,7 +185,7 @@ struct Misc {
   float sc_spub;  // 2^-(beta+gamma): this CTA's state back to the inputs' scale (published summaries)
   float sc_sin;   // 2^(beta+gamma): a state in the inputs' scale into this CTA's scale (start states)
   unsigned int smax[4][3];  // WG_A0: per-warp largest |q|, |k|, |v| bit patterns of the first chunk
-  float segfac[kMaxSegCtas];  // SEGMENTED scan: each segment's start-state factor (its CTA's 2^(beta+gamma))
+  int seg_go;               // SEGMENTED: the start state can be composed (the predecessors published)
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
@@ -272,6 +270,15 @@ __device__ __forceinline__ void red_release_add(unsigned int* ctr, unsigned int 
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Named barrier `id` over the first `n` threads of the CTA (a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Named barrier of one 128-thread warpgroup (ids 1..3).
 __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory"); }
 
@@ -325,6 +332,18 @@ template <> struct In2<__half> {
 template <> struct In2<__nv_bfloat16> {
   static __device__ __forceinline__ float2 unpack(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+};
+
+// Two fp32 values -> two 16-bit values of type T (round to nearest even).
+template <typename T> struct Pack2;
+template <> struct Pack2<__half> {
+  static __device__ __forceinline__ uint32_t pack(float a, float b) { return pack_h2(a, b); }
+};
+template <> struct Pack2<__nv_bfloat16> {
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
   }
 };
 
@@ -493,20 +512,53 @@ __device__ __forceinline__ uint32_t ph_rel(int n) { return ((uint32_t)(n / depth
 // by bulk copy into staging buffer q; one M = 128 MMA puts chunk 2m's rows in lanes
 // 0-63 and chunk 2m+1's in lanes 64-127 of tensor-memory slot q; warp wq of the group
 // takes lanes 32wq .. 32wq+31 (chunk 2m + wq/2, rows 32(wq%2) ..).
-// Largest |x| over a 64 x 64 tile of 16-bit values, as a bit pattern with the sign dropped
-// (for non-negative fp16 and bf16 values the integer order of the patterns is their
-// numeric order), reduced over the calling warp; the warpgroup's 128 threads cover the tile.
-__device__ __forceinline__ unsigned int tile_absmax_bits(const uint8_t* tile, int wtid) {
-  unsigned int m = 0;
+// Byte offset of the 8 bytes holding channels ch0 .. ch0+3 (ch0 a multiple of 4) of row
+// `row` in a 128-byte-swizzled 16-bit tile.
+__device__ __forceinline__ uint32_t sw_off8(int row, int ch0) {
+  return row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
+}
+
+// Largest |x| of the q and k elements a WG_A thread builds (rows row0 .. row0+3, channels
+// 4cc .. 4cc+3 and 32+4cc .. 32+4cc+3) and of the v elements it converts, as bit patterns
+// with the sign dropped (for non-negative fp16 and bf16 values the integer order of the
+// patterns is their numeric order), reduced over the warp.  Out of line: first chunk only.
+__device__ __noinline__ uint3 own_absmax_bits(const uint8_t* sb, int row0, int cc, int wtid) {
+  uint32_t mq = 0, mk = 0, mv = 0;
+  for (int ps = 0; ps < 2; ++ps)
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t o = sw_off8(row0 + i, 32 * ps + 4 * cc);
+      const uint2 a = *reinterpret_cast<const uint2*>(sb + o), c = *reinterpret_cast<const uint2*>(sb + kTile + o);
+      mq = __vmaxu2(__vmaxu2(mq, a.x & 0x7fff7fffu), a.y & 0x7fff7fffu);
+      mk = __vmaxu2(__vmaxu2(mk, c.x & 0x7fff7fffu), c.y & 0x7fff7fffu);
+    }
   for (int i = wtid; i < kTile / 16; i += kWG) {
-    const uint4 x = *reinterpret_cast<const uint4*>(tile + 16 * i);
-    m = __vmaxu2(m, x.x & 0x7fff7fffu);
-    m = __vmaxu2(m, x.y & 0x7fff7fffu);
-    m = __vmaxu2(m, x.z & 0x7fff7fffu);
-    m = __vmaxu2(m, x.w & 0x7fff7fffu);
+    const uint4 x = *reinterpret_cast<const uint4*>(sb + 2 * kTile + 16 * i);
+    mv = __vmaxu2(__vmaxu2(mv, x.x & 0x7fff7fffu), x.y & 0x7fff7fffu);
+    mv = __vmaxu2(__vmaxu2(mv, x.z & 0x7fff7fffu), x.w & 0x7fff7fffu);
   }
-  m = max(m & 0xffffu, m >> 16);
-  return __reduce_max_sync(0xffffffffu, m);
+  return make_uint3(__reduce_max_sync(0xffffffffu, max(mq & 0xffffu, mq >> 16)),
+                    __reduce_max_sync(0xffffffffu, max(mk & 0xffffu, mk >> 16)),
+                    __reduce_max_sync(0xffffffffu, max(mv & 0xffffu, mv >> 16)));
+}
+
+// The q and k elements a WG_A thread builds, times the CTA's factors sq and sk, in place
+// (exact: powers of two that bring the values up into the normal range).  Out of line:
+// only CTAs whose inputs are tiny run it.
+template <typename Tin>
+__device__ __noinline__ void prescale_own(uint8_t* sb, int row0, int cc, float sq, float sk) {
+  for (int ps = 0; ps < 2; ++ps)
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t o = sw_off8(row0 + i, 32 * ps + 4 * cc);
+      for (int t = 0; t < 2; ++t) {
+        uint2* p = reinterpret_cast<uint2*>(sb + t * kTile + o);
+        const float f = t ? sk : sq;
+        uint2 x = *p;
+        const float2 a = In2<Tin>::unpack(x.x), c = In2<Tin>::unpack(x.y);
+        x.x = Pack2<Tin>::pack(a.x * f, a.y * f);
+        x.y = Pack2<Tin>::pack(c.x * f, c.y * f);
+        *p = x;
+      }
+    }
 }
 template <typename T> __device__ __forceinline__ float bits16_to_float(unsigned int b);
 template <> __device__ __forceinline__ float bits16_to_float<__half>(unsigned int b) {
@@ -570,7 +622,6 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
                                                   uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
                                                   Span sp, int& slot, float& nf) {
   const int wq = (wtid >> 5) & 3;
-  if (!wg_wait(q, wtid, &ms->p2_go, 0u, ms, hdr, 0x700u + q, slot)) return;
   const long long L = fp.p.L();
   const int cnt = sp.c1 - sp.c0, npairs = (cnt + 1) / 2;
   uint8_t* sbuf = smem + kOffStage + q * kStageBytes;
@@ -690,7 +741,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ms->go[i][0] = ms->go[i][1] = 0;
     }
     if (i == 8) mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
-    if (i == 9) mbar_init(&ms->p2_go, 1);
     if (i == 10) mbar_init(&ms->mma_final[0], 1);
     if (i == 11) mbar_init(&ms->mma_final[1], 1);
     if (i == 12) ms->abort = 0;
@@ -977,31 +1027,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* sb = smem + kOffStage + st * kStageBytes;
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
       if (n == 0) {
-        // ---- the CTA's input scale, from its first chunk (warpgroup 0, before the tiles
-        // are overwritten): powers of two, so that scaling and undoing it are exact
-        const unsigned int m0 = tile_absmax_bits(sb, wtid), m1 = tile_absmax_bits(sb + kTile, wtid),
-                           m2 = tile_absmax_bits(sb + 2 * kTile, wtid);
-        if (lane == 0) {
-          ms->smax[w4][0] = m0;
-          ms->smax[w4][1] = m1;
-          ms->smax[w4][2] = m2;
-        }
-        wg_sync(wg);
-        if (wtid == 0) {
-          int e[3];
-#pragma unroll
-          for (int t = 0; t < 3; ++t) {
-            const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
-            e[t] = input_scale_exp(bits16_to_float<Tin>(m));
-            ms->sc_in[t] = pow2f(e[t]);
-          }
-          ms->sc_out = pow2f(-(e[0] + e[1] + e[2]));
-          ms->sc_spub = pow2f(-(e[1] + e[2]));
-          ms->sc_sin = pow2f(e[1] + e[2]);
-          mbar_arrive(&ms->scale_ready);
-        }
-      }
-      if (n == hh) {  // this warpgroup's first chunk: take the scale
+        // ---- the CTA's input scale comes from its first chunk (warpgroup 0): the warps'
+        // largest |q|, |k|, |v| travel with the cumsum exchange below
+        const uint3 m = own_absmax_bits(sb, row0, cc, wtid);
+        if (lane == 0) ms->smax[w4][0] = m.x, ms->smax[w4][1] = m.y, ms->smax[w4][2] = m.z;
+      } else if (n == 1) {  // warpgroup 1's first chunk: take the scale warpgroup 0 set
         if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot)) {
           alive = false;
           break;
@@ -1059,6 +1089,31 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_float4(incl[ps][0], incl[ps][1], incl[ps][2], incl[ps][3]);
       }
       wg_sync(wg);
+      if (n == 0) {
+        // powers of two, so that scaling and undoing it are exact (every thread of the
+        // warpgroup derives the same factors; thread 0 publishes them to the other roles)
+        int e[3];
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
+          e[t] = input_scale_exp(bits16_to_float<Tin>(m));
+        }
+        sq = pow2f(e[0]);
+        sk = pow2f(e[1]);
+        sv = pow2f(e[2]);
+        if (wtid == 0) {
+          ms->sc_in[0] = sq;
+          ms->sc_in[1] = sk;
+          ms->sc_in[2] = sv;
+          ms->sc_out = pow2f(-(e[0] + e[1] + e[2]));
+          ms->sc_spub = pow2f(-(e[1] + e[2]));
+          ms->sc_sin = pow2f(e[1] + e[2]);
+          mbar_arrive(&ms->scale_ready);
+        }
+      }
+      // a CTA with tiny inputs first scales the q and k elements this thread builds (the
+      // CUDA-core scores below read them after a barrier)
+      if (sq != 1.f || sk != 1.f) prescale_own<Tin>(sb, row0, cc, sq, sk);
       // offsets of my rows (the rows of earlier lanes and warps) and the chunk decay a
       float off[2][4], last[2][4];
       bool exp_unsafe = false;
@@ -1101,7 +1156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
         tc_fence_after();  // (the wait's barrier also publishes the full A)
         cuda_core_scores<Tin, rev>(sb, G, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU), w4,
-                                   lane, 0.125f * sq * sk);
+                                   lane, 0.125f);
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);  // raw q / k reads done before the overwrite
@@ -1110,11 +1165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) off[ps][e] = 0.f;  // the gate tile holds the full A now
       }
-      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place, times
-      // the CTA's input scale factors
+      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
       const __half2 eighth = __float2half2_rn(0.125f);
-      const bool scl = sq != 1.f || sk != 1.f;
-      const float kf = 0.125f * sk;
 #pragma unroll 1
       for (int ps = 0; ps < 2; ++ps) {  // (rolled: the loop body stays small for the instruction cache)
         const int ch0 = 32 * ps + 4 * cc;
@@ -1142,13 +1194,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float xk0 = fbx ? lastp[2 * e2] - A0 : -A0;
             const float xk1 = fbx ? lastp[2 * e2 + 1] - A1 : -A1;
             __half2 qh, kh;
-            if (std::is_same<Tin, __half>::value && !scl) {
+            if constexpr (std::is_same<Tin, __half>::value) {
               qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
               kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
             } else {
               const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
-              qh = __floats2half2_rn(qv.x * sq * ex2(A0), qv.y * sq * ex2(A1));
-              kh = __floats2half2_rn(kv.x * kf * ex2(xk0), kv.y * kf * ex2(xk1));
+              qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
+              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
             }
             qw[e2] = h2_bits(qh);
             kw[e2] = h2_bits(kh);
@@ -1185,8 +1237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->opready[st]);  // every warp, once its writes are done
     }
-    if (partial && alive) second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
-
   } else if (warp < 12) {
     // ===================================================================== WG_B: masking, state
     // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
@@ -1313,9 +1363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       wg_sync(wg);
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
     }
-    if (segm && alive) {
-      // segment summary: U_seg = local end state (in the inputs' scale), its log2 decay, and
-      // the factor that takes a start state into this CTA's scale
+    if (segm && alive && seg + 1 < fp.n_s) {
+      // segment summary, read by the later segments of the sequence: U_seg = local end state
+      // (in the inputs' scale) and its log2 decay; then the segment's flag
       float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * kAggStride;
       const float f = ms->sc_spub;
 #pragma unroll
@@ -1328,12 +1378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mine[4096 + r0] = a2r0;
         mine[4096 + r1] = a2r1;
       }
-      if (wtid == 0) mine[4096 + 64] = ms->sc_sin;
       __threadfence();
       wg_sync(wg);
-      if (wtid == 0) mbar_arrive(&ms->agg_pub);
-      if (partial) second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
+      if (wtid == 0) st_release_u32(fp.counters + (size_t)seq * fp.n_s + seg, 1u);
     }
+    if (segm && alive && wtid == 0) mbar_arrive(&ms->agg_pub);
   } else if (warp < 16) {
     // ===================================================================== WG_C: epilogue, scan
     const int wg = 3, wtid = tid - 3 * kWG, wq = warp & 3;
@@ -1384,118 +1433,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the O_local rows written above are read back by bulk copy (async proxy)
       if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-    if (segm && alive) {
-      // Scan of the segment summaries.  This CTA owns state entries [4 f0, 4 f1) (float4
-      // units f, F of them).  Threads split into nB blocks of bs consecutive segments x FP
-      // float4 columns (nB * FP <= 128): a thread loads its block's summaries for its f
-      // all at once (consecutive threads read consecutive float4s), composes them
-      // sequentially, and the block compositions are exchanged through shared memory;
-      // each thread then walks its segments again from its block's carry-in, writing
-      // each segment's start state (fp16, MMA layout).
-      const int ns = fp.n_s;
-      const int f0 = (int)((long long)seg * 1024 / ns), f1 = (int)((long long)(seg + 1) * 1024 / ns);
-      const int F = f1 - f0;
-      int nB = kWG / (F > 0 ? F : 1);
-      nB = nB < 1 ? 1 : (nB > ns ? ns : nB);
-      if ((ns + nB - 1) / nB > kScanBlock) nB = (ns + kScanBlock - 1) / kScanBlock;
-      const int bs = (ns + nB - 1) / nB;
-      const int FP = kWG / nB;
-      const int bi = wtid / FP, fi = wtid % FP;
-      const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
-      unsigned int* ctr = fp.counters + (size_t)seq * 2;
-      const float* aggs = fp.agg + (size_t)seq * ns * kAggStride;
-      uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
-      float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
-      float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
-      const unsigned int target = (unsigned int)ns;
-      bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
-      if (ok0) {
-        if (wtid == 0) {
-          // the second phase's first four pairs start loading now (every MMA of this
-          // CTA has completed, so all staging buffers are free; the Qh' and O_local
-          // tiles are written and fenced)
-          if (partial)
-            for (int q = 0; q < 4 && 2 * q < cnt; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
-          red_release_add(ctr, 1u);
-          ok0 = wait_counter(ctr, target, ms, hdr, 0x601);
-        }
-        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
+  }
+
+  if (segm && tid < 4 * kWG) {
+    // ===================================================================== SEGMENTED combine
+    // Every thread of warps 0-15 meets here (every wait before is bounded).  A segment s > 0
+    // waits for the flags of segments 0 .. s-1 of its sequence (their summaries are
+    // published), composes its start state from those summaries itself -- thread t owns the
+    // eight state entries 8t .. 8t+7 (key channel t/8) and walks the segments in order, so
+    // the result does not depend on timing -- and writes it (fp16, MMA layout, in this CTA's
+    // scale) straight into shared memory; then all four warpgroups run the second phase.
+    // Segment 0's outputs are final already.
+    named_sync(7, 4 * kWG);
+    if (seg > 0) {
+      if (tid == 0) {
+        // the Qh' and O_local tiles are written and fenced once the summary is out (WG_B and
+        // the Qh' warp arrive): the first four pairs of the second phase start loading now
+        bool ok = !*(volatile int*)&ms->abort && wait_bar(&ms->agg_pub, 0u, ms, hdr, 0x600);
+        if (ok)
+          for (int q = 0; q < 4 && 2 * q < cnt; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
+        for (int j = 0; j < seg && ok; ++j)
+          ok = wait_counter(fp.counters + (size_t)seq * fp.n_s + j, 1u, ms, hdr, 0x601);
+        ms->seg_go = ok ? 1 : 0;
       }
-      if (ok0) {
-        for (int sg = wtid; sg < ns; sg += kWG) ms->segfac[sg] = __ldcg(aggs + (size_t)sg * kAggStride + 4096 + 64);
-        wg_sync(wg);
-        for (int base = f0; base < f1; base += FP) {
-          const int f = base + fi;
-          const bool act = bi < nB && f < f1;
-          const int kk = f >> 4;
-          float4 u[kScanBlock];
-          float dd[kScanBlock];
-          float4 X = make_float4(0.f, 0.f, 0.f, 0.f);
+      named_sync(7, 4 * kWG);
+      const bool go = *(volatile int*)&ms->seg_go != 0;
+      if (go) {
+        const int kk = tid >> 3, v0 = 8 * (tid & 7);
+        const float* aggs = fp.agg + (size_t)seq * fp.n_s * kAggStride;
+        float x[8];
 #pragma unroll
-          for (int j = 0; j < kScanBlock; ++j) {
-            const int sg = s_lo + j;
-            const bool on = act && sg < s_hi;
-            const float* a2p = aggs + (size_t)(on ? sg : 0) * kAggStride;
-            u[j] = on ? __ldcg(reinterpret_cast<const float4*>(a2p) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-            dd[j] = on ? __ldcg(a2p + 4096 + kk) : 0.f;
-          }
-          // this block's transfer: state_after = D * state_before + U
-          float D = 1.f;
-          float4 U = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        // X <- 2^d_j X + U_j over j = 0 .. s-1, four summaries' loads in flight at a time
+        for (int j0 = 0; j0 < seg; j0 += 4) {
+          float4 ua[4], ub[4];
+          float dj[4];
 #pragma unroll
-          for (int j = 0; j < kScanBlock; ++j) {
-            dd[j] = ex2(dd[j]);  // inactive entries: 2^0 = 1 with a zero summary
-            U = make_float4(fmaf(dd[j], U.x, u[j].x), fmaf(dd[j], U.y, u[j].y), fmaf(dd[j], U.z, u[j].z),
-                            fmaf(dd[j], U.w, u[j].w));
-            D *= dd[j];
+          for (int i = 0; i < 4; ++i) {
+            const bool on = j0 + i < seg;
+            const float* a = aggs + (size_t)(on ? j0 + i : 0) * kAggStride;
+            ua[i] = __ldcg(reinterpret_cast<const float4*>(a + 8 * tid));
+            ub[i] = __ldcg(reinterpret_cast<const float4*>(a + 8 * tid + 4));
+            dj[i] = __ldcg(a + 4096 + kk);
           }
-          if (nB > 1) {
-            if (bi < nB) {
-              xD[bi * FP + fi] = D;
-              xU[bi * FP + fi] = U;
-            }
-            wg_sync(wg);
-            for (int b2 = 0; b2 < bi && b2 < nB; ++b2) {
-              const float d2 = xD[b2 * FP + fi];
-              const float4 u2 = xU[b2 * FP + fi];
-              X = make_float4(fmaf(d2, X.x, u2.x), fmaf(d2, X.y, u2.y), fmaf(d2, X.z, u2.z), fmaf(d2, X.w, u2.w));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (j0 + i < seg) {
+              const float d = ex2(dj[i]);
+              x[0] = fmaf(d, x[0], ua[i].x); x[1] = fmaf(d, x[1], ua[i].y);
+              x[2] = fmaf(d, x[2], ua[i].z); x[3] = fmaf(d, x[3], ua[i].w);
+              x[4] = fmaf(d, x[4], ub[i].x); x[5] = fmaf(d, x[5], ub[i].y);
+              x[6] = fmaf(d, x[6], ub[i].z); x[7] = fmaf(d, x[7], ub[i].w);
             }
           }
-          if (act) {
-            const int v0 = 4 * (f & 15);
-            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (v0 & 7) * 2;
-#pragma unroll
-            for (int j = 0; j < kScanBlock; ++j) {
-              const int sg = s_lo + j;
-              if (sg < s_hi) {
-                const float fs = ms->segfac[sg];  // into segment sg's CTA scale
-                const uint2 w = make_uint2(pack_h2(X.x * fs, X.y * fs), pack_h2(X.z * fs, X.w * fs));
-                __stcg(reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(sst + (size_t)sg * 4096) + soff), w);
-                X = make_float4(fmaf(dd[j], X.x, u[j].x), fmaf(dd[j], X.y, u[j].y), fmaf(dd[j], X.z, u[j].z),
-                                fmaf(dd[j], X.w, u[j].w));
-              }
-            }
-          }
-          if (nB > 1) wg_sync(wg);  // the exchange slots are reused by the next column pass
         }
-        __threadfence();
-        wg_sync(wg);
-        if (wtid == 0) {
-          red_release_add(ctr + 1, 1u);
-          ok0 = wait_counter(ctr + 1, target, ms, hdr, 0x602);
-        }
-        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
+        // row kk, columns v0 .. v0+7: one 16-byte piece of the 128-byte-swizzled start-state tile
+        const float f = ms->sc_sin;
+        const uint4 w = make_uint4(pack_h2(x[0] * f, x[1] * f), pack_h2(x[2] * f, x[3] * f),
+                                   pack_h2(x[4] * f, x[5] * f), pack_h2(x[6] * f, x[7] * f));
+        *reinterpret_cast<uint4*>(smem + kOffSst + kk * 128 + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4)) = w;
+        fence_proxy_async_smem();  // read by the second phase's MMAs
       }
-      if (ok0 && partial) {
-        // this segment's start state -> shared memory (already in the MMA layout), then
-        // the second phase on all four warpgroups
-        const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
-        uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
-        for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
-        fence_proxy_async_smem();
-        wg_sync(wg);
-        if (wtid == 0) mbar_arrive(&ms->p2_go);
-        second_phase<Tout>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
+      named_sync(7, 4 * kWG);
+      if (go) {
+        const int q = warp >> 2;
+        int slot2 = 0;
+        second_phase<Tout>(fp, ms, hdr, smem, tmem, q, tid - kWG * q, lane, seq, b, h, sp, slot2, nonfinite);
       }
     }
   }
@@ -1622,7 +1625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __threadfence();
     const unsigned int done = atomicAdd(&hdr->ticket, 1u);
     if (done == (unsigned int)fp.grid - 1) {
-      for (int i = 0; i < 2 * fp.n_seq; ++i) fp.counters[i] = 0u;
+      for (int i = 0; i < fp.grid; ++i) fp.counters[i] = 0u;
       __threadfence();
       hdr->ticket = 0u;
     }
@@ -1853,7 +1856,6 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.hdr = w.hdr;
   fp.counters = w.counters;
   fp.agg = w.agg;
-  fp.sstart = w.sstart;
   fp.qhp = w.qhp;
   fp.olc = w.olc;
   fp.n_seq = pl.n_seq;
@@ -1878,15 +1880,14 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
     attr[na].val.clusterDim.z = 1;
     ++na;
   }
-  if (pl.mode == 1) {  // the CTAs of a sequence wait on one another
-    attr[na].id = cudaLaunchAttributeCooperative;
-    attr[na].val.cooperative = 1;
-    ++na;
-  } else {  // the prologue may overlap the previous launch's tail
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-  }
+  // the prologue may overlap the previous launch's tail (every mode).  In SEGMENTED mode
+  // the CTAs of a sequence wait on the segments before them: the grid is at most one CTA
+  // per SM (kernel occupancy 1), so every CTA becomes resident once the previous grid has
+  // drained -- a later launch cannot take SMs before every CTA of this one has started
+  // (griddepcontrol.launch_dependents fires per CTA) -- and every wait is bounded.
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
   cfg.attrs = attr;
   cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, kerns[pl.mode], fp) != cudaSuccess) return GTR_ERR_CUDA;
