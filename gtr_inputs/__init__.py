@@ -120,3 +120,81 @@ def make_inputs(w: Workload, seed: int, device: Optional[str] = None):
 
 def empty_out(w: Workload, device=None) -> torch.Tensor:
     return torch.empty((w.B, w.L, w.heads, w.d_v), dtype=DTYPES[w.out_dtype], device=device)
+
+
+# ----------------------------------------------------------------------------- GTR block pieces
+# The recipes below draw the extra inputs of the block-level calls; like make_inputs they
+# hold no arithmetic of the method.  GTR-L's widths (0539edu.com appendix D.1.1): model
+# dimension 384 over 6 heads, S-SwiGLU expansion ratio 4 (hidden width 1536; GTR-X 6).
+GATE_RANK = 16   # rank of the gate factorisation (GTR digest page, "Core method")
+GATE_TAU = 16.0  # gamma = sigmoid(.)^(1/tau)
+
+
+def make_lowrank_gate_inputs(w: Workload, seed: int, rank: int = GATE_RANK, offset: Optional[float] = None):
+    """(z, w2, bias) for the low-rank gate producer, fp32: z = x W1 ~ N(0, 1) [B, L, rank];
+    W2 ~ N(0, 1/rank) [rank, heads * d_k], so that z W2 ~ N(0, 1) per entry like the
+    direct gate recipe; bias = the workload's gate offset (default) [heads * d_k]."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed) + 555)
+    z = torch.randn((w.B, w.L, rank), generator=gen, dtype=torch.float32)
+    w2 = torch.randn((rank, w.heads * w.d_k), generator=gen, dtype=torch.float32) / rank ** 0.5
+    off = w.gate_offset if offset is None else offset
+    bias = torch.full((w.heads * w.d_k,), float(off), dtype=torch.float32)
+    return z, w2, bias
+
+
+def make_gate_epilogue_inputs(w: Workload, seed: int):
+    """(gate, weight, eps) for the RMSNorm + SiLU output gate: gate ~ N(0, 1) in the input
+    dtype [B, L, heads, d_v]; weight ~ 1 + 0.1 N(0, 1) fp32 [d_v]; eps = 1e-6."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed) + 777)
+    gate = torch.randn((w.B, w.L, w.heads, w.d_v), generator=gen, dtype=torch.float32).to(DTYPES[w.dtype])
+    weight = 1.0 + 0.1 * torch.randn((w.d_v,), generator=gen, dtype=torch.float32)
+    return gate, weight, 1e-6
+
+
+@dataclass(frozen=True)
+class StencilWorkload:
+    """Spatial SwiGLU stencil: the two projections X W_g, X W_v of an H x W token grid."""
+    name: str
+    B: int
+    H: int
+    W: int
+    C: int
+    dtype: str = "f16"
+    bias: bool = True
+    index: int = 0
+
+    @property
+    def L(self) -> int:
+        return self.H * self.W
+
+    def algorithmic_bytes(self) -> int:
+        """HBM bytes one call must move: read xg and xv, write z (all in dtype), plus the
+        3x3 weights and bias (fp32)."""
+        es = torch.finfo(DTYPES[self.dtype]).bits // 8
+        return 3 * self.B * self.L * self.C * es + self.C * 10 * 4
+
+    def with_(self, **kw) -> "StencilWorkload":
+        return replace(self, **kw)
+
+
+STENCILS = {
+    s.name: s
+    for s in [
+        # GTR-L hidden width 1536 on the 640^2 / 1024^2 / 2048^2 grids
+        StencilWorkload("sw640", B=1, H=40, W=40, C=1536, dtype="f16", index=11),
+        StencilWorkload("sw1024", B=1, H=64, W=64, C=1536, dtype="bf16", index=12),
+        StencilWorkload("sw2048", B=1, H=128, W=128, C=1536, dtype="f16", index=13),
+    ]
+}
+
+
+def make_stencil_inputs(s: StencilWorkload, seed: int):
+    """(xg, xv, conv_w, conv_b): xg, xv ~ N(0, 1) in the stencil's dtype [B, L, C];
+    3x3 depthwise weights ~ N(0, 1/9) fp32 [C, 3, 3]; bias ~ 0.1 N(0, 1) fp32 [C] (or None)."""
+    gen = torch.Generator(device="cpu").manual_seed(int(seed))
+    dt = DTYPES[s.dtype]
+    xg = torch.randn((s.B, s.L, s.C), generator=gen, dtype=torch.float32).to(dt)
+    xv = torch.randn((s.B, s.L, s.C), generator=gen, dtype=torch.float32).to(dt)
+    conv_w = torch.randn((s.C, 3, 3), generator=gen, dtype=torch.float32) / 3.0
+    conv_b = 0.1 * torch.randn((s.C,), generator=gen, dtype=torch.float32) if s.bias else None
+    return xg, xv, conv_w, conv_b

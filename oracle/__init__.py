@@ -183,3 +183,86 @@ def gla_fwd_chunked(q, k, v, log_gamma, H: int, W: int, direction: int = 0,
                 S = np.exp(A[-1])[:, None] * S + U
             out[b, order, h] = O
     return out
+
+
+# ----------------------------------------------------------------------------- GTR block pieces
+def _log_sigmoid(g: np.ndarray) -> np.ndarray:
+    """log(sigmoid(g)) = -log(1 + exp(-g)), written so that neither branch overflows."""
+    return np.minimum(g, 0.0) - np.log1p(np.exp(-np.abs(g)))
+
+
+def lowrank_log_gamma(z, w2, bias, tau: float, heads: int, d_k: int) -> np.ndarray:
+    """The low-rank data-dependent retention gate of GTR, in log form.
+
+    GTR digest page (paper.rainbus.top), section "Core method": the key-side gate is
+    gamma_t = sigmoid(x_t W1 W2 + b)^(1/tau) with a rank-16 factorisation and tau = 16.
+    With z = x W1 (the rank-r projection of each token, [B, L, r]), W2 of shape
+    [r, heads * d_k] and b of shape [heads * d_k]:
+
+        log gamma[b, m, h, :] = log sigmoid(z[b, m] W2 + b)[h * d_k : (h + 1) * d_k] / tau
+
+    Returns [B, L, heads, d_k] in float64.
+    """
+    z, w2, bias = _f64(z), _f64(w2), _f64(bias)
+    B, L, _ = z.shape
+    g = z @ w2 + bias
+    return (_log_sigmoid(g) / float(tau)).reshape(B, L, heads, d_k)
+
+
+def gla_fwd_lowrank(q, k, v, z, w2, bias, tau: float, H: int, W: int, direction: int = 0) -> np.ndarray:
+    """The recurrence (:func:`gla_fwd`) with its gates produced by :func:`lowrank_log_gamma`."""
+    qq = _f64(q)
+    heads, d_k = qq.shape[2], qq.shape[3]
+    return gla_fwd(qq, k, v, lowrank_log_gamma(z, w2, bias, tau, heads, d_k), H, W, direction)
+
+
+def rmsnorm_silu_gate(o, gate, weight, eps: float) -> np.ndarray:
+    """The GLA output epilogue: RMSNorm over the d_v channels of each token-head, the norm
+    weight, then the SiLU-activated output gate.
+
+    0539edu.com, appendix E.3.1: the end-to-end implementation fuses RMSNorm and a
+    SiLU-activated output gate into the GLA kernel's output epilogue.  Per token-head row
+    o (d_v values), gate r (d_v values) and weight w (d_v values, shared by the heads):
+
+        y_j = o_j / sqrt(mean_i o_i^2 + eps) * w_j * r_j * sigmoid(r_j)
+    """
+    o, r, w = _f64(o), _f64(gate), _f64(weight)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + float(eps))
+    return o / rms * w * (r / (1.0 + np.exp(-r)))
+
+
+def gla_fwd_gated(q, k, v, log_gamma, gate, weight, eps: float, H: int, W: int,
+                  direction: int = 0) -> np.ndarray:
+    """The recurrence (:func:`gla_fwd`) followed by :func:`rmsnorm_silu_gate`."""
+    return rmsnorm_silu_gate(gla_fwd(q, k, v, log_gamma, H, W, direction), gate, weight, eps)
+
+
+def sswiglu_dwconv(xg, xv, conv_w, conv_b, H: int, W: int) -> np.ndarray:
+    """The spatial part of GTR's Spatial SwiGLU: SiLU(X W_g) * DWConv3x3(X W_v).
+
+    GTR digest page, prerequisite "SwiGLU" and section "Core method": the channel mixer is
+    Y = SiLU(X W_g) (.) DWConv3x3(X W_v) W_o, a 3x3 depthwise convolution in the value
+    branch that mixes neighbouring patches (0539edu.com section 3.1 "Spatial SwiGLU").
+    This computes the product before W_o from the two projections xg = X W_g and
+    xv = X W_v, both [B, L, C] with token m = y * W + x on the H x W grid.  The
+    convolution is channel by channel, stride 1, zero padding 1, in the cross-correlation
+    convention of a convolution layer:
+
+        conv[b, y, x, c] = bias[c] + sum_{dy, dx in 0..2} w[c, dy, dx] * xv[b, y+dy-1, x+dx-1, c]
+
+    conv_b may be None (no bias).  Returns [B, L, C] in float64.
+    """
+    xg, xv, w = _f64(xg), _f64(xv), _f64(conv_w)
+    B, L, C = xv.shape
+    if L != H * W or xg.shape != xv.shape or w.shape != (C, 3, 3):
+        raise ValueError("shape mismatch")
+    img = np.zeros((B, H + 2, W + 2, C))
+    img[:, 1:H + 1, 1:W + 1, :] = xv.reshape(B, H, W, C)
+    conv = np.zeros((B, H, W, C))
+    for dy in range(3):
+        for dx in range(3):
+            conv += img[:, dy:dy + H, dx:dx + W, :] * w[:, dy, dx]
+    if conv_b is not None:
+        conv += _f64(conv_b)
+    silu = xg / (1.0 + np.exp(-xg))
+    return silu * conv.reshape(B, L, C)
