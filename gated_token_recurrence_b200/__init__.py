@@ -31,7 +31,7 @@ STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "G
 EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
             "gtr_gla_workspace_bytes", "gtr_gla_fwd_ex", "gtr_gla_fwd_host",
             "gtr_gla_read_error", "gtr_gla_plan", "gtr_gla_workspace_init", "gtr_status_string",
-            "gtr_version", "gtr_gla_fwd_noalloc")
+            "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd")
 
 
 class GTRError(RuntimeError):
@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
     lib.gtr_gla_fwd_ex.argtypes = fwd_args + [i, i, i, vp, sz, vp]
     lib.gtr_gla_fwd_host.argtypes = fwd_args + [i, i, vp]
     lib.gtr_gla_fwd_noalloc.argtypes = fwd_args + [i, i, vp]
+    f = ctypes.c_float
+    lib.gtr_gla_block_fwd.argtypes = [vp] * 7 + [i, f, vp, vp, f, vp] + [i] * 10 + [vp, sz, vp]
     lib.gtr_gla_workspace_bytes.argtypes = [i] * 8
     lib.gtr_gla_workspace_bytes.restype = sz
     lib.gtr_gla_read_error.argtypes = [vp, vp]
@@ -64,7 +66,7 @@ def _load() -> ctypes.CDLL:
     lib.gtr_version.argtypes = []
     for name in ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
                  "gtr_gla_fwd_ex", "gtr_gla_fwd_host", "gtr_gla_read_error", "gtr_gla_plan",
-                 "gtr_gla_workspace_init", "gtr_version", "gtr_gla_fwd_noalloc"):
+                 "gtr_gla_workspace_init", "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -147,6 +149,39 @@ def gla_fwd(q, k, v, log_gamma, grid: Tuple[int, int], direction: int = L2R, out
             workspace = new_workspace(B, heads, H, W, d_k, d_v, _dtype_code(q), path, q.device)
         _check(lib.gtr_gla_fwd_ex(*args, PATHS[path], workspace.data_ptr(), workspace.numel(), s),
                "gtr_gla_fwd_ex")
+    return out
+
+
+def gla_block_fwd(q, k, v, grid: Tuple[int, int], direction: int = L2R, log_gamma=None,
+                  gate_z=None, gate_w2=None, gate_b=None, gate_tau: float = 16.0,
+                  out_gate=None, norm_w=None, norm_eps: float = 1e-6, out=None, path: str = "auto",
+                  workspace=None, stream=None):
+    """The GLA token mixer of a GTR block (``gtr_gla_block_fwd``) on CUDA tensors.
+
+    Gates: either ``log_gamma`` [B, L, heads, d_k] fp32, or the low-rank producer
+    ``gate_z`` [B, L, r] fp32 with ``gate_w2`` [r, heads*d_k] and ``gate_b`` [heads*d_k]
+    (log gamma = logsigmoid(z W2 + b) / gate_tau).  With ``out_gate`` [B, L, heads, d_v]
+    (input dtype) and ``norm_w`` [d_v] fp32 the output is RMSNorm(o) * norm_w * SiLU(out_gate).
+    """
+    import torch
+    B, heads, H, W, d_k, d_v = _shape(q, v, grid)
+    if out is None:
+        out = torch.empty((B, H * W, heads, d_v), dtype=default_out_dtype(q.dtype), device=q.device)
+    tensors = [t for t in (q, k, v, log_gamma, gate_z, gate_w2, gate_b, out_gate, norm_w, out) if t is not None]
+    for t in tensors:
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("gla_block_fwd takes contiguous CUDA tensors")
+    for t in (log_gamma, gate_z, gate_w2, gate_b, norm_w):
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError("gates, gate factors and the norm weight are float32")
+    ptr = lambda t: None if t is None else t.data_ptr()
+    rank = 0 if gate_z is None else int(gate_z.shape[-1])
+    ws, wsb = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    st = lib.gtr_gla_block_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), ptr(log_gamma), ptr(gate_z),
+                               ptr(gate_w2), ptr(gate_b), rank, float(gate_tau), ptr(out_gate), ptr(norm_w),
+                               float(norm_eps), out.data_ptr(), B, heads, H, W, d_k, d_v, int(direction),
+                               _dtype_code(q), _dtype_code(out), PATHS[path], ws, wsb, _stream_handle(stream))
+    _check(st, "gtr_gla_block_fwd")
     return out
 
 

@@ -32,7 +32,7 @@ gtr_status_t check_shape(int B, int heads, int H, int W, int d_k, int d_v, int d
   if (in_dtype < GTR_F32 || in_dtype > GTR_BF16 || out_dtype < GTR_F32 || out_dtype > GTR_BF16)
     return GTR_ERR_INVALID_ARG;
   if (!dtype_pair_ok(in_dtype, out_dtype)) return GTR_ERR_UNSUPPORTED;
-  if (d_k != kD || d_v != kD) return GTR_ERR_UNSUPPORTED;
+  if ((d_k != kD && d_k != 32) || d_v != kD) return GTR_ERR_UNSUPPORTED;
   const long long L = (long long)H * W;
   if (L > (1ll << 28) || B > 65535 || heads > 65535) return GTR_ERR_UNSUPPORTED;
   if ((long long)B * L * heads * kD >= (1ll << 40)) return GTR_ERR_UNSUPPORTED;
@@ -240,6 +240,57 @@ gtr_status_t gtr_gla_fwd_ex(const void* q, const void* k, const void* v, const f
   const Problem p = make_problem(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v,
                                  direction, in_dtype, out_dtype);
   return run(p, path, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+gtr_status_t gtr_gla_block_fwd(const void* q, const void* k, const void* v, const float* log_gamma,
+                               const float* gate_z, const float* gate_w2, const float* gate_b, int gate_rank,
+                               float gate_tau, const void* out_gate, const float* norm_w, float norm_eps, void* out,
+                               int B, int heads, int grid_H, int grid_W, int d_k, int d_v, int direction,
+                               int in_dtype, int out_dtype, int path, void* workspace, size_t ws_bytes,
+                               gtr_stream_t stream) {
+  gtr_status_t st = check_shape(B, heads, grid_H, grid_W, d_k, d_v, direction, in_dtype, out_dtype);
+  if (st != GTR_OK) return st;
+  // exactly one source of the gates
+  if ((log_gamma == nullptr) == (gate_z == nullptr)) return GTR_ERR_INVALID_ARG;
+  const float* lg = log_gamma ? log_gamma : gate_z;  // (pointer checks below cover both)
+  st = check_ptrs(q, k, v, lg, out);
+  if (st != GTR_OK) return st;
+  if (gate_z) {
+    if (!gate_w2 || !gate_b || !is_aligned(gate_w2, 16) || !is_aligned(gate_b, 16)) return GTR_ERR_INVALID_ARG;
+    if (gate_rank < 4 || gate_rank > 16 || gate_rank % 4 != 0) return GTR_ERR_INVALID_ARG;
+    if (!(gate_tau > 0.f) || !(gate_tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+  }
+  if (out_gate) {
+    if (!norm_w || !is_aligned(out_gate, 16) || !is_aligned(norm_w, 16)) return GTR_ERR_INVALID_ARG;
+    if (!(norm_eps >= 0.f) || !(norm_eps < 3.0e38f)) return GTR_ERR_INVALID_ARG;
+  }
+  if (path < GTR_PATH_AUTO || path > GTR_PATH_FUSED_SEQUENTIAL) return GTR_ERR_INVALID_ARG;
+  Problem p = make_problem(q, k, v, log_gamma, out, B, heads, grid_H, grid_W, d_k, d_v, direction, in_dtype,
+                           out_dtype);
+  if (gate_z) {
+    p.gz = gate_z;
+    p.gw2 = gate_w2;
+    p.gb = gate_b;
+    p.grank = gate_rank;
+    p.gtau = gate_tau;
+  }
+  if (out_gate) {
+    p.ogate = out_gate;
+    p.onorm_w = norm_w;
+    p.oeps = norm_eps;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (workspace) return run(p, path, workspace, ws_bytes, s);
+  int dev;
+  st = current_device(&dev);
+  if (st != GTR_OK) return st;
+  DeviceCache& c = g_cache[dev];
+  std::lock_guard<std::mutex> lock(c.mu);
+  const size_t need = path_workspace_bytes(p, choose_path(p, path));
+  if (need == 0) return GTR_ERR_UNSUPPORTED;
+  st = ensure(c.ws, need, s);
+  if (st != GTR_OK) return st;
+  return run(p, path, c.ws.ptr, c.ws.bytes, s);
 }
 
 gtr_status_t gtr_gla_workspace_init(void* workspace, size_t ws_bytes, gtr_stream_t stream) {

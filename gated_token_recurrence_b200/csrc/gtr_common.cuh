@@ -39,6 +39,20 @@ struct Problem {
   const float* log_gamma;
   void* out;
   int B, heads, H, W, d_k, d_v, direction, in_dtype, out_dtype;
+  // Low-rank gate producer (gz != nullptr; log_gamma is then not read): log gamma of
+  // token m, head h = logsigmoid(gz[b, m, :] gw2[:, h*d_k .. h*d_k+d_k-1] + gb[h*d_k ..]) / gtau,
+  // gz [B, L, grank] fp32, gw2 [grank, heads * d_k] fp32, gb [heads * d_k] fp32.
+  const float* gz = nullptr;
+  const float* gw2 = nullptr;
+  const float* gb = nullptr;
+  float gtau = 1.f;
+  int grank = 0;
+  // RMSNorm + SiLU output gate (ogate != nullptr): out = o / sqrt(mean_j o_j^2 + oeps) *
+  // onorm_w * SiLU(ogate), per token-head over d_v; ogate [B, L, heads, d_v] in the input
+  // dtype, onorm_w [d_v] fp32.
+  const void* ogate = nullptr;
+  const float* onorm_w = nullptr;
+  float oeps = 0.f;
 
   __host__ __device__ long long L() const { return (long long)H * (long long)W; }
   __host__ __device__ int n_chunks() const { return (int)((L() + kChunk - 1) / kChunk); }

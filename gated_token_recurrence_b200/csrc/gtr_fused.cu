@@ -1,7 +1,7 @@
 // Fused path, host side: workspace layout and the dtype dispatch of the launches.
 // The kernel and its launch live in gtr_fused_kernel.cuh; each input/output dtype
-// pair is instantiated in a translation unit of its own (gtr_fused_<in>_<out>.cu) so
-// that the kernels compile in parallel.
+// pair and key width is instantiated in a translation unit of its own
+// (gtr_fused_<in>_<out>_dk<d_k>.cu) so that the kernels compile in parallel.
 #include "gtr_fused_kernel.cuh"
 
 namespace gtr {
@@ -46,11 +46,18 @@ int fused_launches(const Problem& p) {
 
 gtr_status_t launch_fused(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
   if ((long long)p.B * p.L() >= (1ll << 31)) return GTR_ERR_UNSUPPORTED;
+  const bool dk32 = p.d_k == 32;
   switch (p.in_dtype * 3 + p.out_dtype) {
-    case GTR_F16 * 3 + GTR_F16: return launch_fused_f16_f16(p, ws, stream, force_mode);
-    case GTR_F16 * 3 + GTR_F32: return launch_fused_f16_f32(p, ws, stream, force_mode);
-    case GTR_BF16 * 3 + GTR_F32: return launch_fused_bf16_f32(p, ws, stream, force_mode);
-    case GTR_BF16 * 3 + GTR_BF16: return launch_fused_bf16_bf16(p, ws, stream, force_mode);
+    case GTR_F16 * 3 + GTR_F16:
+      return dk32 ? launch_fused_f16_f16_dk32(p, ws, stream, force_mode) : launch_fused_f16_f16_dk64(p, ws, stream, force_mode);
+    case GTR_F16 * 3 + GTR_F32:
+      return dk32 ? launch_fused_f16_f32_dk32(p, ws, stream, force_mode) : launch_fused_f16_f32_dk64(p, ws, stream, force_mode);
+    case GTR_BF16 * 3 + GTR_F32:
+      return dk32 ? launch_fused_bf16_f32_dk32(p, ws, stream, force_mode)
+                  : launch_fused_bf16_f32_dk64(p, ws, stream, force_mode);
+    case GTR_BF16 * 3 + GTR_BF16:
+      return dk32 ? launch_fused_bf16_bf16_dk32(p, ws, stream, force_mode)
+                  : launch_fused_bf16_bf16_dk64(p, ws, stream, force_mode);
     default: return GTR_ERR_UNSUPPORTED;
   }
 }

@@ -1,0 +1,11 @@
+// Fused-path kernels for f16 inputs, f16 outputs and d_k = 32 (one translation unit per
+// dtype pair and key width, so that the kernel instantiations compile in parallel).
+#include "gtr_fused_kernel.cuh"
+
+namespace gtr {
+
+gtr_status_t launch_fused_f16_f16_dk32(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
+  return launch_fused_typed<__half, __half, 32>(p, ws, stream, force_mode);
+}
+
+}  // namespace gtr

@@ -74,6 +74,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTile = 8192;
 constexpr int kGTile = 16384;                        // fp32 log-gates [64][64]
 constexpr int kStageBytes = 3 * kTile + kGTile;      // Q (-> Qh), K (-> Kh), V, G
+// d_k = 32: the gates take the first half of the gate tile (64 rows of 32 fp32), and the
+// raw q and k (dense 64-byte rows) its second half; Qh and Kh are built, zero-padded to 64
+// channels, into the Q and K tiles
+constexpr int kRawQ = 8192, kRawK = 12288;  // byte offsets in the gate tile
+// bytes one chunk's loads bring: q, k (64 x d_k x 2 B), v (8 KB), log-gates (64 x d_k x 4 B)
+template <int kDK> constexpr uint32_t chunk_load_bytes() { return 2u * 64 * kDK * 2 + kTile + 64u * kDK * 4; }
+
 constexpr int kOffStage = 0;
 constexpr int kNS = 5;                                     // chunk-start state tiles
 constexpr int kOffS = kOffStage + kStages * kStageBytes;   // [kNS] chunk-start states
@@ -81,7 +88,7 @@ constexpr int kOffSst = kOffS;                             // segment start stat
 constexpr int kOffStg = kOffS + kNS * kTile;               // output staging, 4 warps x 32 rows x 128 B
 constexpr int kStgBytes = 4 * 32 * 128;                    // (CLUSTER: first the segment summary, fp32)
 constexpr int kOffMisc = kOffStg + kStgBytes;
-constexpr int kMiscBytes = 8192;
+constexpr int kMiscBytes = 9216;
 constexpr int kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 // second phase, pair slot q (one per warpgroup) in staging buffer q: Qh' of the pair
 // (16 KB, the A operand; then the warps' fp32 output staging) and O_local (16 KB)
@@ -130,6 +137,7 @@ struct alignas(64) FusedParams {
   // row view [B][L][heads][64] (4-D) or column view [B][H][W][heads][64] (5-D), boxes of
   // 64 consecutive scan positions of one (batch, head)
   CUtensorMap tq, tk, tv, tg;
+  CUtensorMap tz;          // low-rank gate producer: the rank-r token projections z (fp32), same views
   Problem p;
   WsHeader* hdr;
   unsigned int* counters;  // SEGMENTED: [n_seq][n_s] segment flags (summary published), zero between calls
@@ -142,6 +150,9 @@ struct alignas(64) FusedParams {
   int tma;                 // 1: one TMA box per tensor; 2: 4-row TMA gathers; 0: cp.async row copies
   int rev;                 // 1: chunks are staged in reverse scan order (right-to-left, bottom-to-top)
   FastDiv divW, divH;      // the grid width and height as invariant divisors
+  int lowrank;             // 1: the log-gates come from the low-rank producer (z tiles, p.gw2, p.gb)
+  float gtau_inv;          // 1 / tau of the gate producer
+  int gated;               // 1: RMSNorm + SiLU output gate on the final outputs (p.ogate, p.onorm_w)
 };
 
 // Scan position s (< L < 2^31) -> token index y*W + x: the direction remap (rows top to
@@ -162,6 +173,13 @@ __device__ __forceinline__ uint32_t scan_token(const FusedParams& fp, uint32_t s
   return y * W + x;
 }
 static_assert(alignof(FusedParams) >= 64, "tensor maps need 64-byte alignment");
+
+// Bytes one chunk's loads bring with the low-rank gate producer: the z rows (64 x rank
+// fp32) instead of the log-gates.
+template <int kDK>
+__device__ __forceinline__ uint32_t chunk_load_bytes(const FusedParams& fp, bool lowrank) {
+  return lowrank ? 2u * 64 * kDK * 2 + kTile + 64u * fp.p.grank * 4 : chunk_load_bytes<kDK>();
+}
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
@@ -186,6 +204,10 @@ struct Misc {
   float sc_sin;   // 2^(beta+gamma): a state in the inputs' scale into this CTA's scale (start states)
   unsigned int smax[4][3];  // WG_A0: per-warp largest |q|, |k|, |v| bit patterns of the first chunk
   int seg_go;               // SEGMENTED: the start state can be composed (the predecessors published)
+  alignas(16) float w2s[16][64];  // low-rank gate producer: this head's W2 columns [rank][64] (zero past d_k)
+  alignas(16) float bs[64];       // ... and bias (zero past d_k)
+  alignas(16) float nw[64];       // output gate: RMSNorm weight
+  int zrow[2][64];                // producer: z row b*L + m of each chunk row (gathers; -1 past the end)
   int abort;
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
@@ -213,6 +235,24 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// log2(x) on the special-function unit.
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log(sigmoid(x)) = min(x, 0) - log(1 + e^-|x|): neither term overflows; the log of
+// 1 + e^-|x| is taken in base 2 on the special-function unit.
+__device__ __forceinline__ float log_sigmoid_fast(float x) {
+  return fminf(x, 0.f) - 0.69314718055994531f * lg2(1.f + ex2(-fabsf(x) * 1.4426950408889634f));
+}
+
+// SiLU(x) = x * sigmoid(x) = x / (1 + e^-x).
+__device__ __forceinline__ float silu_fast(float x) {
+  return x * __frcp_rn(1.f + ex2(-x * 1.4426950408889634f));
 }
 
 // Bounded mbarrier wait: the thread sleeps in hardware until the phase completes; only
@@ -358,20 +398,74 @@ __device__ __forceinline__ int stage_chunk(int R, int j) {
   return R * kRowB + 16 * (j ^ swz);
 }
 
-// The 32 rows of one warp (its lanes of a tensor-memory region, 64 fp32 columns) ->
-// memory as Tout, 32 columns at a time.  Each lane writes its row into a per-warp
-// staging tile in shared memory; after __syncwarp the warp copies the tile out with
-// whole rows per 8 (fp32) or 4 (16-bit) lanes, so every 16-byte global store covers
-// 4 or 8 full row segments.  `rowdst` is this lane's destination row (nullptr: not
-// stored).  `nf` collects x * 0 over the values: it turns NaN once any is not finite.
-// Every value is multiplied by `osc` (a power of two: the CTA's input scale undone).
+// One half (32 columns) of the 32 rows of one warp -> memory as Tout: `v` holds this
+// lane's row.  Each lane writes its row into a per-warp staging tile in shared memory;
+// after __syncwarp the warp copies the tile out with whole rows per 8 (fp32) or 4 (16-bit)
+// lanes, so every 16-byte global store covers 4 or 8 full row segments.  `rowdst` is this
+// lane's destination row (nullptr: not stored).  `nf` collects x * 0 over the values: it
+// turns NaN once any is not finite.
 template <typename Tout>
-__device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, uint8_t* wstage, int lane,
-                                              float& nf, float osc) {
+__device__ __forceinline__ void stage_store_half(const float (&v)[32], uint8_t* rowdst, uint8_t* wstage, int lane,
+                                                 int half, float& nf) {
   constexpr int kRowB = 32 * (int)sizeof(Tout);  // staged bytes per row and half
   constexpr int kLanesPerRow = kRowB / 16;       // 8 (fp32) or 4 (16-bit)
   constexpr int kRowsPerOp = 32 / kLanesPerRow;
   const unsigned long long myrow = reinterpret_cast<unsigned long long>(rowdst);
+  uint8_t* buf = wstage;  // one 32-row tile, reused by both halves
+  if constexpr (sizeof(Tout) == 4) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      nf = fmaf(v[4 * j], 0.f, nf);
+      nf = fmaf(v[4 * j + 1], 0.f, nf);
+      nf = fmaf(v[4 * j + 2], 0.f, nf);
+      nf = fmaf(v[4 * j + 3], 0.f, nf);
+      *reinterpret_cast<float4*>(buf + stage_chunk<kRowB>(lane, j)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    }
+  } else {
+    __half2 acc = __float2half2_rn(0.f);
+    const __half2 zero = __float2half2_rn(0.f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float x0 = v[8 * j + 2 * u], x1 = v[8 * j + 2 * u + 1];
+        if constexpr (std::is_same<Tout, __half>::value) {
+          pk[u] = pack_h2(x0, x1);
+          acc = __hfma2(bits_h2(pk[u]), zero, acc);
+        } else {
+          __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+          pk[u] = *reinterpret_cast<uint32_t*>(&hb);
+          nf = fmaf(x0, 0.f, nf);
+          nf = fmaf(x1, 0.f, nf);
+        }
+      }
+      *reinterpret_cast<uint4*>(buf + stage_chunk<kRowB>(lane, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    if constexpr (std::is_same<Tout, __half>::value) {
+      const float2 a = __half22float2(acc);
+      nf += a.x + a.y;
+    }
+  }
+  __syncwarp();
+  const int jj = lane % kLanesPerRow;
+#pragma unroll
+  for (int it = 0; it < kLanesPerRow; ++it) {
+    const int R = it * kRowsPerOp + lane / kLanesPerRow;
+    const unsigned long long dr = __shfl_sync(0xffffffffu, myrow, R);
+    const uint4 x = *reinterpret_cast<const uint4*>(buf + stage_chunk<kRowB>(R, jj));
+    if (dr) __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dr) + kRowB * half + 16 * jj), x);
+  }
+  __syncwarp();  // the staging tile is free again
+}
+
+// The 32 rows of one warp (its lanes of a tensor-memory region, 64 fp32 columns) ->
+// memory as Tout, 32 columns at a time, every value multiplied by `osc` (a power of two:
+// the CTA's input scale undone; times 2^-1/2 when d_k = 32).
+template <typename Tout>
+__device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, uint8_t* wstage, int lane,
+                                              float& nf, float osc) {
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     float v[32];
@@ -379,53 +473,48 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, u
     tmem_wait_ld();
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] *= osc;
-    uint8_t* buf = wstage;  // one 32-row tile, reused by both halves
-    if constexpr (sizeof(Tout) == 4) {
+    stage_store_half<Tout>(v, rowdst, wstage, lane, half, nf);
+  }
+}
+
+// The same rows through the GLA output epilogue (0539edu.com appendix E.3.1: RMSNorm and a
+// SiLU-activated output gate fused into the kernel): with o = osc * (tensor memory row
+// [+ the row's partial output olc, fp16, SEGMENTED second phase]),
+//   y_j = o_j / sqrt(mean_i o_i^2 + eps) * nw_j * SiLU(gate_j),
+// the lane's gate row `grow` (Tin, 64 values; nullptr for rows that are not stored).  Two
+// passes over tensor memory: the row's sum of squares, then the values.  Out of line.
+template <typename Tout, typename Tin>
+__device__ __noinline__ void gated_rows(uint32_t taddr, const uint8_t* olc, uint8_t* rowdst, const Tin* grow,
+                                        const float* nw, float eps, uint8_t* wstage, int lane, float& nf, float osc) {
+  float ss = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        nf = fmaf(v[4 * j], 0.f, nf);
-        nf = fmaf(v[4 * j + 1], 0.f, nf);
-        nf = fmaf(v[4 * j + 2], 0.f, nf);
-        nf = fmaf(v[4 * j + 3], 0.f, nf);
-        *reinterpret_cast<float4*>(buf + stage_chunk<kRowB>(lane, j)) =
-            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      }
-    } else {
-      __half2 acc = __float2half2_rn(0.f);
-      const __half2 zero = __float2half2_rn(0.f);
+  for (int half = 0; half < 2; ++half) {
+    float v[32];
+    tmem_ld32(taddr + 32u * half, v);
+    tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float x0 = v[8 * j + 2 * u], x1 = v[8 * j + 2 * u + 1];
-          if constexpr (std::is_same<Tout, __half>::value) {
-            pk[u] = pack_h2(x0, x1);
-            acc = __hfma2(bits_h2(pk[u]), zero, acc);
-          } else {
-            __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-            pk[u] = *reinterpret_cast<uint32_t*>(&hb);
-            nf = fmaf(x0, 0.f, nf);
-            nf = fmaf(x1, 0.f, nf);
-          }
-        }
-        *reinterpret_cast<uint4*>(buf + stage_chunk<kRowB>(lane, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      if constexpr (std::is_same<Tout, __half>::value) {
-        const float2 a = __half22float2(acc);
-        nf += a.x + a.y;
-      }
+    for (int j = 0; j < 32; j += 2) {
+      float2 o = make_float2(0.f, 0.f);
+      if (olc) o = __half22float2(bits_h2(*reinterpret_cast<const uint32_t*>(olc + 2 * (32 * half + j))));
+      const float x0 = (v[j] + o.x) * osc, x1 = (v[j + 1] + o.y) * osc;
+      ss = fmaf(x0, x0, fmaf(x1, x1, ss));
     }
-    __syncwarp();
-    const int jj = lane % kLanesPerRow;
+  }
+  const float rinv = rsqrtf(ss * (1.f / 64.f) + eps);
 #pragma unroll
-    for (int it = 0; it < kLanesPerRow; ++it) {
-      const int R = it * kRowsPerOp + lane / kLanesPerRow;
-      const unsigned long long dr = __shfl_sync(0xffffffffu, myrow, R);
-      const uint4 x = *reinterpret_cast<const uint4*>(buf + stage_chunk<kRowB>(R, jj));
-      if (dr) __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dr) + kRowB * half + 16 * jj), x);
+  for (int half = 0; half < 2; ++half) {
+    float v[32];
+    tmem_ld32(taddr + 32u * half, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      float2 o = make_float2(0.f, 0.f), g = make_float2(0.f, 0.f);
+      if (olc) o = __half22float2(bits_h2(*reinterpret_cast<const uint32_t*>(olc + 2 * (32 * half + j))));
+      if (grow) g = In2<Tin>::unpack(__ldg(reinterpret_cast<const unsigned int*>(grow + 32 * half + j)));
+      v[j] = (v[j] + o.x) * osc * rinv * nw[32 * half + j] * silu_fast(g.x);
+      v[j + 1] = (v[j + 1] + o.y) * osc * rinv * nw[32 * half + j + 1] * silu_fast(g.y);
     }
-    __syncwarp();  // the staging tile is free again
+    stage_store_half<Tout>(v, rowdst, wstage, lane, half, nf);
   }
 }
 
@@ -435,6 +524,51 @@ __device__ __forceinline__ uint8_t* out_row(const FusedParams& fp, int b, int h,
   if (!valid) return nullptr;
   const long long m = ((long long)b * fp.p.L() + scan_token(fp, (uint32_t)s)) * fp.p.heads + h;
   return reinterpret_cast<uint8_t*>(reinterpret_cast<Tout*>(fp.p.out) + m * 64);
+}
+
+// Output-gate row (64 values of the input dtype) of output row s of (b, h), or nullptr.
+template <typename Tin>
+__device__ __forceinline__ const Tin* gate_row(const FusedParams& fp, int b, int h, bool valid, long long s) {
+  if (!valid) return nullptr;
+  const long long m = ((long long)b * fp.p.L() + scan_token(fp, (uint32_t)s)) * fp.p.heads + h;
+  return reinterpret_cast<const Tin*>(fp.p.ogate) + m * 64;
+}
+
+// Low-rank gate producer (GTR digest page, "Core method": gamma = sigmoid(x W1 W2 + b)^(1/tau),
+// rank 16): ln gamma of this thread's rows row0 .. row0+3 and channels 32p + 4cc .. +3
+// (p < d_k / 32) from the chunk's z rows (dense [64][rank] fp32 at zt) and this head's W2
+// columns and bias (shared memory), into lr[p][row][channel].  Out of line.
+template <int kDK>
+__device__ __noinline__ void lowrank_gate_values(const float* zt, const Misc* ms, int rank, float tinv, int row0,
+                                                 int cc, float (*lr)[4][4]) {
+  for (int ps = 0; ps < kDK / 32; ++ps) {
+    const int ch0 = 32 * ps + 4 * cc;
+    const float4 b4 = *reinterpret_cast<const float4*>(ms->bs + ch0);
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = b4.x, acc[i][1] = b4.y, acc[i][2] = b4.z, acc[i][3] = b4.w;
+    for (int j = 0; j < rank; j += 4) {
+      float4 zr[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) zr[i] = *reinterpret_cast<const float4*>(zt + (row0 + i) * rank + j);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const float4 w4 = *reinterpret_cast<const float4*>(&ms->w2s[j + jj][ch0]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float zv = jj == 0 ? zr[i].x : jj == 1 ? zr[i].y : jj == 2 ? zr[i].z : zr[i].w;
+          acc[i][0] = fmaf(zv, w4.x, acc[i][0]);
+          acc[i][1] = fmaf(zv, w4.y, acc[i][1]);
+          acc[i][2] = fmaf(zv, w4.z, acc[i][2]);
+          acc[i][3] = fmaf(zv, w4.w, acc[i][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lr[ps][i][e] = log_sigmoid_fast(acc[i][e]) * tinv;
+  }
 }
 
 // Segmented mode, second phase: the 32 rows of one warp hold the correction Qh' S_start
@@ -518,21 +652,31 @@ __device__ __forceinline__ uint32_t sw_off8(int row, int ch0) {
   return row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
 }
 
+// Byte offset of channels ch0 .. ch0+3 of row `row` in the raw q / k tiles as loaded:
+// 128-byte-swizzled 64-channel rows (d_k = 64), dense 64-byte rows (d_k = 32).
+template <int kDK>
+__device__ __forceinline__ uint32_t raw_off8(int row, int ch0) {
+  return kDK == 64 ? sw_off8(row, ch0) : (uint32_t)(row * 64 + 2 * ch0);
+}
+
 // Largest |x| of the q and k elements a WG_A thread builds (rows row0 .. row0+3, channels
-// 4cc .. 4cc+3 and 32+4cc .. 32+4cc+3) and of the v elements it converts, as bit patterns
-// with the sign dropped (for non-negative fp16 and bf16 values the integer order of the
-// patterns is their numeric order), reduced over the warp.  Out of line: first chunk only.
-__device__ __noinline__ uint3 own_absmax_bits(const uint8_t* sb, int row0, int cc, int wtid) {
+// 32p + 4cc .. 32p + 4cc + 3 for the d_k / 32 passes p; raw tiles at qr / kr) and of the v
+// elements it converts, as bit patterns with the sign dropped (for non-negative fp16 and
+// bf16 values the integer order of the patterns is their numeric order), reduced over the
+// warp.  Out of line: first chunk only.
+template <int kDK>
+__device__ __noinline__ uint3 own_absmax_bits(const uint8_t* qr, const uint8_t* kr, const uint8_t* vt, int row0,
+                                              int cc, int wtid) {
   uint32_t mq = 0, mk = 0, mv = 0;
-  for (int ps = 0; ps < 2; ++ps)
+  for (int ps = 0; ps < kDK / 32; ++ps)
     for (int i = 0; i < 4; ++i) {
-      const uint32_t o = sw_off8(row0 + i, 32 * ps + 4 * cc);
-      const uint2 a = *reinterpret_cast<const uint2*>(sb + o), c = *reinterpret_cast<const uint2*>(sb + kTile + o);
+      const uint32_t o = raw_off8<kDK>(row0 + i, 32 * ps + 4 * cc);
+      const uint2 a = *reinterpret_cast<const uint2*>(qr + o), c = *reinterpret_cast<const uint2*>(kr + o);
       mq = __vmaxu2(__vmaxu2(mq, a.x & 0x7fff7fffu), a.y & 0x7fff7fffu);
       mk = __vmaxu2(__vmaxu2(mk, c.x & 0x7fff7fffu), c.y & 0x7fff7fffu);
     }
   for (int i = wtid; i < kTile / 16; i += kWG) {
-    const uint4 x = *reinterpret_cast<const uint4*>(sb + 2 * kTile + 16 * i);
+    const uint4 x = *reinterpret_cast<const uint4*>(vt + 16 * i);
     mv = __vmaxu2(__vmaxu2(mv, x.x & 0x7fff7fffu), x.y & 0x7fff7fffu);
     mv = __vmaxu2(__vmaxu2(mv, x.z & 0x7fff7fffu), x.w & 0x7fff7fffu);
   }
@@ -544,13 +688,13 @@ __device__ __noinline__ uint3 own_absmax_bits(const uint8_t* sb, int row0, int c
 // The q and k elements a WG_A thread builds, times the CTA's factors sq and sk, in place
 // (exact: powers of two that bring the values up into the normal range).  Out of line:
 // only CTAs whose inputs are tiny run it.
-template <typename Tin>
-__device__ __noinline__ void prescale_own(uint8_t* sb, int row0, int cc, float sq, float sk) {
-  for (int ps = 0; ps < 2; ++ps)
+template <typename Tin, int kDK>
+__device__ __noinline__ void prescale_own(uint8_t* qr, uint8_t* kr, int row0, int cc, float sq, float sk) {
+  for (int ps = 0; ps < kDK / 32; ++ps)
     for (int i = 0; i < 4; ++i) {
-      const uint32_t o = sw_off8(row0 + i, 32 * ps + 4 * cc);
+      const uint32_t o = raw_off8<kDK>(row0 + i, 32 * ps + 4 * cc);
       for (int t = 0; t < 2; ++t) {
-        uint2* p = reinterpret_cast<uint2*>(sb + t * kTile + o);
+        uint2* p = reinterpret_cast<uint2*>((t ? kr : qr) + o);
         const float f = t ? sk : sq;
         uint2 x = *p;
         const float2 a = In2<Tin>::unpack(x.x), c = In2<Tin>::unpack(x.y);
@@ -583,9 +727,14 @@ __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) 
 // tiles and the full A in the gate tile, into the 16 rows of warp w4 of the chunk's score
 // region (16x256b shape: register 4c+q is row r0 + 8(q>>1), column 8c + cq + (q&1)).
 // Out of line: the chunk loops stay small for the instruction cache.
-template <typename Tin, bool kRev>
+// d_k = 64: the raw q and k tiles are the 128-byte-swizzled Q and K tiles; d_k = 32: dense
+// 64-byte rows at `qraw` / `kraw` (the upper half of the gate tile), the gate tile rows 32
+// floats apart.
+template <typename Tin, bool kRev, int kDK>
 __device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G, uint32_t taddr, int w4, int lane,
                                               float ssc) {
+  const uint8_t* qraw = kDK == 64 ? sb : reinterpret_cast<const uint8_t*>(G) + kRawQ;
+  const uint8_t* kraw = kDK == 64 ? sb + kTile : reinterpret_cast<const uint8_t*>(G) + kRawK;
   const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
   for (int ps = 0; ps < 2; ++ps) {
     float sv[16];
@@ -594,14 +743,16 @@ __device__ __noinline__ void cuda_core_scores(const uint8_t* sb, const float* G,
       const int j = 32 * ps + 8 * (x >> 2) + cq + (x & 1);
       float acc = 0.f;
       if (kRev ? j >= i : j <= i) {  // scan(j) <= scan(i)
-        for (int k = 0; k < 64; k += 2) {
-          const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + sw128_offset(i, k)));
-          const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(sb + kTile + sw128_offset(j, k)));
-          acc = fmaf(qv.x * kv.x, ex2(G[i * 64 + k] - G[j * 64 + k]), acc);
-          acc = fmaf(qv.y * kv.y, ex2(G[i * 64 + k + 1] - G[j * 64 + k + 1]), acc);
+        for (int k = 0; k < kDK; k += 2) {
+          const uint32_t oi = kDK == 64 ? sw128_offset(i, k) : (uint32_t)(i * 64 + 2 * k);
+          const uint32_t oj = kDK == 64 ? sw128_offset(j, k) : (uint32_t)(j * 64 + 2 * k);
+          const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(qraw + oi));
+          const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(kraw + oj));
+          acc = fmaf(qv.x * kv.x, ex2(G[i * kDK + k] - G[j * kDK + k]), acc);
+          acc = fmaf(qv.y * kv.y, ex2(G[i * kDK + k + 1] - G[j * kDK + k + 1]), acc);
         }
       }
-      sv[x] = acc * ssc;  // d_k^-1/2 times the CTA's q and k scale factors
+      sv[x] = acc * ssc;  // the power of two that Kh carries (1/8, or 1/4 when d_k = 32)
     }
     tmem_st16x256_x4(taddr + 32u * ps, sv);
   }
@@ -617,7 +768,7 @@ __device__ __forceinline__ void p2_load(const FusedParams& fp, Misc* ms, uint8_t
   bulk_load(sbuf + kP2Olc, fp.olc + t0, (uint32_t)(nb * kTile), &ms->p2_full[q]);
 }
 
-template <typename Tout>
+template <typename Tin, typename Tout, int kDK, bool kBlock>
 __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
                                                   uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
                                                   Span sp, int& slot, float& nf) {
@@ -636,7 +787,7 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
     if (wtid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < kDK / 16; ++k)
         mma_f16(dq, sw128_desc(a0 + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_128, k > 0);
       mma_commit(&ms->p2_mma[q]);
     }
@@ -646,8 +797,14 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
     const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
     const uint8_t* olc_rows = sbuf + kP2Olc + (wq >> 1) * kTile + 32 * (wq & 1) * 128;
     // fp32 staging over the pair's Qh' (its MMA has completed)
-    epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp, b, h, ci < cnt && s < L, s),
-                            olc_rows, sbuf + wq * 4096, lane, nf, ms->sc_out);
+    const bool valid = ci < cnt && s < L;
+    if (kBlock && fp.gated)
+      gated_rows<Tout, Tin>(dq + ((uint32_t)(32 * wq) << 16), olc_rows + lane * 128, out_row<Tout>(fp, b, h, valid, s),
+                            gate_row<Tin>(fp, b, h, valid, s), ms->nw, fp.p.oeps, sbuf + wq * 4096, lane, nf,
+                            ms->sc_out);
+    else
+      epilogue_rows_add<Tout>(dq + ((uint32_t)(32 * wq) << 16), out_row<Tout>(fp, b, h, valid, s), olc_rows,
+                              sbuf + wq * 4096, lane, nf, ms->sc_out);
     tc_fence_before();
     fence_proxy_async_smem();  // generic accesses of the buffer before the next pair's copies
     wg_sync(q);
@@ -658,32 +815,41 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
 // launches: fp16 outputs inline, bf16 outputs as the compiler decides, fp32 outputs (twice
 // the staging traffic and registers) as a call, which keeps the kernel's own register
 // allocation from spilling.
-template <typename Tout>
+template <typename Tin, typename Tout, int kDK, bool kBlock>
 __device__ __noinline__ void second_phase_call(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
                                                uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
                                                Span sp, int& slot, float& nf) {
-  second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+  second_phase_body<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
 }
-template <typename Tout>
+template <typename Tin, typename Tout, int kDK, bool kBlock>
 __device__ void second_phase_auto(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem, uint32_t tmem,
                                   int q, int wtid, int lane, int seq, int b, int h, Span sp, int& slot, float& nf) {
-  second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+  second_phase_body<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
 }
-template <typename Tout>
+template <typename Tin, typename Tout, int kDK, bool kBlock>
 __device__ __forceinline__ void second_phase(const FusedParams& fp, Misc* ms, WsHeader* hdr, uint8_t* smem,
                                              uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h, Span sp,
                                              int& slot, float& nf) {
   if constexpr (sizeof(Tout) == 4)
-    second_phase_call<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+    second_phase_call<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
   else if constexpr (std::is_same<Tout, __half>::value)
-    second_phase_body<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+    second_phase_body<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
   else
-    second_phase_auto<Tout>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
+    second_phase_auto<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, wtid, lane, seq, b, h, sp, slot, nf);
 }
 
-template <typename Tin, typename Tout, bool kRev, bool kBox, int kMode>
+// kBlock: the kernel also carries the optional pieces of the GTR block (low-rank gate
+// producer, RMSNorm + SiLU output gate), switched on at run time by fp.lowrank / fp.gated;
+// the kernels without them keep none of their code.
+template <typename Tin, typename Tout, bool kRev, bool kBox, int kMode, int kDK, bool kBlock>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_gla_kernel(const __grid_constant__ FusedParams fp) {
+  const bool lowrank = kBlock && fp.lowrank != 0;
+  const bool gated = kBlock && fp.gated != 0;
+  static_assert(kDK == 64 || kDK == 32, "key widths 64 and 32");
+  // the power of two of d_k^-1/2 that Kh carries; d_k = 32 applies the remaining 2^-1/2 to
+  // the outputs (sc_out)
+  constexpr float kKf = kDK == 64 ? 0.125f : 0.25f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Misc* ms = reinterpret_cast<Misc*>(smem + kOffMisc);
@@ -779,7 +945,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = n % kStages;
           if (!stage_free(n, st)) break;
           uint8_t* sb = smem + kOffStage + st * kStageBytes;
-          mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);
+          uint8_t* qd = kDK == 64 ? sb : sb + 3 * kTile + kRawQ;  // raw q and k (d_k = 32: dense, in the gate tile)
+          uint8_t* kd = kDK == 64 ? sb + kTile : sb + 3 * kTile + kRawK;
+          mbar_arrive_expect_tx(&ms->full[st], chunk_load_bytes<kDK>(fp, lowrank));
           const long long s0 = (long long)c * kChunk;
           if (p.direction <= GTR_R2L) {
             // row view: 64 consecutive grid cells m (right-to-left: one image row)
@@ -788,19 +956,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               const long long y = s0 / p.W;
               m0 = y * p.W + (p.W - 64 - (s0 - y * p.W));
             }
-            tma_load_4d(sb, &fp.tq, &ms->full[st], 0, h, (int)m0, b);
-            tma_load_4d(sb + kTile, &fp.tk, &ms->full[st], 0, h, (int)m0, b);
+            tma_load_4d(qd, &fp.tq, &ms->full[st], 0, h, (int)m0, b);
+            tma_load_4d(kd, &fp.tk, &ms->full[st], 0, h, (int)m0, b);
             tma_load_4d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, (int)m0, b);
-            tma_load_4d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, (int)m0, b);
+            if (lowrank)  // the token's z row (per-token tensor: heads coordinate 0)
+              tma_load_4d(sb + 3 * kTile, &fp.tz, &ms->full[st], 0, 0, (int)m0, b);
+            else
+              tma_load_4d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, (int)m0, b);
           } else {
             // column view: 64 consecutive y of one column x
             const int x = (int)(s0 / p.H);
             int y0 = (int)(s0 - (long long)x * p.H);
             if (p.direction == GTR_B2T) y0 = p.H - 64 - y0;
-            tma_load_5d(sb, &fp.tq, &ms->full[st], 0, h, x, y0, b);
-            tma_load_5d(sb + kTile, &fp.tk, &ms->full[st], 0, h, x, y0, b);
+            tma_load_5d(qd, &fp.tq, &ms->full[st], 0, h, x, y0, b);
+            tma_load_5d(kd, &fp.tk, &ms->full[st], 0, h, x, y0, b);
             tma_load_5d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, x, y0, b);
-            tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, x, y0, b);
+            if (lowrank)
+              tma_load_5d(sb + 3 * kTile, &fp.tz, &ms->full[st], 0, 0, x, y0, b);
+            else
+              tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, x, y0, b);
           }
         }
       }
@@ -815,7 +989,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rbase = (int)((long long)b * L * p.heads + h);
       const int t = lane >> 3, g0 = 2 * (lane & 7);
       const void* tmap = t == 0 ? (const void*)&fp.tq : t == 1 ? (const void*)&fp.tk
-                                                               : t == 2 ? (const void*)&fp.tv : (const void*)&fp.tg;
+                         : t == 2 ? (const void*)&fp.tv : lowrank ? (const void*)&fp.tz : (const void*)&fp.tg;
+      // low-rank gate producer: z rows of a per-token [B*L][rank] view
+      const int zoob = (int)((long long)p.B * L), zbase = (int)((long long)b * L);
       for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
         const int st = n % kStages;
         int* rows = ms->rowoff[n & 1];
@@ -823,22 +999,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hlf = 0; hlf < 2; ++hlf) {
           const int pt = lane + 32 * hlf;
           const long long s = (long long)c * kChunk + pt;
-          rows[kRev ? 63 - pt : pt] = s < L ? rbase + (int)scan_token(fp, (uint32_t)s) * p.heads : oob;
+          const int tok = s < L ? (int)scan_token(fp, (uint32_t)s) : -1;
+          rows[kRev ? 63 - pt : pt] = tok >= 0 ? rbase + tok * p.heads : oob;
+          ms->zrow[n & 1][kRev ? 63 - pt : pt] = tok >= 0 ? zbase + tok : zoob;
         }
         int ok = 0;
         if (lane == 0) {
           ok = stage_free(n, st) ? 1 : 0;
-          if (ok) mbar_arrive_expect_tx(&ms->full[st], (uint32_t)kStageBytes);  // the arrival comes first
+          if (ok) mbar_arrive_expect_tx(&ms->full[st], chunk_load_bytes<kDK>(fp, lowrank));  // the arrival comes first
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         __syncwarp();  // (the row table is complete)
         uint8_t* sb = smem + kOffStage + st * kStageBytes;
-        uint8_t* tile = t < 3 ? sb + t * kTile : sb + 3 * kTile;
-        const int rowb = t < 3 ? 128 : 256;
+        // q, k: 64-channel swizzled tiles, or (d_k = 32) dense 64-byte rows in the gate tile
+        uint8_t* tile = t == 2 ? sb + 2 * kTile
+                        : t == 3 ? sb + 3 * kTile
+                        : kDK == 64 ? sb + t * kTile : sb + 3 * kTile + (t == 0 ? kRawQ : kRawK);
+        const bool zt = t == 3 && lowrank;
+        const int rowb = t == 2 ? 128 : t == 3 ? (zt ? 4 * p.grank : 4 * kDK) : 2 * kDK;
+        const int* rr = zt ? ms->zrow[n & 1] : rows;
 #pragma unroll
         for (int gi = g0; gi < g0 + 2; ++gi)
-          tma_gather4(tile + gi * 4 * rowb, tmap, &ms->full[st], 0, rows[4 * gi], rows[4 * gi + 1], rows[4 * gi + 2],
-                      rows[4 * gi + 3]);
+          tma_gather4(tile + gi * 4 * rowb, tmap, &ms->full[st], 0, rr[4 * gi], rr[4 * gi + 1], rr[4 * gi + 2],
+                      rr[4 * gi + 3]);
       }
     } else {
       // Per chunk, lane t first resolves the grid cells of scan positions c*64 + t and
@@ -867,24 +1050,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ok = stage_free(n, st) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // (the row table is complete, too)
         const uint32_t sb = smem_u32(smem + kOffStage + st * kStageBytes);
+        if constexpr (kDK == 64) {
 #pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-          const int row = 4 * it + rq;
-          const int cell = rows[row];
-          const uint32_t nb = cell >= 0 ? 16u : 0u;
-          const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
-          const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
-          cp_async16(dst, gq + src, nb);
-          cp_async16(dst + kTile, gk + src, nb);
-          cp_async16(dst + 2 * kTile, gv + src, nb);
+          for (int it = 0; it < 16; ++it) {
+            const int row = 4 * it + rq;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
+            const uint32_t dst = sb + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4);
+            cp_async16(dst, gq + src, nb);
+            cp_async16(dst + kTile, gk + src, nb);
+            cp_async16(dst + 2 * kTile, gv + src, nb);
+          }
+#pragma unroll 4
+          for (int it = 0; it < 32 && !lowrank; ++it) {
+            const int row = 2 * it + rg;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
+                       gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
+          }
+        } else {
+          // d_k = 32: q and k 64-byte rows (groups of 4 lanes) dense into the gate tile's
+          // upper half; v 128-byte rows (swizzled) and gate 128-byte rows per group of 8
+          const int j4 = lane & 3, r8 = lane >> 2;
+#pragma unroll 4
+          for (int it = 0; it < 8; ++it) {
+            const int row = 8 * it + r8;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 64 + 16 * j4;
+            cp_async16(sb + 3 * kTile + kRawQ + row * 64 + 16 * j4, gq + src, nb);
+            cp_async16(sb + 3 * kTile + kRawK + row * 64 + 16 * j4, gk + src, nb);
+          }
+#pragma unroll 4
+          for (int it = 0; it < 16; ++it) {
+            const int row = 4 * it + rq;
+            const int cell = rows[row];
+            const uint32_t nb = cell >= 0 ? 16u : 0u;
+            const long long src = ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 128 + 16 * j8;
+            cp_async16(sb + 2 * kTile + row * 128 + (uint32_t)((j8 ^ (row & 7)) << 4), gv + src, nb);
+            if (!lowrank) cp_async16(sb + 3 * kTile + row * 128 + 16 * j8, gg + src, nb);
+          }
         }
-#pragma unroll 4
-        for (int it = 0; it < 32; ++it) {
-          const int row = 2 * it + rg;
-          const int cell = rows[row];
-          const uint32_t nb = cell >= 0 ? 16u : 0u;
-          cp_async16(sb + 3 * kTile + row * 256 + 16 * j16,
-                     gg + ((long long)(cell >= 0 ? cell : 0) * p.heads + h) * 256 + 16 * j16, nb);
+        if (lowrank) {
+          // z rows (rank / 4 pieces of 16 bytes a row) dense at the start of the gate tile
+          const int P = p.grank / 4;
+          const uint8_t* gz = reinterpret_cast<const uint8_t*>(p.gz);
+          for (int idx = lane; idx < 64 * P; idx += 32) {
+            const int row = idx / P, pc = idx - row * P;
+            const int cell = rows[row];
+            cp_async16(sb + 3 * kTile + row * 16 * P + 16 * pc,
+                       gz + (long long)(cell >= 0 ? cell : 0) * 16 * P + 16 * pc, cell >= 0 ? 16u : 0u);
+          }
         }
         cp_async_arrive_noinc(&ms->full[st]);
       }
@@ -952,8 +1170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_v = a_q + 2 * kTile;
         tc_fence_after();
         const uint32_t su = tmem + kColSU + 64u * (uint32_t)(n % kSU);
-        if (!*(volatile int*)&ms->fb[st]) {
-          for (int k = 0; k < 4; ++k)
+        if (!*(volatile int*)&ms->fb[st]) {  // (K = d_k: channels past d_k are zero)
+          for (int k = 0; k < kDK / 16; ++k)
             mma_f16(su, sw128_desc(a_q + 32 * k), sw128_desc(a_k + 32 * k), id_qk, k > 0);
         }
         for (int k = 0; k < 4; ++k)
@@ -987,7 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
         const uint32_t a_s = s_base + kOffS + (m % kNS) * kTile;
         tc_fence_after();
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < kDK / 16; ++k)
           mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
         if (!wait_spin(&ms->pready[su], ph_use<kSU>(m), ms, hdr, 0x204)) break;
         // P sits in the lane tile of the chunk's output (A and D rows share lanes)
@@ -1008,8 +1226,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // ===================================================================== WG_A: operand tiles
     // The two warpgroups take alternate chunks (warpgroup hh: chunks n = hh, hh+2, ...),
-    // each in two passes over the key-channel halves: its warp w4 takes rows 16w4 ..
-    // 16w4+15, a thread 4 rows x 4 channels per pass.
+    // each in d_k / 32 passes over the key channels (two halves when d_k = 64): its warp w4
+    // takes rows 16w4 .. 16w4+15, a thread 4 rows x 4 channels per pass.  d_k = 32: the
+    // raw q and k sit in the upper half of the gate tile and Qh, Kh are built into the Q
+    // and K tiles with channels 32 .. 63 zero.
+    constexpr int kPasses = kDK / 32;
     const int hh = warp >> 2, w4 = warp & 3;
     const int wg = hh, wtid = tid - kWG * hh;
     const int cc = lane & 7;                     // channels 32p + 4cc .. 32p + 4cc + 3 in pass p
@@ -1018,6 +1239,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     int slot = 0;
     bool alive = true;
     float sq = 1.f, sk = 1.f, sv = 1.f;  // this CTA's input scale factors (set at the first chunk)
+    if (hh == 0 && (lowrank || gated)) {
+      // warpgroup 0: this head's gate-producer columns and bias (zero past d_k) and the output
+      // norm weight into shared memory; the other roles read them after the scale barrier
+      // (warpgroup 1, WG_B, WG_C) or a CTA barrier
+      if (lowrank) {
+        const int ld = p.heads * kDK;
+        for (int i = wtid; i < 16 * 64; i += kWG) {
+          const int j = i >> 6, c = i & 63;
+          ms->w2s[j][c] = (j < p.grank && c < kDK) ? __ldg(p.gw2 + (long long)j * ld + h * kDK + c) : 0.f;
+        }
+        if (wtid < 64) ms->bs[wtid] = wtid < kDK ? __ldg(p.gb + h * kDK + wtid) : 0.f;
+      }
+      if (gated && wtid < 64) ms->nw[wtid] = __ldg(p.onorm_w + wtid);
+      wg_sync(wg);
+    }
     for (int n = hh; n < cnt; n += 2) {
       const int st = n % kStages;
       if (!wg_wait(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
@@ -1026,10 +1262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint8_t* sb = smem + kOffStage + st * kStageBytes;
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
+      uint8_t* qr = kDK == 64 ? sb : sb + 3 * kTile + kRawQ;  // raw q, k
+      uint8_t* kr = kDK == 64 ? sb + kTile : sb + 3 * kTile + kRawK;
       if (n == 0) {
         // ---- the CTA's input scale comes from its first chunk (warpgroup 0): the warps'
         // largest |q|, |k|, |v| travel with the cumsum exchange below
-        const uint3 m = own_absmax_bits(sb, row0, cc, wtid);
+        const uint3 m = own_absmax_bits<kDK>(qr, kr, sb + 2 * kTile, row0, cc, wtid);
         if (lane == 0) ms->smax[w4][0] = m.x, ms->smax[w4][1] = m.y, ms->smax[w4][2] = m.z;
       } else if (n == 1) {  // warpgroup 1's first chunk: take the scale warpgroup 0 set
         if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot)) {
@@ -1045,14 +1283,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp's 4 row blocks, then over the 4 warps through shared memory (staged rows run
       // backwards in scan order when the chunk is reversed)
       float run[2][4], incl[2][4];
+      float lr[2][4][4];  // low-rank producer: this thread's ln gamma values
+      if (lowrank) {
+        // the gates come from the chunk's z rows (where the gate tile starts); every thread
+        // has read its z rows before any thread writes the gate tile
+        lowrank_gate_values<kDK>(G, ms, p.grank, fp.gtau_inv, row0, cc, lr);
+        wg_sync(wg);
+      }
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
+      for (int ps = 0; ps < kPasses; ++ps) {
         const int ch0 = 32 * ps + 4 * cc;
         float gv[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * 64 + ch0);
-          gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
+          if (lowrank) {
+            gv[i][0] = lr[ps][i][0]; gv[i][1] = lr[ps][i][1]; gv[i][2] = lr[ps][i][2]; gv[i][3] = lr[ps][i][3];
+          } else {
+            const float4 g4 = *reinterpret_cast<const float4*>(G + (row0 + i) * kDK + ch0);
+            gv[i][0] = g4.x; gv[i][1] = g4.y; gv[i][2] = g4.z; gv[i][3] = g4.w;
+          }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) run[ps][e] = 0.f;
@@ -1067,7 +1316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<float4*>(G + (row0 + i) * 64 + ch0) = make_float4(gv[i][0], gv[i][1], gv[i][2], gv[i][3]);
+          *reinterpret_cast<float4*>(G + (row0 + i) * kDK + ch0) = make_float4(gv[i][0], gv[i][1], gv[i][2], gv[i][3]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float v = run[ps][e];
@@ -1105,7 +1354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ms->sc_in[0] = sq;
           ms->sc_in[1] = sk;
           ms->sc_in[2] = sv;
-          ms->sc_out = pow2f(-(e[0] + e[1] + e[2]));
+          ms->sc_out = pow2f(-(e[0] + e[1] + e[2])) * (kDK == 64 ? 1.f : 0.70710678118654752f);
           ms->sc_spub = pow2f(-(e[1] + e[2]));
           ms->sc_sin = pow2f(e[1] + e[2]);
           mbar_arrive(&ms->scale_ready);
@@ -1113,12 +1362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // a CTA with tiny inputs first scales the q and k elements this thread builds (the
       // CUDA-core scores below read them after a barrier)
-      if (sq != 1.f || sk != 1.f) prescale_own<Tin>(sb, row0, cc, sq, sk);
+      if (sq != 1.f || sk != 1.f) prescale_own<Tin, kDK>(qr, kr, row0, cc, sq, sk);
       // offsets of my rows (the rows of earlier lanes and warps) and the chunk decay a
       float off[2][4], last[2][4];
       bool exp_unsafe = false;
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
+      for (int ps = 0; ps < kPasses; ++ps) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           off[ps][e] = incl[ps][e] - run[ps][e];
@@ -1138,7 +1387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e)
           if (-last[ps][e] > fp.max_exp2) exp_unsafe = true;
       }
-      // CUDA-core decision: the lanes of every warp hold the decays of all 64 channels
+      // CUDA-core decision: the lanes of every warp hold the decays of all d_k channels
       const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
       if (fbx) {
         // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
@@ -1146,29 +1395,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The full A goes to the gate tile so that every thread can read every row and
         // channel.
 #pragma unroll
-        for (int ps = 0; ps < 2; ++ps)
+        for (int ps = 0; ps < kPasses; ++ps)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float4* gp = reinterpret_cast<float4*>(G + (row0 + i) * 64 + 32 * ps + 4 * cc);
+            float4* gp = reinterpret_cast<float4*>(G + (row0 + i) * kDK + 32 * ps + 4 * cc);
             const float4 a4 = *gp;
             *gp = make_float4(a4.x + off[ps][0], a4.y + off[ps][1], a4.z + off[ps][2], a4.w + off[ps][3]);
           }
         if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) { alive = false; break; }
         tc_fence_after();  // (the wait's barrier also publishes the full A)
-        cuda_core_scores<Tin, rev>(sb, G, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU), w4,
-                                   lane, 0.125f);
+        cuda_core_scores<Tin, rev, kDK>(sb, G, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU),
+                                        w4, lane, kKf);
         tmem_wait_st();
         tc_fence_before();
         wg_sync(wg);  // raw q / k reads done before the overwrite
 #pragma unroll
-        for (int ps = 0; ps < 2; ++ps)
+        for (int ps = 0; ps < kPasses; ++ps)
 #pragma unroll
           for (int e = 0; e < 4; ++e) off[ps][e] = 0.f;  // the gate tile holds the full A now
       }
-      // ---- Qh = q 2^A, Kh = k 2^-A / 8 (k 2^(a-A) / 8 for CUDA-core chunks), in place
-      const __half2 eighth = __float2half2_rn(0.125f);
+      // ---- Qh = q 2^A, Kh = k 2^-A kKf (k 2^(a-A) kKf for CUDA-core chunks), kKf = 1/8
+      // (d_k = 64: in place) or 1/4 (d_k = 32, the remaining 2^-1/2 of d_k^-1/2 is applied
+      // to the outputs)
+      const __half2 kfh = __float2half2_rn(kKf);
 #pragma unroll 1
-      for (int ps = 0; ps < 2; ++ps) {  // (rolled: the loop body stays small for the instruction cache)
+      for (int ps = 0; ps < kPasses; ++ps) {  // (rolled: the loop body stays small for the instruction cache)
         const int ch0 = 32 * ps + 4 * cc;
         float offp[4], lastp[4];
 #pragma unroll
@@ -1179,13 +1430,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int row = row0 + i;
-          const float4 a4 = *reinterpret_cast<const float4*>(G + row * 64 + ch0);
+          const float4 a4 = *reinterpret_cast<const float4*>(G + row * kDK + ch0);
           const float Ar[4] = {a4.x + offp[0], a4.y + offp[1], a4.z + offp[2], a4.w + offp[3]};
           // channels ch0 .. ch0+3: 8 bytes at 16-byte chunk ch0/8, half (ch0/4) & 1
-          const uint32_t off8 =
-              row * 128u + ((((uint32_t)ch0 >> 3) ^ ((uint32_t)row & 7u)) << 4) + ((ch0 >> 2) & 1) * 8;
-          uint2 qraw = *reinterpret_cast<const uint2*>(sb + off8);
-          uint2 kraw = *reinterpret_cast<const uint2*>(sb + kTile + off8);
+          const uint32_t off8 = sw_off8(row, ch0);
+          const uint32_t roff = raw_off8<kDK>(row, ch0);
+          uint2 qraw = *reinterpret_cast<const uint2*>(qr + roff);
+          uint2 kraw = *reinterpret_cast<const uint2*>(kr + roff);
           uint32_t* qw = reinterpret_cast<uint32_t*>(&qraw);
           uint32_t* kw = reinterpret_cast<uint32_t*>(&kraw);
 #pragma unroll
@@ -1196,17 +1447,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             __half2 qh, kh;
             if constexpr (std::is_same<Tin, __half>::value) {
               qh = __hmul2(bits_h2(qw[e2]), bits_h2(pack_h2(ex2(A0), ex2(A1))));
-              kh = __hmul2(__hmul2(bits_h2(kw[e2]), eighth), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
+              kh = __hmul2(__hmul2(bits_h2(kw[e2]), kfh), bits_h2(pack_h2(ex2(xk0), ex2(xk1))));
             } else {
               const float2 qv = In2<Tin>::unpack(qw[e2]), kv = In2<Tin>::unpack(kw[e2]);
               qh = __floats2half2_rn(qv.x * ex2(A0), qv.y * ex2(A1));
-              kh = __floats2half2_rn(kv.x * 0.125f * ex2(xk0), kv.y * 0.125f * ex2(xk1));
+              kh = __floats2half2_rn(kv.x * kKf * ex2(xk0), kv.y * kKf * ex2(xk1));
             }
             qw[e2] = h2_bits(qh);
             kw[e2] = h2_bits(kh);
           }
           *reinterpret_cast<uint2*>(sb + off8) = qraw;
           *reinterpret_cast<uint2*>(sb + kTile + off8) = kraw;
+          if constexpr (kDK == 32) {  // channels 32 .. 63 of Qh and Kh are zero
+            const uint32_t offz = sw_off8(row, 32 + ch0);
+            *reinterpret_cast<uint2*>(sb + offz) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2*>(sb + kTile + offz) = make_uint2(0u, 0u);
+          }
         }
       }
       if (!std::is_same<Tin, __half>::value || sv != 1.f) {
@@ -1226,11 +1482,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (w4 == 0 && lane < 8) {
-        // gate row 0 (read by this thread only, above) now holds the chunk's decay a per
-        // channel
+        // the first 64 floats of the gate tile (rows read by these lanes only, above) now
+        // hold the chunk's decay a per key channel (0 for channels d_k .. 63)
 #pragma unroll
         for (int ps = 0; ps < 2; ++ps)
-          *reinterpret_cast<float4*>(G + 32 * ps + 4 * cc) = make_float4(last[ps][0], last[ps][1], last[ps][2], last[ps][3]);
+          *reinterpret_cast<float4*>(G + 32 * ps + 4 * cc) =
+              ps < kPasses ? make_float4(last[ps][0], last[ps][1], last[ps][2], last[ps][3])
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (wtid == 0) ms->fb[st] = fbx ? 1 : 0;
       fence_proxy_async_smem();
@@ -1423,6 +1681,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp.c0 + ci) * 4096) + trow * 128
                               : nullptr;
           epilogue_rows<__half>(src, od, wstage, lane, nonfinite, 1.f);  // (kept in this CTA's scale)
+        } else if (gated) {
+          gated_rows<Tout, Tin>(src, nullptr, out_row<Tout>(fp, b, h, valid, s), gate_row<Tin>(fp, b, h, valid, s),
+                                ms->nw, fp.p.oeps, wstage, lane, nonfinite, osc);
         } else {
           epilogue_rows<Tout>(src, out_row<Tout>(fp, b, h, valid, s), wstage, lane, nonfinite, osc);
         }
@@ -1498,7 +1759,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (go) {
         const int q = warp >> 2;
         int slot2 = 0;
-        second_phase<Tout>(fp, ms, hdr, smem, tmem, q, tid - kWG * q, lane, seq, b, h, sp, slot2, nonfinite);
+        second_phase<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, tid - kWG * q, lane, seq, b, h, sp, slot2,
+                                             nonfinite);
       }
     }
   }
@@ -1597,7 +1859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < cnt; ++g) {
           const uint32_t d_o = tmem + kColO + 64u * (uint32_t)(g >> 1) + ((g & 1) ? kLaneTile1 : 0u);
           const uint32_t a_q = s_base + kOffStage + g * (inplace ? kStageBytes : kTile);  // the chunk's Qh'
-          for (int k = 0; k < 4; ++k)
+          for (int k = 0; k < kDK / 16; ++k)
             mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(s_base + kOffSst + 2048 * k), id_qs, 1);
           if ((g & 1) || g + 1 == cnt) mma_commit(&ms->corr_done[g >> 1]);
         }
@@ -1607,8 +1869,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int ci = 2 * pr + tsel;
         const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
-        epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(fp, b, h, ci < cnt && s < L, s), wstage,
-                            lane, nonfinite, ms->sc_out);
+        const bool valid = ci < cnt && s < L;
+        if (gated)
+          gated_rows<Tout, Tin>(tl + kColO + 64u * (uint32_t)pr, nullptr, out_row<Tout>(fp, b, h, valid, s),
+                                gate_row<Tin>(fp, b, h, valid, s), ms->nw, fp.p.oeps, wstage, lane, nonfinite,
+                                ms->sc_out);
+        else
+          epilogue_rows<Tout>(tl + kColO + 64u * (uint32_t)pr, out_row<Tout>(fp, b, h, valid, s), wstage, lane,
+                              nonfinite, ms->sc_out);
       }
     }
   }
@@ -1646,43 +1914,44 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// Tensor map over a [B][H][W][heads][64] tensor (row-major grid cells m = y*W + x) whose
-// box is 64 consecutive scan positions of one (batch, head): the row view [B][L][heads][64]
-// with a box of 64 cells m, or the column view with a box of 64 rows y of one column x.
+// Tensor map over a [B][H][W][nh][d] tensor (row-major grid cells m = y*W + x) whose box
+// is 64 consecutive scan positions of one (batch, head): the row view [B][L][nh][d] with a
+// box of 64 cells m, or the column view with a box of 64 rows y of one column x.  nh is the
+// heads dimension (1 for a per-token tensor), d the channels (d * esize a multiple of 16).
 bool make_chunk_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, const Problem& p,
-                    bool column, bool swizzle) {
+                    bool column, bool swizzle, int d, int nh) {
   auto enc = get_encode();
   if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
-  const cuuint64_t e = (cuuint64_t)esize, hd = (cuuint64_t)p.heads;
+  const cuuint64_t e = (cuuint64_t)esize, hd = (cuuint64_t)nh, dd = (cuuint64_t)d;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle sw = swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r;
   if (!column) {
-    cuuint64_t dims[4] = {64, hd, (cuuint64_t)p.L(), (cuuint64_t)p.B};
-    cuuint64_t strides[3] = {64 * e, hd * 64 * e, (cuuint64_t)p.L() * hd * 64 * e};
-    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint64_t dims[4] = {dd, hd, (cuuint64_t)p.L(), (cuuint64_t)p.B};
+    cuuint64_t strides[3] = {dd * e, hd * dd * e, (cuuint64_t)p.L() * hd * dd * e};
+    cuuint32_t box[4] = {(cuuint32_t)d, 1, 64, 1};
     r = enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
-    cuuint64_t dims[5] = {64, hd, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)p.B};
-    cuuint64_t strides[4] = {64 * e, hd * 64 * e, (cuuint64_t)p.W * hd * 64 * e,
-                             (cuuint64_t)p.H * p.W * hd * 64 * e};
-    cuuint32_t box[5] = {64, 1, 1, 64, 1};
+    cuuint64_t dims[5] = {dd, hd, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)p.B};
+    cuuint64_t strides[4] = {dd * e, hd * dd * e, (cuuint64_t)p.W * hd * dd * e,
+                             (cuuint64_t)p.H * p.W * hd * dd * e};
+    cuuint32_t box[5] = {(cuuint32_t)d, 1, 1, 64, 1};
     r = enc(m, dt, 5, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   }
   return r == CUDA_SUCCESS;
 }
 
-// Tensor map over a [rows][64] view (one token-head a row) whose box is one row: the
-// source of 4-row TMA gathers.
+// Tensor map over a [rows][d] view (one token-head a row) whose box is one row: the source
+// of 4-row TMA gathers.
 bool make_row_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, long long rows,
-                  bool swizzle) {
+                  bool swizzle, int d) {
   auto enc = get_encode();
   if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) || rows >= (1ll << 31)) return false;
-  cuuint64_t dims[2] = {64, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(64 * esize)};
-  cuuint32_t box[2] = {64, 1};
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * esize};
+  cuuint32_t box[2] = {(cuuint32_t)d, 1};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1771,13 +2040,15 @@ int max_active_clusters(K kern, int dev, int kind, int cs) {
   return c;
 }
 
-template <typename Tin, typename Tout, int kMode>
+template <typename Tin, typename Tout, int kMode, int kDK, bool kBlock = false>
 void (*pick_kernel(bool rev, bool box))(FusedParams) {
-  return rev ? (box ? fused_gla_kernel<Tin, Tout, true, true, kMode> : fused_gla_kernel<Tin, Tout, true, false, kMode>)
-             : (box ? fused_gla_kernel<Tin, Tout, false, true, kMode> : fused_gla_kernel<Tin, Tout, false, false, kMode>);
+  return rev ? (box ? fused_gla_kernel<Tin, Tout, true, true, kMode, kDK, kBlock>
+                    : fused_gla_kernel<Tin, Tout, true, false, kMode, kDK, kBlock>)
+             : (box ? fused_gla_kernel<Tin, Tout, false, true, kMode, kDK, kBlock>
+                    : fused_gla_kernel<Tin, Tout, false, false, kMode, kDK, kBlock>);
 }
 
-template <typename Tin, typename Tout>
+template <typename Tin, typename Tout, int kDK>
 gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream, int force_mode) {
   const bool rev = p.direction == GTR_R2L || p.direction == GTR_B2T;
   FusedParams fp;
@@ -1792,19 +2063,29 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
                        (column && p.H % 64 == 0);
   const CUtensorMapDataType dt16 =
       std::is_same<Tin, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  fp.tma = one_box && make_chunk_map(&fp.tq, p.q, dt16, 2, p, column, true) &&
-                   make_chunk_map(&fp.tk, p.k, dt16, 2, p, column, true) &&
-                   make_chunk_map(&fp.tv, p.v, dt16, 2, p, column, true) &&
-                   make_chunk_map(&fp.tg, p.log_gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, column, false)
+  // optional pieces of the GTR block: the low-rank gate producer (z tiles instead of the
+  // log-gates) and the RMSNorm + SiLU output gate
+  fp.lowrank = p.gz != nullptr ? 1 : 0;
+  fp.gtau_inv = fp.lowrank ? 1.f / p.gtau : 1.f;
+  fp.gated = p.ogate != nullptr ? 1 : 0;
+  // q, k: 128-byte swizzle (d_k = 64; built in place), or dense rows (d_k = 32)
+  const bool swqk = kDK == 64;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  fp.tma = one_box && make_chunk_map(&fp.tq, p.q, dt16, 2, p, column, swqk, kDK, p.heads) &&
+                   make_chunk_map(&fp.tk, p.k, dt16, 2, p, column, swqk, kDK, p.heads) &&
+                   make_chunk_map(&fp.tv, p.v, dt16, 2, p, column, true, 64, p.heads) &&
+                   (fp.lowrank ? make_chunk_map(&fp.tz, p.gz, f32, 4, p, column, false, p.grank, 1)
+                               : make_chunk_map(&fp.tg, p.log_gamma, f32, 4, p, column, false, kDK, p.heads))
                ? 1
                : 0;
   fp.divW = make_fastdiv((uint32_t)p.W);
   fp.divH = make_fastdiv((uint32_t)p.H);
-  if (!fp.tma) {  // other chunks: 4-row gathers from [B*L*heads][64] row views
+  if (!fp.tma) {  // other chunks: 4-row gathers from [B*L*heads][d] row views
     const long long rows = (long long)p.B * p.L() * p.heads;
-    fp.tma = make_row_map(&fp.tq, p.q, dt16, 2, rows, true) && make_row_map(&fp.tk, p.k, dt16, 2, rows, true) &&
-                     make_row_map(&fp.tv, p.v, dt16, 2, rows, true) &&
-                     make_row_map(&fp.tg, p.log_gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, false)
+    fp.tma = make_row_map(&fp.tq, p.q, dt16, 2, rows, swqk, kDK) && make_row_map(&fp.tk, p.k, dt16, 2, rows, swqk, kDK) &&
+                     make_row_map(&fp.tv, p.v, dt16, 2, rows, true, 64) &&
+                     (fp.lowrank ? make_row_map(&fp.tz, p.gz, f32, 4, (long long)p.B * p.L(), false, p.grank)
+                                 : make_row_map(&fp.tg, p.log_gamma, f32, 4, rows, false, kDK))
                  ? 2
                  : 0;
   }
@@ -1814,17 +2095,22 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   const bool box = fp.tma == 1;
   const int kind = (rev ? 2 : 0) + (box ? 1 : 0);
   using Kern = void (*)(FusedParams);
-  const Kern kerns[3] = {pick_kernel<Tin, Tout, 0>(rev, box), pick_kernel<Tin, Tout, -1>(rev, box),
-                         pick_kernel<Tin, Tout, 2>(rev, box)};
-  static std::atomic<unsigned long long> configured[4];
+  // with the optional block pieces: one kernel that reads the plan mode at run time
+  const bool blk = fp.lowrank || fp.gated;
+  const Kern kb = pick_kernel<Tin, Tout, -1, kDK, true>(rev, box);
+  const Kern kerns[3] = {blk ? kb : pick_kernel<Tin, Tout, 0, kDK>(rev, box),
+                         blk ? kb : pick_kernel<Tin, Tout, -1, kDK>(rev, box),
+                         blk ? kb : pick_kernel<Tin, Tout, 2, kDK>(rev, box)};
+  static std::atomic<unsigned long long> configured[8];
+  const int ckind = kind + (blk ? 4 : 0);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GTR_ERR_CUDA;
-  if (!(configured[kind].load() & (1ull << dev))) {
+  if (!(configured[ckind].load() & (1ull << dev))) {
     for (Kern k : kerns)
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
         return GTR_ERR_CUDA;
-    configured[kind].fetch_or(1ull << dev);
+    configured[ckind].fetch_or(1ull << dev);
   }
   Plan pl = make_plan(p, device_sms());
   if (pl.mode == 1 && force_mode < 0) {

@@ -42,10 +42,14 @@ int fused_launches(const Problem& p);
 size_t fused_reset_bytes();  // header + counters: what a zeroed workspace must have zero
 // force_mode: -1 = let the plan decide, 0 = one CTA per sequence (stream mode)
 gtr_status_t launch_fused(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
-// one per input/output dtype pair, each in its own translation unit
-gtr_status_t launch_fused_f16_f16(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
-gtr_status_t launch_fused_f16_f32(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
-gtr_status_t launch_fused_bf16_f32(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
-gtr_status_t launch_fused_bf16_bf16(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
+// one per input/output dtype pair and key width, each in its own translation unit
+#define GTR_DECLARE_FUSED(tag)                                                                         \
+  gtr_status_t launch_fused_##tag##_dk64(const Problem& p, void* ws, cudaStream_t stream, int force_mode); \
+  gtr_status_t launch_fused_##tag##_dk32(const Problem& p, void* ws, cudaStream_t stream, int force_mode);
+GTR_DECLARE_FUSED(f16_f16)
+GTR_DECLARE_FUSED(f16_f32)
+GTR_DECLARE_FUSED(bf16_f32)
+GTR_DECLARE_FUSED(bf16_bf16)
+#undef GTR_DECLARE_FUSED
 
 }  // namespace gtr

@@ -26,8 +26,30 @@ namespace {
 constexpr int LD = kD + 1;  // padded smem row (floats)
 constexpr int kTile = kChunk * LD;
 
+// log gamma of channels g .. g+3 of scan position s of (b, h) from the low-rank gate
+// producer: logsigmoid(z W2 + bias) / tau (the rank-r projection z of the token).
+__device__ __forceinline__ float4 lowrank_log_gamma4(const Problem& p, int b, int h, long long s, int g) {
+  const long long m = scan_to_token(s, p.direction, p.H, p.W);
+  const float* z = p.gz + ((long long)b * p.L() + m) * p.grank;
+  const int col = h * p.d_k + g, ld = p.heads * p.d_k;
+  float x[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = p.gb[col + e];
+  for (int i = 0; i < p.grank; ++i) {
+    const float zi = z[i];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = fmaf(zi, p.gw2[(long long)i * ld + col + e], x[e]);
+  }
+  float r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) r[e] = (fminf(x[e], 0.f) - log1pf(expf(-fabsf(x[e])))) / p.gtau;
+  return make_float4(r[0], r[1], r[2], r[3]);
+}
+
 // Load one chunk's rows (scan positions c*64 + r) of up to four tensors into
-// padded fp32 smem; rows past the sequence end are zero (log-gate 0 = no decay).
+// padded fp32 smem; rows past the sequence end are zero (log-gate 0 = no decay).  q, k
+// and the log-gates have d_k channels a row (32 or 64): key channels d_k .. 63 are zero,
+// so they add nothing to any product and the state rows they would feed stay zero.
 template <typename Tin>
 __device__ __forceinline__ void load_chunk(const Problem& p, int b, int h, int c,
                                            const Tin* q, const Tin* k, const Tin* v,
@@ -38,11 +60,14 @@ __device__ __forceinline__ void load_chunk(const Problem& p, int b, int h, int c
     const long long s = (long long)c * kChunk + r;
     float4 qq = make_float4(0.f, 0.f, 0.f, 0.f), kk = qq, vv = qq, gg = qq;
     if (s < L) {
-      const long long row = token_head_row(p, b, h, s) * kD + g;
-      if (Qs) qq = load4<Tin>(q + row);
-      if (Ks) kk = load4<Tin>(k + row);
-      if (Vs) vv = load4<Tin>(v + row);
-      if (Gs) gg = load4<float>(p.log_gamma + row);
+      const long long th = token_head_row(p, b, h, s);
+      const long long rk = th * p.d_k + g, rv = th * kD + g;
+      if (g < p.d_k) {
+        if (Qs) qq = load4<Tin>(q + rk);
+        if (Ks) kk = load4<Tin>(k + rk);
+        if (Gs) gg = p.gz ? lowrank_log_gamma4(p, b, h, s, g) : load4<float>(p.log_gamma + rk);
+      }
+      if (Vs) vv = load4<Tin>(v + rv);
     }
     const int o = r * LD + g;
     if (Qs) { Qs[o] = qq.x; Qs[o + 1] = qq.y; Qs[o + 2] = qq.z; Qs[o + 3] = qq.w; }
@@ -239,12 +264,35 @@ __global__ void __launch_bounds__(256) split_output_kernel(Problem p, const floa
   const float scale = rsqrtf((float)p.d_k);
   Tout* out = (Tout*)p.out;
 #pragma unroll
+  for (int e = 0; e < 4; ++e)
+#pragma unroll
+    for (int f = 0; f < 4; ++f) acc[e][f] *= scale;
+  if (p.ogate) {
+    // RMSNorm over the 64 value channels of each row (held by the 16 threads tid & 15 of
+    // its row group, consecutive lanes), the norm weight and the SiLU output gate
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float ss = acc[e][0] * acc[e][0] + acc[e][1] * acc[e][1] + acc[e][2] * acc[e][2] + acc[e][3] * acc[e][3];
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float rinv = rsqrtf(ss * (1.f / kD) + p.oeps);
+      const long long s = (long long)c * kChunk + i0 + e;
+      if (s < L) {
+        const long long row = token_head_row(p, b, h, s);
+        const float4 gt = load4<Tin>(reinterpret_cast<const Tin*>(p.ogate) + row * kD + j0);
+        const float gv[4] = {gt.x, gt.y, gt.z, gt.w};
+#pragma unroll
+        for (int f = 0; f < 4; ++f)
+          acc[e][f] = acc[e][f] * rinv * p.onorm_w[j0 + f] * (gv[f] / (1.f + expf(-gv[f])));
+      }
+    }
+  }
+#pragma unroll
   for (int e = 0; e < 4; ++e) {
     const long long s = (long long)c * kChunk + i0 + e;
     if (s < L) {
       const long long row = token_head_row(p, b, h, s);
-      store4<Tout>(out + row * kD + j0, make_float4(acc[e][0] * scale, acc[e][1] * scale,
-                                                     acc[e][2] * scale, acc[e][3] * scale));
+      store4<Tout>(out + row * kD + j0, make_float4(acc[e][0], acc[e][1], acc[e][2], acc[e][3]));
     }
   }
 }

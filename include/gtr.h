@@ -90,8 +90,11 @@ typedef enum {
 } gtr_path_t;
 
 /*
- * Supported shapes: d_k = d_v = 64.  dtype pairings (in -> out):
- * F32 -> F32;  F16 -> F16 or F32;  BF16 -> F32 or BF16.
+ * Supported shapes: d_v = 64 and d_k = 64 or 32 (d_k = 32: the pages' operator shape, GTR
+ * digest page, step 5 of "Method details").  dtype pairings (in -> out):
+ * F32 -> F32;  F16 -> F16 or F32;  BF16 -> F32 or BF16.  A BF16 OUTPUT is an opt-in
+ * outside the 1e-2 * rms accuracy bound: rounding o to bf16 alone costs up to 2^-9 max|o|
+ * (about 1.5% of rms on the GTR workloads); bf16 inputs give fp32 outputs by default.
  * Limits: B*heads <= 65535 * 64, L <= 2^28, B*L*heads*64 < 2^40 elements.
  */
 
@@ -190,6 +193,45 @@ gtr_status_t gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v,
                                  int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
                                  int direction, int in_dtype, int out_dtype,
                                  gtr_stream_t stream);
+
+/*
+ * The GLA token mixer of one GTR block in a single call: the key-only recurrence above
+ * with two optional pieces fused into it.
+ *
+ * LOW-RANK GATE PRODUCER (when gate_z != NULL; log_gamma must then be NULL).  GTR digest
+ * page (paper.rainbus.top), section "Core method": the retention gate is
+ * gamma_t = sigmoid(x_t W1 W2 + b)^(1/tau), a rank-16 factorisation with tau = 16.  The
+ * call takes z = x W1 (the rank-r projection of every token) and computes
+ *     log_gamma[b, m, h, :] = logsigmoid(z[b, m, :] W2 + b)[h*d_k .. h*d_k + d_k - 1] / tau
+ * on the fly instead of reading a log_gamma tensor (a quarter to a third of the bytes).
+ *   gate_z  [B, L, gate_rank] fp32 (token m = y * grid_W + x, shared by the heads)
+ *   gate_w2 [gate_rank, heads * d_k] fp32;  gate_b [heads * d_k] fp32
+ *   gate_rank in {4, 8, 12, 16};  gate_tau > 0 (finite)
+ * When gate_z is NULL, log_gamma [B, L, heads, d_k] fp32 is read as in gtr_gla_fwd.
+ *
+ * RMSNORM + SILU OUTPUT GATE (when out_gate != NULL).  0539edu.com, appendix E.3.1: the
+ * end-to-end implementation fuses RMSNorm and a SiLU-activated output gate into the GLA
+ * kernel's output epilogue.  With o the recurrence's output row of a token-head (d_v
+ * values):
+ *     out[b, m, h, j] = o_j / sqrt(mean_i o_i^2 + norm_eps) * norm_w[j] * SiLU(out_gate[b, m, h, j])
+ *   out_gate [B, L, heads, d_v] in in_dtype;  norm_w [d_v] fp32 (shared by the heads);
+ *   norm_eps >= 0 (finite).
+ * When out_gate is NULL, norm_w and norm_eps are ignored and out is o itself.
+ *
+ * Every other argument, layout, alignment rule and return code is that of gtr_gla_fwd_ex
+ * (all pointers 16-byte aligned device pointers).  `workspace` may be NULL: the library's
+ * cached workspace is then used, with the rules of gtr_gla_fwd; otherwise it is a caller
+ * workspace as for gtr_gla_fwd_ex (gtr_gla_workspace_bytes gives its size: the optional
+ * pieces need no extra workspace).  A bf16 OUTPUT (out_dtype GTR_BF16) is outside the
+ * 1e-2 * rms accuracy bound of this library: its own rounding costs up to 2^-9 max|o|.
+ */
+gtr_status_t gtr_gla_block_fwd(const void *q, const void *k, const void *v, const float *log_gamma,
+                               const float *gate_z, const float *gate_w2, const float *gate_b,
+                               int gate_rank, float gate_tau,
+                               const void *out_gate, const float *norm_w, float norm_eps,
+                               void *out, int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
+                               int direction, int in_dtype, int out_dtype, int path,
+                               void *workspace, size_t ws_bytes, gtr_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of

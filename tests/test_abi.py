@@ -54,7 +54,7 @@ def _fwd_ex(**kw):
     (dict(q=None), 1), (dict(out=None), 1), (dict(g=8), 1),          # null / misaligned
     (dict(B=0), 1), (dict(heads=-1), 1), (dict(H=0), 1), (dict(W=-3), 1),
     (dict(direction=4), 1), (dict(direction=-1), 1), (dict(din=7), 1), (dict(path=9), 1),
-    (dict(dk=32), 2), (dict(dv=128), 2),                              # valid but unsupported
+    (dict(dk=48), 2), (dict(dk=128), 2), (dict(dv=128), 2),           # valid but unsupported
     (dict(din=gtr.F32, dout=gtr.F16), 2), (dict(din=gtr.BF16, dout=gtr.F16), 2),
     (dict(ws=None, ws_bytes=0), 5),                                   # workspace missing
 ])
@@ -68,7 +68,8 @@ def test_workspace_query():
     assert n == 256 + 2048 + units * (2 * 64 * 64 + 64) * 4
     assert gtr.workspace_bytes(1, 6, 40, 40, 64, 64, gtr.F16, "auto") >= n
     assert gtr.workspace_bytes(0, 6, 40, 40) == 0
-    assert gtr.workspace_bytes(1, 6, 40, 40, 32, 64) == 0
+    assert gtr.workspace_bytes(1, 6, 40, 40, 48, 64) == 0
+    assert gtr.workspace_bytes(1, 6, 40, 40, 32, 64) > 0   # d_k = 32 is supported
 
 
 def test_typed_entries_validate_too():
@@ -116,3 +117,33 @@ def test_noalloc_validates_arguments_before_the_size_limit():
     assert _noalloc(1, 1, 64, 635, out=8) == 1                        # misaligned
     assert _noalloc(1, 1, 64, 635, din=gtr.BF16, dout=gtr.F16) == 2   # unsupported pairing
     assert _noalloc(1, 1, 64, 635, dk=48) == 2                        # unsupported d_k
+
+
+# ---------------------------------------------------------------- gtr_gla_block_fwd (host side)
+def _block(**kw):
+    a = dict(q=256, k=256, v=256, lg=256, z=None, w2=None, b=None, rank=0, tau=16.0, og=None, nw=None,
+             eps=1e-6, out=256, B=1, heads=2, H=8, W=8, dk=64, dv=64, direction=0, din=gtr.F16, dout=gtr.F16,
+             path=0, ws=None, wsb=0)
+    a.update(kw)
+    return gtr.lib.gtr_gla_block_fwd(a["q"], a["k"], a["v"], a["lg"], a["z"], a["w2"], a["b"], a["rank"],
+                                     a["tau"], a["og"], a["nw"], a["eps"], a["out"], a["B"], a["heads"], a["H"],
+                                     a["W"], a["dk"], a["dv"], a["direction"], a["din"], a["dout"], a["path"],
+                                     a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lg=None), 1),                                               # no gates at all
+    (dict(z=256, w2=256, b=256, rank=16), 1),                         # both gate sources
+    (dict(lg=None, z=256, w2=None, b=256, rank=16), 1),               # factor missing
+    (dict(lg=None, z=256, w2=256, b=256, rank=6), 1),                 # rank not a multiple of 4
+    (dict(lg=None, z=256, w2=256, b=256, rank=20), 1),                # rank above 16
+    (dict(lg=None, z=256, w2=256, b=256, rank=16, tau=0.0), 1),       # tau must be positive
+    (dict(lg=None, z=256, w2=256, b=256, rank=16, tau=float("inf")), 1),
+    (dict(og=256, nw=None), 1),                                       # norm weight missing
+    (dict(og=264, nw=256), 1),                                        # misaligned output gate
+    (dict(og=256, nw=256, eps=-1.0), 1),                              # negative eps
+    (dict(path=7), 1), (dict(dk=48), 2), (dict(din=gtr.BF16, dout=gtr.F16), 2),
+    (dict(ws=256, wsb=16), 5),                                        # caller workspace too small
+])
+def test_block_arguments_rejected_on_host(kw, code):
+    assert _block(**kw) == code

@@ -122,6 +122,35 @@ def test_no_decay_gates(path):
     assert rel_err(out, ref) <= 1e-2
 
 
+# ------------------------------------------------------------------ d_k = 32 (the pages' kernel shape)
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+@pytest.mark.parametrize("name", ["640", "1024", "2048"])
+def test_key_width_32_all_directions(name, path):
+    """d_k = 32, d_v = 64 (C = 64, the operator specialisation of the GTR digest page, step 5
+    of "Method details"): the 640^2 and 2048^2 fp16 and the 1024^2 bf16 grids in all four
+    directions against the oracle."""
+    w = WORKLOADS[name].with_(d_k=32)
+    for d in range(4):
+        check(w, d, w.seed(d) + 32, path)
+
+
+@pytest.mark.parametrize("path", ["auto"] + PATHS)
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1), (1, 3, 7, 9), (1, 2, 33, 31), (2, 3, 65, 1), (13, 6, 8, 16)])
+def test_key_width_32_ragged_shapes(shape, path):
+    B, heads, H, W = shape
+    w = Workload("odd32", B=B, heads=heads, H=H, W=W, d_k=32, dtype="bf16", index=9)
+    for d in range(4):
+        check(w, d, 7300 + 100 * H + W + d, path)
+
+
+def test_key_width_32_tiny_inputs_and_strong_decay():
+    """The input rescale and the CUDA-core scores with the 32-channel layout."""
+    for w, d in ((Workload("tiny32", B=1, heads=2, H=40, W=40, d_k=32, dtype="bf16", scale=2.0 ** -20), 1),
+                 (Workload("strong32", B=1, heads=2, H=24, W=24, d_k=32, dtype="f16", gate_offset=-2.0,
+                           gate_tau=2.0), 2)):
+        check(w, d, 7400 + d, "fused", out_dtype=torch.float32)
+
+
 # shapes that take each plan of the fused kernel: one cluster per sequence (2 x 25 chunks),
 # several CTAs per sequence exchanging segment summaries (2 x 224 chunks), one CTA per
 # sequence (78 sequences of 2 chunks)
