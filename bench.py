@@ -31,7 +31,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from gtr_inputs import DTYPES, WORKLOADS, make_inputs  # noqa: E402
+from gtr_inputs import (DTYPES, STENCILS, WORKLOADS, make_gate_epilogue_inputs, make_inputs,  # noqa: E402
+                        make_lowrank_gate_inputs, make_stencil_inputs)
 
 METRIC = "GLA fwd tokens/s and % of HBM roofline at 1.6K/4.1K/16.4K tokens, 1×B200"
 L2_BYTES = 126 * 2 ** 20
@@ -302,6 +303,100 @@ def sweep(gtr, names, path, device, stream, hbm):
     return res
 
 
+def time_rotating(call, n_sets, stream, reps=3):
+    """Median per-call time (ms) of `call(i)` over rotating buffer sets i, 2 * n_sets calls
+    captured in one CUDA graph and timed with one event pair on the capture stream."""
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            call(i)
+    torch.cuda.synchronize()
+    steps = 2 * n_sets
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            call(i)
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / steps)
+    del g
+    return statistics.median(times)
+
+
+def sweep_pieces(gtr, device, stream, hbm):
+    """The d_k = 32 operator (the pages' kernel shape), the full GTR block call (low-rank
+    gate producer + RMSNorm/SiLU output gate) and the Spatial SwiGLU stencil, each on its
+    own rotating buffer sets; algorithmic bytes per call / device time per call."""
+    res = {}
+    code = {"f32": 0, "f16": 1, "bf16": 2}
+
+    def line(name, bytes_, ms, tokens, extra=None):
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        d = {"us_per_call": ms * 1e3, "tokens_per_s": tokens / (ms * 1e-3), "GBps": gbs, "hbm_frac": gbs / hbm,
+             "bytes_per_call": bytes_}
+        d.update(extra or {})
+        res[name] = d
+
+    for base in ("640", "2048"):  # d_k = 32, d_v = 64
+        w = WORKLOADS[base].with_(d_k=32)
+        sets = make_sets(w, n_sets_for(w), device, 0)
+        ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, w.d_k, w.d_v, code[w.dtype], "auto", device)
+
+        def call(i, sets=sets, w=w, ws=ws):
+            d, q, k, v, lg, out = sets[i % len(sets)]
+            gtr.gla_fwd(q, k, v, lg, grid=(w.H, w.W), direction=d, out=out, workspace=ws, stream=stream)
+        line(base + "_dk32", w.algorithmic_bytes(), time_rotating(call, len(sets), stream), w.B * w.L,
+             {"d_k": 32, "path": gtr.plan(w.B, w.heads, w.H, w.W, 32, 64, code[w.dtype])[0]})
+        del sets
+        torch.cuda.empty_cache()
+
+    # the block call at 2048^2: z (rank 16, per token) replaces the fp32 gates, the output
+    # gate is read in the epilogue
+    w = WORKLOADS["2048"]
+    es = torch.finfo(DTYPES[w.dtype]).bits // 8
+    eo = torch.finfo(DTYPES[w.out_dtype]).bits // 8
+    blk_bytes = w.token_heads * ((2 * w.d_k + w.d_v) * es + w.d_v * es + w.d_v * eo) + w.B * w.L * 16 * 4
+    n = max(3, min(64, math.ceil(3 * L2_BYTES / blk_bytes)))
+    bsets = []
+    for i in range(n):
+        d = w.direction_of_call(i)
+        q, k, v, _ = make_inputs(w, w.seed(d, i), device=device)
+        z, w2, b = (t.to(device) for t in make_lowrank_gate_inputs(w, w.seed(d, i)))
+        og, nw, eps = make_gate_epilogue_inputs(w, w.seed(d, i))
+        out = torch.empty((w.B, w.L, w.heads, w.d_v), dtype=DTYPES[w.out_dtype], device=device)
+        bsets.append((d, q, k, v, z, w2, b, og.to(device), nw.to(device), eps, out))
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, w.d_k, w.d_v, code[w.dtype], "auto", device)
+
+    def bcall(i):
+        d, q, k, v, z, w2, b, og, nw, eps, out = bsets[i % n]
+        gtr.gla_block_fwd(q, k, v, grid=(w.H, w.W), direction=d, gate_z=z, gate_w2=w2, gate_b=b, gate_tau=16.0,
+                          out_gate=og, norm_w=nw, norm_eps=eps, out=out, workspace=ws, stream=stream)
+    line("2048_block", blk_bytes, time_rotating(bcall, n, stream), w.B * w.L, {"pieces": "lowrank gate + output gate"})
+    del bsets
+    torch.cuda.empty_cache()
+
+    for name, st in STENCILS.items():  # SiLU(xg) * DWConv3x3(xv)
+        n = max(3, min(64, math.ceil(3 * L2_BYTES / st.algorithmic_bytes())))
+        ssets = []
+        for i in range(n):
+            xg, xv, cw, cb = (t.to(device) for t in make_stencil_inputs(st, 9000 + i))
+            ssets.append((xg, xv, cw, cb, torch.empty_like(xv)))
+
+        def scall(i, ssets=ssets, st=st):
+            xg, xv, cw, cb, out = ssets[i % len(ssets)]
+            gtr.sswiglu_dwconv(xg, xv, cw, cb, grid=(st.H, st.W), out=out, stream=stream)
+        line(name, st.algorithmic_bytes(), time_rotating(scall, n, stream), st.B * st.L,
+             {"C": st.C, "dtype": st.dtype})
+        del ssets
+        torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- arms
 def run_reference(args):
     world, rank, _ = dist_env()
@@ -394,6 +489,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_sweep:
         extra["sweep"] = sweep(gtr, [n for n in ("640", "1024", "2048", "stack") if n != w.name],
                                args.path, device, stream, hbm)
+        extra["sweep"].update(sweep_pieces(gtr, device, stream, hbm))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(w, seconds=args.cpu_seconds)

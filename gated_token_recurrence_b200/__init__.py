@@ -31,7 +31,8 @@ STATUS = {0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED", 3: "G
 EXPORTED = ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
             "gtr_gla_workspace_bytes", "gtr_gla_fwd_ex", "gtr_gla_fwd_host",
             "gtr_gla_read_error", "gtr_gla_plan", "gtr_gla_workspace_init", "gtr_status_string",
-            "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd")
+            "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd", "gtr_sswiglu_dwconv",
+            "gtr_gla_workspace_debug")
 
 
 class GTRError(RuntimeError):
@@ -56,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.gtr_gla_fwd_noalloc.argtypes = fwd_args + [i, i, vp]
     f = ctypes.c_float
     lib.gtr_gla_block_fwd.argtypes = [vp] * 7 + [i, f, vp, vp, f, vp] + [i] * 10 + [vp, sz, vp]
+    lib.gtr_sswiglu_dwconv.argtypes = [vp] * 5 + [i] * 5 + [vp]
+    lib.gtr_gla_workspace_debug.argtypes = [vp, i, ctypes.c_uint, vp]
     lib.gtr_gla_workspace_bytes.argtypes = [i] * 8
     lib.gtr_gla_workspace_bytes.restype = sz
     lib.gtr_gla_read_error.argtypes = [vp, vp]
@@ -66,7 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.gtr_version.argtypes = []
     for name in ("gtr_gla_fwd", "gtr_gla_fwd_f16", "gtr_gla_fwd_bf16", "gtr_gla_fwd_f32",
                  "gtr_gla_fwd_ex", "gtr_gla_fwd_host", "gtr_gla_read_error", "gtr_gla_plan",
-                 "gtr_gla_workspace_init", "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd"):
+                 "gtr_gla_workspace_init", "gtr_version", "gtr_gla_fwd_noalloc", "gtr_gla_block_fwd",
+                 "gtr_sswiglu_dwconv", "gtr_gla_workspace_debug"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -182,6 +186,26 @@ def gla_block_fwd(q, k, v, grid: Tuple[int, int], direction: int = L2R, log_gamm
                                float(norm_eps), out.data_ptr(), B, heads, H, W, d_k, d_v, int(direction),
                                _dtype_code(q), _dtype_code(out), PATHS[path], ws, wsb, _stream_handle(stream))
     _check(st, "gtr_gla_block_fwd")
+    return out
+
+
+def sswiglu_dwconv(xg, xv, conv_w, conv_b, grid: Tuple[int, int], out=None, stream=None):
+    """SiLU(xg) * DWConv3x3(xv) on CUDA tensors ([B, L, C], L = H * W; conv_w [C, 3, 3] fp32,
+    conv_b [C] fp32 or None) through ``gtr_sswiglu_dwconv``."""
+    import torch
+    B, L, C = xv.shape
+    H, W = grid
+    if H * W != L or xg.shape != xv.shape or xg.dtype != xv.dtype:
+        raise ValueError("xg and xv must both be [B, H*W, C] of one dtype")
+    if out is None:
+        out = torch.empty_like(xv)
+    for t in (xg, xv, conv_w, out) + (() if conv_b is None else (conv_b,)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("sswiglu_dwconv takes contiguous CUDA tensors")
+    st = lib.gtr_sswiglu_dwconv(xg.data_ptr(), xv.data_ptr(), conv_w.data_ptr(),
+                                None if conv_b is None else conv_b.data_ptr(), out.data_ptr(), B, H, W, C,
+                                _dtype_code(xv), _stream_handle(stream))
+    _check(st, "gtr_sswiglu_dwconv")
     return out
 
 

@@ -1,5 +1,6 @@
 // C ABI of libgtr.so: argument validation, workspace management, length-aware
 // dispatch and the host-buffer entry.  The arithmetic lives in the kernel files.
+#include <cstddef>
 #include <mutex>
 #include <vector>
 
@@ -291,6 +292,18 @@ gtr_status_t gtr_gla_block_fwd(const void* q, const void* k, const void* v, cons
   st = ensure(c.ws, need, s);
   if (st != GTR_OK) return st;
   return run(p, path, c.ws.ptr, c.ws.bytes, s);
+}
+
+gtr_status_t gtr_gla_workspace_debug(void* workspace, int skip_segment, unsigned int wait_limit_us,
+                                     gtr_stream_t stream) {
+  if (!workspace || !is_aligned(workspace, 256)) return GTR_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GTR_ERR_CUDA;
+  const unsigned int v[2] = {skip_segment >= 0 ? (unsigned int)skip_segment + 1u : 0u,
+                             skip_segment >= 0 ? wait_limit_us : 0u};
+  return cudaMemcpy(reinterpret_cast<uint8_t*>(workspace) + offsetof(WsHeader, dbg_skip_seg), v, sizeof(v),
+                    cudaMemcpyHostToDevice) == cudaSuccess
+             ? GTR_OK
+             : GTR_ERR_CUDA;
 }
 
 gtr_status_t gtr_gla_workspace_init(void* workspace, size_t ws_bytes, gtr_stream_t stream) {

@@ -19,7 +19,12 @@ struct WsHeader {
   unsigned int error_aux;  // where it happened (kernel-specific)
   unsigned int ticket;     // dynamic work counter for ticketed kernels
   unsigned int epoch;      // call counter, bumps every fused call
-  unsigned int pad[60];
+  // failure injection (gtr_gla_workspace_debug; zero = off): segment dbg_skip_seg - 1 of
+  // every sequence withholds its summary flag, and waits for other segments' flags give
+  // up after dbg_wait_us microseconds instead of about a second
+  unsigned int dbg_skip_seg;
+  unsigned int dbg_wait_us;
+  unsigned int pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header must stay 256 bytes");
 

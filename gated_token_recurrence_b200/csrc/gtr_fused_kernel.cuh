@@ -289,16 +289,17 @@ __device__ bool wait_spin(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hd
   }
 }
 
-// Bounded wait until a global counter reaches `target`.
+// Bounded wait until a global counter reaches `target` (`limit_ns`: about a second, or the
+// workspace's failure-injection limit).
 __device__ bool wait_counter(const unsigned int* ctr, unsigned int target, Misc* ms, WsHeader* hdr,
-                             uint32_t where) {
+                             uint32_t where, uint64_t limit_ns = 1000000000ull) {
   const uint64_t t0 = globaltimer();
   while (true) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
     if (*(volatile int*)&ms->abort) return false;
-    if (globaltimer() - t0 > 1000000000ull) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(hdr, GTR_ERR_TIMEOUT, where);
       *(volatile int*)&ms->abort = 1;
       return false;
@@ -1638,7 +1639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __threadfence();
       wg_sync(wg);
-      if (wtid == 0) st_release_u32(fp.counters + (size_t)seq * fp.n_s + seg, 1u);
+      // (failure injection: a segment may withhold its flag, so that the later ones time out)
+      if (wtid == 0 && *(volatile unsigned int*)&hdr->dbg_skip_seg != (unsigned int)seg + 1u)
+        st_release_u32(fp.counters + (size_t)seq * fp.n_s + seg, 1u);
     }
     if (segm && alive && wtid == 0) mbar_arrive(&ms->agg_pub);
   } else if (warp < 16) {
@@ -1711,10 +1714,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the Qh' and O_local tiles are written and fenced once the summary is out (WG_B and
         // the Qh' warp arrive): the first four pairs of the second phase start loading now
         bool ok = !*(volatile int*)&ms->abort && wait_bar(&ms->agg_pub, 0u, ms, hdr, 0x600);
-        if (ok)
-          for (int q = 0; q < 4 && 2 * q < cnt; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
+        const int loads = ok ? min(4, (cnt + 1) / 2) : 0;
+        for (int q = 0; q < loads; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
+        const unsigned int dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
+        const uint64_t limit = dbg_us ? 1000ull * dbg_us : 1000000000ull;
         for (int j = 0; j < seg && ok; ++j)
-          ok = wait_counter(fp.counters + (size_t)seq * fp.n_s + j, 1u, ms, hdr, 0x601);
+          ok = wait_counter(fp.counters + (size_t)seq * fp.n_s + j, 1u, ms, hdr, 0x601, limit);
+        if (!ok) {
+          // giving up: this CTA's own bulk copies land before it leaves (they read the
+          // workspace only, so they complete on their own; the wait is bounded all the same)
+          for (int q = 0; q < loads; ++q)
+            for (int it = 0; it < 1000 && !mbar_wait_sleep(&ms->p2_full[q], 0u, 1000000u); ++it) {
+            }
+        }
         ms->seg_go = ok ? 1 : 0;
       }
       named_sync(7, 4 * kWG);

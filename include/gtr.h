@@ -148,6 +148,21 @@ gtr_status_t gtr_gla_fwd_ex(const void *q, const void *k, const void *v,
                             int direction, int in_dtype, int out_dtype, int path,
                             void *workspace, size_t ws_bytes, gtr_stream_t stream);
 
+/*
+ * Failure injection, for tests of the device-side failure detection (not for production
+ * use; the paper has no counterpart).  Synchronises `stream`, then marks `workspace` (a
+ * caller workspace of gtr_gla_fwd_ex) so that in the next fused-path calls that split a
+ * sequence over several CTAs (the segmented plan), segment `skip_segment` of every
+ * sequence withholds its summary, and the later segments' waits for it give up after
+ * `wait_limit_us` microseconds (0 keeps the default of about a second): they record
+ * GTR_ERR_TIMEOUT in the workspace's error word, skip their second phase and leave
+ * cleanly, so the call ends and the GPU context stays usable; the outputs of those
+ * segments are not valid.  gtr_gla_read_error() then returns GTR_ERR_TIMEOUT and clears
+ * the mark together with the error.  skip_segment < 0 clears the mark.
+ */
+gtr_status_t gtr_gla_workspace_debug(void *workspace, int skip_segment, unsigned int wait_limit_us,
+                                     gtr_stream_t stream);
+
 /* Zero `ws_bytes` of a caller workspace on `stream` (asynchronous; capturable). */
 gtr_status_t gtr_gla_workspace_init(void *workspace, size_t ws_bytes, gtr_stream_t stream);
 
@@ -232,6 +247,32 @@ gtr_status_t gtr_gla_block_fwd(const void *q, const void *k, const void *v, cons
                                void *out, int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
                                int direction, int in_dtype, int out_dtype, int path,
                                void *workspace, size_t ws_bytes, gtr_stream_t stream);
+
+/*
+ * Spatial SwiGLU stencil of a GTR block: out = SiLU(xg) * DWConv3x3(xv).
+ *
+ * GTR digest page (paper.rainbus.top), prerequisite "SwiGLU" and section "Core method";
+ * page 0539edu.com section 3.1 ("Spatial SwiGLU"): the channel mixer is
+ * Y = SiLU(X W_g) (.) DWConv3x3(X W_v) W_o, a 3x3 depthwise convolution in the value branch
+ * that mixes neighbouring patches.  This call takes the two projections xg = X W_g and
+ * xv = X W_v and returns the product in front of W_o (the projections are GEMMs outside
+ * this library):
+ *     out[b, y, x, c] = SiLU(xg[b, y, x, c]) *
+ *         (conv_b[c] + sum_{dy, dx in 0..2} conv_w[c, dy, dx] * xv[b, y+dy-1, x+dx-1, c])
+ * with zero padding at the grid border (the cross-correlation convention of a
+ * convolution layer).
+ *   xg, xv, out: [B, grid_H * grid_W, C] in `dtype` (GTR_F16, GTR_BF16 or GTR_F32), token
+ *                m = y * grid_W + x, 16-byte aligned device pointers; out must not overlap
+ *                the inputs.
+ *   conv_w: [C, 3, 3] fp32;  conv_b: [C] fp32 or NULL (no bias); device pointers.
+ *   C: a multiple of 64 (16-bit data) or of 32 (fp32) -- whole 128-byte channel blocks;
+ *      otherwise GTR_ERR_UNSUPPORTED.
+ * Asynchronous on `stream`; no workspace; allocates nothing; capturable.  Returns
+ * GTR_ERR_INVALID_ARG for null or misaligned pointers and non-positive sizes.
+ */
+gtr_status_t gtr_sswiglu_dwconv(const void *xg, const void *xv, const float *conv_w, const float *conv_b,
+                                void *out, int B, int grid_H, int grid_W, int C, int dtype,
+                                gtr_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of

@@ -147,3 +147,15 @@ def _block(**kw):
 ])
 def test_block_arguments_rejected_on_host(kw, code):
     assert _block(**kw) == code
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, 256, 256, None, 256, 1, 8, 8, 64, 1), 1),      # null xg
+    ((256, 256, 256, None, 264, 1, 8, 8, 64, 1), 1),       # misaligned out
+    ((256, 256, 256, None, 256, 0, 8, 8, 64, 1), 1),       # B = 0
+    ((256, 256, 256, None, 256, 1, 8, 8, 64, 5), 1),       # bad dtype
+    ((256, 256, 256, None, 256, 1, 8, 8, 96, 1), 2),       # C not whole 64-channel blocks (16-bit)
+    ((256, 256, 256, None, 256, 1, 8, 8, 48, 0), 2),       # C not whole 32-channel blocks (fp32)
+])
+def test_stencil_arguments_rejected_on_host(args, code):
+    assert gtr.lib.gtr_sswiglu_dwconv(*args, None) == code

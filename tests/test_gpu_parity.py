@@ -406,3 +406,26 @@ def test_graph_of_calls_in_every_plan_matches_the_oracle():
             assert err <= TOL[w.dtype], f"{w.name} rep={rep}: max err / rms = {err:.3e}"
             assert gtr.read_error(ws) == 0, f"{w.name} rep={rep}: device error"
     del g
+
+
+# ------------------------------------------------------------------ device-side failure detection
+def test_a_withheld_segment_summary_times_out_and_the_workspace_recovers():
+    """Failure injection (gtr_gla_workspace_debug): segment 1 of every sequence withholds
+    its summary and the later segments' waits give up after 200 us.  The call must end,
+    report GTR_ERR_TIMEOUT through the workspace's error word, and leave the workspace and
+    the context usable: the next call on the same workspace matches the oracle."""
+    w = Workload("inj", B=1, heads=2, H=128, W=112, dtype="f16", scale=0.5, index=9)  # segmented plan
+    q, k, v, lg = make_inputs(w, 4321)
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 0)
+    dev = torch.device("cuda:0")
+    t = tuple(x.to(dev) for x in (q, k, v, lg))
+    ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, in_dtype=gtr.F16, path="fused", device=dev)
+    s = torch.cuda.current_stream().cuda_stream
+    assert gtr.lib.gtr_gla_workspace_debug(ws.data_ptr(), 1, 200, s) == 0
+    gtr.gla_fwd(*t, grid=(w.H, w.W), direction=0, path="fused", workspace=ws)
+    assert gtr.read_error(ws) == 4  # GTR_ERR_TIMEOUT, and the mark is cleared with it
+    assert gtr.read_error(ws) == 0
+    out = gtr.gla_fwd(*t, grid=(w.H, w.W), direction=0, path="fused", workspace=ws)
+    torch.cuda.synchronize()
+    assert rel_err(out, ref) <= 1e-2
+    assert gtr.read_error(ws) == 0
