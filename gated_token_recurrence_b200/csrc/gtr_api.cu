@@ -258,7 +258,7 @@ gtr_status_t gtr_gla_block_fwd(const void* q, const void* k, const void* v, cons
   if (st != GTR_OK) return st;
   if (gate_z) {
     if (!gate_w2 || !gate_b || !is_aligned(gate_w2, 16) || !is_aligned(gate_b, 16)) return GTR_ERR_INVALID_ARG;
-    if (gate_rank < 4 || gate_rank > 16 || gate_rank % 4 != 0) return GTR_ERR_INVALID_ARG;
+    if (gate_rank != 8 && gate_rank != 16) return GTR_ERR_INVALID_ARG;
     if (!(gate_tau > 0.f) || !(gate_tau < 3.0e38f)) return GTR_ERR_INVALID_ARG;
   }
   if (out_gate) {

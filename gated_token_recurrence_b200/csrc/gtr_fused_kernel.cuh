@@ -111,8 +111,9 @@ static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) re
 // the problem size, so that a workspace kept zero between calls stays valid across shapes.
 constexpr size_t kMaxSegCtas = 256;  // CTAs of one launch in SEGMENTED mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
-// per-segment summary: U_seg [64][64] fp32 and the log2 decay [64]
-constexpr size_t kAggStride = 4096 + 64;
+constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
+// per-segment summary: U_seg [64][64] fp32, the log2 decay [64], the start-state factor, padding
+constexpr size_t kAggStride = 4096 + 128;
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 // floor(n / d) for 0 <= n < 2^31 by one wide multiply and a shift: with l = ceil(log2 d)
@@ -140,8 +141,9 @@ struct alignas(64) FusedParams {
   CUtensorMap tz;          // low-rank gate producer: the rank-r token projections z (fp32), same views
   Problem p;
   WsHeader* hdr;
-  unsigned int* counters;  // SEGMENTED: [n_seq][n_s] segment flags (summary published), zero between calls
-  float* agg;              // [n_seq][n_s][64*64 + 64] segment summaries (U_seg, log2 decay)
+  unsigned int* counters;  // SEGMENTED: [n_seq][2] arrival counters, monotonic within a call, zero between calls
+  float* agg;              // [n_seq][n_s][kAggStride] segment summaries (U_seg, log2 decay, start-state factor)
+  uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
   uint16_t* qhp;           // [n_seq][Nc][64*64] Qh' per chunk, fp16, MMA layout
   uint16_t* olc;           // [n_seq][Nc][64][64] outputs from a zero segment start, fp16
   int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED, 2 = CLUSTER
@@ -190,7 +192,7 @@ struct Misc {
   uint64_t sready[kNS];                              // per chunk-start state tile
   uint64_t qdone[kStages];                           // Qh' of the staged chunk copied out
   uint64_t o_full[kOPairs], o_free[kOPairs];         // per output pair
-  uint64_t agg_pub, mma_final[2], corr_done[kOPairs];
+  uint64_t agg_pub, p2_go, mma_final[2], corr_done[kOPairs];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
   uint64_t scale_ready;            // the input scale factors below are set (WG_A, first chunk)
   uint32_t tmem_base;
@@ -203,7 +205,6 @@ struct Misc {
   float sc_spub;  // 2^-(beta+gamma): this CTA's state back to the inputs' scale (published summaries)
   float sc_sin;   // 2^(beta+gamma): a state in the inputs' scale into this CTA's scale (start states)
   unsigned int smax[4][3];  // WG_A0: per-warp largest |q|, |k|, |v| bit patterns of the first chunk
-  int seg_go;               // SEGMENTED: the start state can be composed (the predecessors published)
   alignas(16) float w2s[16][64];  // low-rank gate producer: this head's W2 columns [rank][64] (zero past d_k)
   alignas(16) float bs[64];       // ... and bias (zero past d_k)
   alignas(16) float nw[64];       // output gate: RMSNorm weight
@@ -311,14 +312,6 @@ __device__ __forceinline__ void red_release_add(unsigned int* ctr, unsigned int 
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Named barrier `id` over the first `n` threads of the CTA (a multiple of 32).
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // Named barrier of one 128-thread warpgroup (ids 1..3).
 __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory"); }
@@ -327,9 +320,9 @@ __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128
 // group takes the same decision (no thread is left alone at a named barrier) and
 // observes the completed phase itself.
 __device__ bool wg_wait(int wg, int wtid, uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr,
-                        uint32_t where, int& slot) {
+                        uint32_t where, int& slot, bool spin = false) {
   if (wtid == 0) {
-    const bool ok = wait_bar(bar, parity, ms, hdr, where);
+    const bool ok = spin ? wait_spin(bar, parity, ms, hdr, where) : wait_bar(bar, parity, ms, hdr, where);
     ms->go[wg][slot] = ok && !*(volatile int*)&ms->abort;
   }
   wg_sync(wg);
@@ -774,6 +767,7 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
                                                   uint32_t tmem, int q, int wtid, int lane, int seq, int b, int h,
                                                   Span sp, int& slot, float& nf) {
   const int wq = (wtid >> 5) & 3;
+  if (!wg_wait(q, wtid, &ms->p2_go, 0u, ms, hdr, 0x700u + q, slot)) return;
   const long long L = fp.p.L();
   const int cnt = sp.c1 - sp.c0, npairs = (cnt + 1) / 2;
   uint8_t* sbuf = smem + kOffStage + q * kStageBytes;
@@ -910,6 +904,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (i == 8) mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
     if (i == 10) mbar_init(&ms->mma_final[0], 1);
     if (i == 11) mbar_init(&ms->mma_final[1], 1);
+    if (i == 9) mbar_init(&ms->p2_go, 1);
     if (i == 12) ms->abort = 0;
     if (i == 13) mbar_init(&ms->scale_ready, 1);
     fence_mbar_init();
@@ -1271,7 +1266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint3 m = own_absmax_bits<kDK>(qr, kr, sb + 2 * kTile, row0, cc, wtid);
         if (lane == 0) ms->smax[w4][0] = m.x, ms->smax[w4][1] = m.y, ms->smax[w4][2] = m.z;
       } else if (n == 1) {  // warpgroup 1's first chunk: take the scale warpgroup 0 set
-        if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot)) {
+        if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot, true)) {
           alive = false;
           break;
         }
@@ -1388,8 +1383,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e)
           if (-last[ps][e] > fp.max_exp2) exp_unsafe = true;
       }
-      // CUDA-core decision: the lanes of every warp hold the decays of all d_k channels
-      const bool fbx = __any_sync(0xffffffffu, exp_unsafe);
+      // CUDA-core decision: the lanes of every warp hold the decays of all d_k channels.  With
+      // the output gate, the sequence's first chunk also takes the exact CUDA-core scores: its
+      // first tokens' outputs sum few terms, and the RMSNorm scales each row to unit size, so
+      // the fp16 rounding of the factorised operands would no longer be averaged away.
+      const bool fbx = __any_sync(0xffffffffu, exp_unsafe) || (gated && sp.c0 + n == 0);
       if (fbx) {
         // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
         // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i).
@@ -1496,6 +1494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->opready[st]);  // every warp, once its writes are done
     }
+    if (partial && alive)
+      second_phase<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
   } else if (warp < 12) {
     // ===================================================================== WG_B: masking, state
     // Tensor-memory rows through the 16-lane shape: register 4c+q of this thread is row
@@ -1520,9 +1520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->sready[0]);
     }
-    // the input scale (published summaries go back to the inputs' scale)
-    if (!wait_bar(&ms->scale_ready, 0u, ms, hdr, 0x405)) alive = false;
-    for (int n = 0; n < cnt && alive; ++n) {
+    for (int n = 0; n < cnt; ++n) {
       const int st = n % kStages, su = n % kSU;
       if (!wait_bar(&ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400)) { alive = false; break; }
       tc_fence_after();
@@ -1602,7 +1600,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&ms->sready[(n + 1) % kNS]);
       }
     }
-    // every thread leaves the loop (the waits are bounded): agree on the outcome
+    // every thread leaves the loop (the waits are bounded): agree on the outcome, and that
+    // the input scale is known (the summaries go back to the inputs' scale; the scale was
+    // set before chunk 0's operands, so this spin finds it complete)
+    if ((segm || clus) && alive) alive = wait_spin(&ms->scale_ready, 0u, ms, hdr, 0x405);
     alive = wg_all(wg, alive);
     if (clus && alive) {
       // segment summary for the cluster's scan, read by the other CTAs after the cluster
@@ -1622,9 +1623,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       wg_sync(wg);
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
     }
-    if (segm && alive && seg + 1 < fp.n_s) {
-      // segment summary, read by the later segments of the sequence: U_seg = local end state
-      // (in the inputs' scale) and its log2 decay; then the segment's flag
+    if (segm && alive) {
+      // segment summary: U_seg = local end state (in the inputs' scale), its log2 decay, and
+      // the factor that takes a start state into this CTA's scale
       float* mine = fp.agg + ((size_t)seq * fp.n_s + seg) * kAggStride;
       const float f = ms->sc_spub;
 #pragma unroll
@@ -1637,13 +1638,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mine[4096 + r0] = a2r0;
         mine[4096 + r1] = a2r1;
       }
+      if (wtid == 0) mine[4096 + 64] = ms->sc_sin;
       __threadfence();
       wg_sync(wg);
-      // (failure injection: a segment may withhold its flag, so that the later ones time out)
-      if (wtid == 0 && *(volatile unsigned int*)&hdr->dbg_skip_seg != (unsigned int)seg + 1u)
-        st_release_u32(fp.counters + (size_t)seq * fp.n_s + seg, 1u);
+      if (wtid == 0) mbar_arrive(&ms->agg_pub);
+      if (partial)
+        second_phase<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
     }
-    if (segm && alive && wtid == 0) mbar_arrive(&ms->agg_pub);
   } else if (warp < 16) {
     // ===================================================================== WG_C: epilogue, scan
     const int wg = 3, wtid = tid - 3 * kWG, wq = warp & 3;
@@ -1652,7 +1653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
-    // the input scale (the outputs are stored in the inputs' scale)
+    // the input scale (the outputs are stored in the inputs' scale; a sleeping wait: the
+    // first outputs come microseconds after the scale)
     bool alive = wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x505, slot);
     if (clus) {
       // the outputs stay in tensor memory until the start state is known: wait for their
@@ -1697,82 +1699,130 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the O_local rows written above are read back by bulk copy (async proxy)
       if (partial) asm volatile("fence.proxy.async.global;" ::: "memory");
     }
-  }
-
-  if (segm && tid < 4 * kWG) {
-    // ===================================================================== SEGMENTED combine
-    // Every thread of warps 0-15 meets here (every wait before is bounded).  A segment s > 0
-    // waits for the flags of segments 0 .. s-1 of its sequence (their summaries are
-    // published), composes its start state from those summaries itself -- thread t owns the
-    // eight state entries 8t .. 8t+7 (key channel t/8) and walks the segments in order, so
-    // the result does not depend on timing -- and writes it (fp16, MMA layout, in this CTA's
-    // scale) straight into shared memory; then all four warpgroups run the second phase.
-    // Segment 0's outputs are final already.
-    named_sync(7, 4 * kWG);
-    if (seg > 0) {
-      if (tid == 0) {
-        // the Qh' and O_local tiles are written and fenced once the summary is out (WG_B and
-        // the Qh' warp arrive): the first four pairs of the second phase start loading now
-        bool ok = !*(volatile int*)&ms->abort && wait_bar(&ms->agg_pub, 0u, ms, hdr, 0x600);
-        const int loads = ok ? min(4, (cnt + 1) / 2) : 0;
-        for (int q = 0; q < loads; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
-        const unsigned int dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
-        const uint64_t limit = dbg_us ? 1000ull * dbg_us : 1000000000ull;
-        for (int j = 0; j < seg && ok; ++j)
-          ok = wait_counter(fp.counters + (size_t)seq * fp.n_s + j, 1u, ms, hdr, 0x601, limit);
-        if (!ok) {
-          // giving up: this CTA's own bulk copies land before it leaves (they read the
-          // workspace only, so they complete on their own; the wait is bounded all the same)
-          for (int q = 0; q < loads; ++q)
-            for (int it = 0; it < 1000 && !mbar_wait_sleep(&ms->p2_full[q], 0u, 1000000u); ++it) {
-            }
+    if (segm && alive) {
+      // Scan of the segment summaries.  This CTA owns state entries [4 f0, 4 f1) (float4
+      // units f, F of them).  Threads split into nB blocks of bs consecutive segments x FP
+      // float4 columns (nB * FP <= 128): a thread loads its block's summaries for its f
+      // all at once (consecutive threads read consecutive float4s), composes them
+      // sequentially, and the block compositions are exchanged through shared memory;
+      // each thread then walks its segments again from its block's carry-in, writing
+      // each segment's start state (fp16, MMA layout, in that segment's CTA scale).
+      const int ns = fp.n_s;
+      const int f0 = (int)((long long)seg * 1024 / ns), f1 = (int)((long long)(seg + 1) * 1024 / ns);
+      const int F = f1 - f0;
+      int nB = kWG / (F > 0 ? F : 1);
+      nB = nB < 1 ? 1 : (nB > ns ? ns : nB);
+      if ((ns + nB - 1) / nB > kScanBlock) nB = (ns + kScanBlock - 1) / kScanBlock;
+      const int bs = (ns + nB - 1) / nB;
+      const int FP = kWG / nB;
+      const int bi = wtid / FP, fi = wtid % FP;
+      const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
+      unsigned int* ctr = fp.counters + (size_t)seq * 2;
+      const float* aggs = fp.agg + (size_t)seq * ns * kAggStride;
+      uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
+      float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
+      float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
+      float* segfac = reinterpret_cast<float*>(smem + kOffSst + 4096);   // [ns] start-state factors
+      const unsigned int target = (unsigned int)ns;
+      // failure injection: a segment withholds its arrival, and the waits give up early
+      const unsigned int dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
+      const uint64_t limit = dbg_us ? 1000ull * dbg_us : 1000000000ull;
+      const int loads = partial ? min(4, (cnt + 1) / 2) : 0;
+      bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
+      int issued = 0;
+      if (ok0) {
+        if (wtid == 0) {
+          // the second phase's first four pairs start loading now (every MMA of this
+          // CTA has completed, so all staging buffers are free; the Qh' and O_local
+          // tiles are written and fenced)
+          for (int q = 0; q < loads; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
+          issued = loads;
+          if (*(volatile unsigned int*)&hdr->dbg_skip_seg != (unsigned int)seg + 1u) red_release_add(ctr, 1u);
+          ok0 = wait_counter(ctr, target, ms, hdr, 0x601, limit);
         }
-        ms->seg_go = ok ? 1 : 0;
+        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
       }
-      named_sync(7, 4 * kWG);
-      const bool go = *(volatile int*)&ms->seg_go != 0;
-      if (go) {
-        const int kk = tid >> 3, v0 = 8 * (tid & 7);
-        const float* aggs = fp.agg + (size_t)seq * fp.n_s * kAggStride;
-        float x[8];
+      if (ok0) {
+        for (int sg = wtid; sg < ns; sg += kWG) segfac[sg] = __ldcg(aggs + (size_t)sg * kAggStride + 4096 + 64);
+        wg_sync(wg);
+        for (int base = f0; base < f1; base += FP) {
+          const int f = base + fi;
+          const bool act = bi < nB && f < f1;
+          const int kk = f >> 4;
+          float4 u[kScanBlock];
+          float dd[kScanBlock];
+          float4 X = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = 0.f;
-        // X <- 2^d_j X + U_j over j = 0 .. s-1, four summaries' loads in flight at a time
-        for (int j0 = 0; j0 < seg; j0 += 4) {
-          float4 ua[4], ub[4];
-          float dj[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const bool on = j0 + i < seg;
-            const float* a = aggs + (size_t)(on ? j0 + i : 0) * kAggStride;
-            ua[i] = __ldcg(reinterpret_cast<const float4*>(a + 8 * tid));
-            ub[i] = __ldcg(reinterpret_cast<const float4*>(a + 8 * tid + 4));
-            dj[i] = __ldcg(a + 4096 + kk);
+          for (int j = 0; j < kScanBlock; ++j) {
+            const int sg = s_lo + j;
+            const bool on = act && sg < s_hi;
+            const float* a2p = aggs + (size_t)(on ? sg : 0) * kAggStride;
+            u[j] = on ? __ldcg(reinterpret_cast<const float4*>(a2p) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            dd[j] = on ? __ldcg(a2p + 4096 + kk) : 0.f;
           }
+          // this block's transfer: state_after = D * state_before + U
+          float D = 1.f;
+          float4 U = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (j0 + i < seg) {
-              const float d = ex2(dj[i]);
-              x[0] = fmaf(d, x[0], ua[i].x); x[1] = fmaf(d, x[1], ua[i].y);
-              x[2] = fmaf(d, x[2], ua[i].z); x[3] = fmaf(d, x[3], ua[i].w);
-              x[4] = fmaf(d, x[4], ub[i].x); x[5] = fmaf(d, x[5], ub[i].y);
-              x[6] = fmaf(d, x[6], ub[i].z); x[7] = fmaf(d, x[7], ub[i].w);
+          for (int j = 0; j < kScanBlock; ++j) {
+            dd[j] = ex2(dd[j]);  // inactive entries: 2^0 = 1 with a zero summary
+            U = make_float4(fmaf(dd[j], U.x, u[j].x), fmaf(dd[j], U.y, u[j].y), fmaf(dd[j], U.z, u[j].z),
+                            fmaf(dd[j], U.w, u[j].w));
+            D *= dd[j];
+          }
+          if (nB > 1) {
+            if (bi < nB) {
+              xD[bi * FP + fi] = D;
+              xU[bi * FP + fi] = U;
+            }
+            wg_sync(wg);
+            for (int b2 = 0; b2 < bi && b2 < nB; ++b2) {
+              const float d2 = xD[b2 * FP + fi];
+              const float4 u2 = xU[b2 * FP + fi];
+              X = make_float4(fmaf(d2, X.x, u2.x), fmaf(d2, X.y, u2.y), fmaf(d2, X.z, u2.z), fmaf(d2, X.w, u2.w));
             }
           }
+          if (act) {
+            const int v0 = 4 * (f & 15);
+            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (v0 & 7) * 2;
+#pragma unroll
+            for (int j = 0; j < kScanBlock; ++j) {
+              const int sg = s_lo + j;
+              if (sg < s_hi) {
+                const float fs = segfac[sg];  // into segment sg's CTA scale
+                const uint2 w = make_uint2(pack_h2(X.x * fs, X.y * fs), pack_h2(X.z * fs, X.w * fs));
+                __stcg(reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(sst + (size_t)sg * 4096) + soff), w);
+                X = make_float4(fmaf(dd[j], X.x, u[j].x), fmaf(dd[j], X.y, u[j].y), fmaf(dd[j], X.z, u[j].z),
+                                fmaf(dd[j], X.w, u[j].w));
+              }
+            }
+          }
+          if (nB > 1) wg_sync(wg);  // the exchange slots are reused by the next column pass
         }
-        // row kk, columns v0 .. v0+7: one 16-byte piece of the 128-byte-swizzled start-state tile
-        const float f = ms->sc_sin;
-        const uint4 w = make_uint4(pack_h2(x[0] * f, x[1] * f), pack_h2(x[2] * f, x[3] * f),
-                                   pack_h2(x[4] * f, x[5] * f), pack_h2(x[6] * f, x[7] * f));
-        *reinterpret_cast<uint4*>(smem + kOffSst + kk * 128 + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4)) = w;
-        fence_proxy_async_smem();  // read by the second phase's MMAs
+        __threadfence();
+        wg_sync(wg);
+        if (wtid == 0) {
+          red_release_add(ctr + 1, 1u);
+          ok0 = wait_counter(ctr + 1, target, ms, hdr, 0x602, limit);
+        }
+        ok0 = wg_agree(wg, wtid, ok0, ms, slot);
       }
-      named_sync(7, 4 * kWG);
-      if (go) {
-        const int q = warp >> 2;
-        int slot2 = 0;
-        second_phase<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, q, tid - kWG * q, lane, seq, b, h, sp, slot2,
-                                             nonfinite);
+      if (ok0 && partial) {
+        // this segment's start state -> shared memory (already in the MMA layout), then
+        // the second phase on all four warpgroups
+        const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
+        uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
+        for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
+        fence_proxy_async_smem();
+        wg_sync(wg);
+        if (wtid == 0) mbar_arrive(&ms->p2_go);
+        second_phase<Tin, Tout, kDK, kBlock>(fp, ms, hdr, smem, tmem, wg, wtid, lane, seq, b, h, sp, slot, nonfinite);
+      } else if (wtid == 0) {
+        // giving up: this CTA's own bulk copies land before it leaves (they read the
+        // workspace only, so they complete on their own; the wait is bounded all the same)
+        for (int q = 0; q < issued; ++q)
+          for (int it = 0; it < 1000 && !mbar_wait_sleep(&ms->p2_full[q], 0u, 1000000u); ++it) {
+          }
       }
     }
   }
@@ -1905,7 +1955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __threadfence();
     const unsigned int done = atomicAdd(&hdr->ticket, 1u);
     if (done == (unsigned int)fp.grid - 1) {
-      for (int i = 0; i < fp.grid; ++i) fp.counters[i] = 0u;
+      for (int i = 0; i < 2 * fp.n_seq; ++i) fp.counters[i] = 0u;
       __threadfence();
       hdr->ticket = 0u;
     }
@@ -2154,6 +2204,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.hdr = w.hdr;
   fp.counters = w.counters;
   fp.agg = w.agg;
+  fp.sstart = w.sstart;
   fp.qhp = w.qhp;
   fp.olc = w.olc;
   fp.n_seq = pl.n_seq;
@@ -2179,8 +2230,8 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
     ++na;
   }
   // the prologue may overlap the previous launch's tail (every mode).  In SEGMENTED mode
-  // the CTAs of a sequence wait on the segments before them: the grid is at most one CTA
-  // per SM (kernel occupancy 1), so every CTA becomes resident once the previous grid has
+  // the CTAs of a sequence wait on one another: the grid is at most one CTA per SM
+  // (kernel occupancy 1), so every CTA becomes resident once the previous grid has
   // drained -- a later launch cannot take SMs before every CTA of this one has started
   // (griddepcontrol.launch_dependents fires per CTA) -- and every wait is bounded.
   attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -221,7 +221,8 @@ gtr_status_t gtr_gla_fwd_noalloc(const void *q, const void *k, const void *v,
  * on the fly instead of reading a log_gamma tensor (a quarter to a third of the bytes).
  *   gate_z  [B, L, gate_rank] fp32 (token m = y * grid_W + x, shared by the heads)
  *   gate_w2 [gate_rank, heads * d_k] fp32;  gate_b [heads * d_k] fp32
- *   gate_rank in {4, 8, 12, 16};  gate_tau > 0 (finite)
+ *   gate_rank 8 or 16 (the rows of z are then whole 32-byte pieces, which the tensor-memory
+ *   loads need);  gate_tau > 0 (finite)
  * When gate_z is NULL, log_gamma [B, L, heads, d_k] fp32 is read as in gtr_gla_fwd.
  *
  * RMSNORM + SILU OUTPUT GATE (when out_gate != NULL).  0539edu.com, appendix E.3.1: the

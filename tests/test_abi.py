@@ -135,8 +135,9 @@ def _block(**kw):
     (dict(lg=None), 1),                                               # no gates at all
     (dict(z=256, w2=256, b=256, rank=16), 1),                         # both gate sources
     (dict(lg=None, z=256, w2=None, b=256, rank=16), 1),               # factor missing
-    (dict(lg=None, z=256, w2=256, b=256, rank=6), 1),                 # rank not a multiple of 4
-    (dict(lg=None, z=256, w2=256, b=256, rank=20), 1),                # rank above 16
+    (dict(lg=None, z=256, w2=256, b=256, rank=4), 1),                 # ranks 8 and 16 only
+    (dict(lg=None, z=256, w2=256, b=256, rank=12), 1),
+    (dict(lg=None, z=256, w2=256, b=256, rank=20), 1),
     (dict(lg=None, z=256, w2=256, b=256, rank=16, tau=0.0), 1),       # tau must be positive
     (dict(lg=None, z=256, w2=256, b=256, rank=16, tau=float("inf")), 1),
     (dict(og=256, nw=None), 1),                                       # norm weight missing
