@@ -653,30 +653,17 @@ __device__ __forceinline__ uint32_t raw_off8(int row, int ch0) {
   return kDK == 64 ? sw_off8(row, ch0) : (uint32_t)(row * 64 + 2 * ch0);
 }
 
-// Largest |x| of the q and k elements a WG_A thread builds (rows row0 .. row0+3, channels
-// 32p + 4cc .. 32p + 4cc + 3 for the d_k / 32 passes p; raw tiles at qr / kr) and of the v
-// elements it converts, as bit patterns with the sign dropped (for non-negative fp16 and
-// bf16 values the integer order of the patterns is their numeric order), reduced over the
-// warp.  Out of line: first chunk only.
-template <int kDK>
-__device__ __noinline__ uint3 own_absmax_bits(const uint8_t* qr, const uint8_t* kr, const uint8_t* vt, int row0,
-                                              int cc, int wtid) {
-  uint32_t mq = 0, mk = 0, mv = 0;
-  for (int ps = 0; ps < kDK / 32; ++ps)
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t o = raw_off8<kDK>(row0 + i, 32 * ps + 4 * cc);
-      const uint2 a = *reinterpret_cast<const uint2*>(qr + o), c = *reinterpret_cast<const uint2*>(kr + o);
-      mq = __vmaxu2(__vmaxu2(mq, a.x & 0x7fff7fffu), a.y & 0x7fff7fffu);
-      mk = __vmaxu2(__vmaxu2(mk, c.x & 0x7fff7fffu), c.y & 0x7fff7fffu);
-    }
-  for (int i = wtid; i < kTile / 16; i += kWG) {
-    const uint4 x = *reinterpret_cast<const uint4*>(vt + 16 * i);
-    mv = __vmaxu2(__vmaxu2(mv, x.x & 0x7fff7fffu), x.y & 0x7fff7fffu);
-    mv = __vmaxu2(__vmaxu2(mv, x.z & 0x7fff7fffu), x.w & 0x7fff7fffu);
+// Largest |x| over `bytes` bytes of 16-bit values as a bit pattern with the sign dropped
+// (for non-negative fp16 and bf16 values the integer order of the patterns is their
+// numeric order), reduced over the calling warp; a warpgroup's 128 threads cover the tile.
+__device__ __forceinline__ uint32_t absmax_bits(const uint8_t* t, int bytes, int wtid) {
+  uint32_t m = 0;
+  for (int i = wtid; i < bytes / 16; i += kWG) {
+    const uint4 x = *reinterpret_cast<const uint4*>(t + 16 * i);
+    m = __vmaxu2(__vmaxu2(m, x.x & 0x7fff7fffu), x.y & 0x7fff7fffu);
+    m = __vmaxu2(__vmaxu2(m, x.z & 0x7fff7fffu), x.w & 0x7fff7fffu);
   }
-  return make_uint3(__reduce_max_sync(0xffffffffu, max(mq & 0xffffu, mq >> 16)),
-                    __reduce_max_sync(0xffffffffu, max(mk & 0xffffu, mk >> 16)),
-                    __reduce_max_sync(0xffffffffu, max(mv & 0xffffu, mv >> 16)));
+  return __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
 }
 
 // The q and k elements a WG_A thread builds, times the CTA's factors sq and sk, in place
@@ -1260,20 +1247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
       uint8_t* qr = kDK == 64 ? sb : sb + 3 * kTile + kRawQ;  // raw q, k
       uint8_t* kr = kDK == 64 ? sb + kTile : sb + 3 * kTile + kRawK;
-      if (n == 0) {
-        // ---- the CTA's input scale comes from its first chunk (warpgroup 0): the warps'
-        // largest |q|, |k|, |v| travel with the cumsum exchange below
-        const uint3 m = own_absmax_bits<kDK>(qr, kr, sb + 2 * kTile, row0, cc, wtid);
-        if (lane == 0) ms->smax[w4][0] = m.x, ms->smax[w4][1] = m.y, ms->smax[w4][2] = m.z;
-      } else if (n == 1) {  // warpgroup 1's first chunk: take the scale warpgroup 0 set
-        if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot, true)) {
-          alive = false;
-          break;
-        }
-        sq = ms->sc_in[0];
-        sk = ms->sc_in[1];
-        sv = ms->sc_in[2];
-      }
       // ---- in-chunk cumulative log2-gates in scan order: my 4 rows (written back over
       // the gates, still without the offset of the rows before them), a scan over the
       // warp's 4 row blocks, then over the 4 warps through shared memory (staged rows run
@@ -1334,27 +1307,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_float4(incl[ps][0], incl[ps][1], incl[ps][2], incl[ps][3]);
       }
       wg_sync(wg);
-      if (n == 0) {
-        // powers of two, so that scaling and undoing it are exact (every thread of the
-        // warpgroup derives the same factors; thread 0 publishes them to the other roles)
-        int e[3];
-#pragma unroll
-        for (int t = 0; t < 3; ++t) {
-          const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
-          e[t] = input_scale_exp(bits16_to_float<Tin>(m));
+      if (n == hh) {
+        // this warpgroup's first chunk: the CTA's input scale, which WG_C derives from the
+        // first chunk's raw tiles while the gates are summed (they are overwritten below)
+        if (!wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x305, slot, true)) {
+          alive = false;
+          break;
         }
-        sq = pow2f(e[0]);
-        sk = pow2f(e[1]);
-        sv = pow2f(e[2]);
-        if (wtid == 0) {
-          ms->sc_in[0] = sq;
-          ms->sc_in[1] = sk;
-          ms->sc_in[2] = sv;
-          ms->sc_out = pow2f(-(e[0] + e[1] + e[2])) * (kDK == 64 ? 1.f : 0.70710678118654752f);
-          ms->sc_spub = pow2f(-(e[1] + e[2]));
-          ms->sc_sin = pow2f(e[1] + e[2]);
-          mbar_arrive(&ms->scale_ready);
-        }
+        sq = ms->sc_in[0];
+        sk = ms->sc_in[1];
+        sv = ms->sc_in[2];
       }
       // a CTA with tiny inputs first scales the q and k elements this thread builds (the
       // CUDA-core scores below read them after a barrier)
@@ -1653,9 +1615,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
-    // the input scale (the outputs are stored in the inputs' scale; a sleeping wait: the
-    // first outputs come microseconds after the scale)
-    bool alive = wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x505, slot);
+    // ---- the CTA's input scale, from its first chunk's raw q, k, v tiles (WG_A waits for it
+    // before it overwrites them with its operands): powers of two that bring a tiny tile
+    // maximum into [1, 2), so that scaling and undoing it are exact
+    bool alive = wg_wait(wg, wtid, &ms->full[0], 0u, ms, hdr, 0x506, slot, true);
+    if (alive) {
+      const uint8_t* sb0 = smem + kOffStage;
+      const uint32_t m0 = absmax_bits(kDK == 64 ? sb0 : sb0 + 3 * kTile + kRawQ, 128 * kDK, wtid);
+      const uint32_t m1 = absmax_bits(kDK == 64 ? sb0 + kTile : sb0 + 3 * kTile + kRawK, 128 * kDK, wtid);
+      const uint32_t m2 = absmax_bits(sb0 + 2 * kTile, kTile, wtid);
+      if (lane == 0) ms->smax[wq][0] = m0, ms->smax[wq][1] = m1, ms->smax[wq][2] = m2;
+      wg_sync(wg);
+      if (wtid == 0) {
+        int e[3];
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
+          e[t] = input_scale_exp(bits16_to_float<Tin>(m));
+          ms->sc_in[t] = pow2f(e[t]);
+        }
+        ms->sc_out = pow2f(-(e[0] + e[1] + e[2])) * (kDK == 64 ? 1.f : 0.70710678118654752f);
+        ms->sc_spub = pow2f(-(e[1] + e[2]));
+        ms->sc_sin = pow2f(e[1] + e[2]);
+        mbar_arrive(&ms->scale_ready);
+      }
+      wg_sync(wg);  // (the factors are read by this warpgroup's epilogues)
+    }
     if (clus) {
       // the outputs stay in tensor memory until the start state is known: wait for their
       // last MMAs; then (segments s > 0) the chunks' Qh' tiles start loading into the idle
@@ -2229,14 +2214,16 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
     attr[na].val.clusterDim.z = 1;
     ++na;
   }
-  // the prologue may overlap the previous launch's tail (every mode).  In SEGMENTED mode
-  // the CTAs of a sequence wait on one another: the grid is at most one CTA per SM
-  // (kernel occupancy 1), so every CTA becomes resident once the previous grid has
-  // drained -- a later launch cannot take SMs before every CTA of this one has started
-  // (griddepcontrol.launch_dependents fires per CTA) -- and every wait is bounded.
-  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[na].val.programmaticStreamSerializationAllowed = 1;
-  ++na;
+  if (pl.mode == 1) {  // the CTAs of a sequence wait on one another (measured faster than
+    // a normal launch with programmatic dependent launch: 2048^2 58.5 against 62.9 us)
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  } else {  // the prologue may overlap the previous launch's tail
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, kerns[pl.mode], fp) != cudaSuccess) return GTR_ERR_CUDA;

@@ -1,8 +1,13 @@
 """Parity of the Spatial SwiGLU stencil (gtr_sswiglu_dwconv) with the fp64 oracle:
 SiLU(xg) * DWConv3x3(xv), zero padding, every dtype, ragged grids (tiles that cross the
-grid edge), with and without bias.  Bound: max |z - z_ref| <= tol * rms(z_ref), tol =
-1e-2 for 16-bit data (the output's own rounding is 2^-9 relative for bf16) and 1e-5 for
-fp32."""
+grid edge), with and without bias.
+
+Bound, derived from the arithmetic: the kernel reads the inputs exactly, computes the
+nine taps, the bias and SiLU in fp32 and rounds once to the output dtype, so per element
+    |z - z_ref| <= u_out * |z_ref| + 1e-5 * rms(z_ref)
+with u_out the output dtype's unit roundoff (2^-8 bf16, 2^-11 fp16, 2^-24 fp32) and the
+second term the fp32 arithmetic.  (Measured against rms(z_ref) alone, the bf16 rounding
+of the heavy-tailed product would exceed 1e-2 by itself: max |z| is 10-20 rms.)"""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +18,7 @@ from gtr_inputs import STENCILS, StencilWorkload, make_stencil_inputs
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"f32": 1e-5, "f16": 1e-2, "bf16": 1e-2}
+UNIT_ROUNDOFF = {"f32": 2.0 ** -24, "f16": 2.0 ** -11, "bf16": 2.0 ** -8}
 
 
 def check(s: StencilWorkload, seed: int):
@@ -24,8 +29,9 @@ def check(s: StencilWorkload, seed: int):
     torch.cuda.synchronize()
     o = out.to("cpu", torch.float64).numpy()
     assert np.isfinite(o).all()
-    err = float(np.abs(o - ref).max() / np.sqrt(np.mean(ref ** 2)))
-    assert err <= TOL[s.dtype], f"{s.name}: max err / rms = {err:.3e}"
+    bound = UNIT_ROUNDOFF[s.dtype] * np.abs(ref) + 1e-5 * np.sqrt(np.mean(ref ** 2))
+    worst = float((np.abs(o - ref) / bound).max())
+    assert worst <= 1.0, f"{s.name}: max |z - z_ref| / bound = {worst:.3f}"
 
 
 @pytest.mark.parametrize("name", list(STENCILS))
