@@ -112,8 +112,8 @@ static_assert(4 * 64 <= kColO, "second-phase slots (M = 128, 64 columns each) re
 constexpr size_t kMaxSegCtas = 256;  // CTAs of one launch in SEGMENTED mode (>= the SM count)
 constexpr size_t kCounterBytes = 2 * kMaxSegCtas * sizeof(unsigned int);
 constexpr int kScanBlock = 8;       // segments one WG_C thread composes in registers
-// per-segment summary: U_seg [64][64] fp32, the log2 decay [64], the start-state factor, padding
-constexpr size_t kAggStride = 4096 + 128;
+// per-segment summary: U_seg [64][64] fp32 and the log2 decay [64]
+constexpr size_t kAggStride = 4096 + 64;
 static_assert(sizeof(WsHeader) + kCounterBytes == kWsPrefixBytes, "counters fill the shared workspace prefix");
 
 // floor(n / d) for 0 <= n < 2^31 by one wide multiply and a shift: with l = ceil(log2 d)
@@ -143,7 +143,7 @@ struct alignas(64) FusedParams {
   WsHeader* hdr;
   unsigned int* counters;  // SEGMENTED: [n_seq][2] arrival counters, monotonic within a call, zero between calls
   float* agg;              // [n_seq][n_s][kAggStride] segment summaries (U_seg, log2 decay, start-state factor)
-  uint16_t* sstart;        // [n_seq][n_s][64*64] segment start states, fp16, MMA layout
+  float* sstart;           // [n_seq][n_s][64*64] segment start states, fp32, row-major, inputs' scale
   uint16_t* qhp;           // [n_seq][Nc][64*64] Qh' per chunk, fp16, MMA layout
   uint16_t* olc;           // [n_seq][Nc][64][64] outputs from a zero segment start, fp16
   int n_seq, n_s, Nc, mode;  // mode 0 = STREAM, 1 = SEGMENTED, 2 = CLUSTER
@@ -210,6 +210,7 @@ struct Misc {
   alignas(16) float nw[64];       // output gate: RMSNorm weight
   int zrow[2][64];                // producer: z row b*L + m of each chunk row (gathers; -1 past the end)
   int abort;
+  unsigned int dbg_skip, dbg_us;  // failure injection (workspace header), read once at the start
   int go[4][2];          // per-warpgroup wait decisions, alternating slots
   int fb[kStages];       // stage -> scores from the CUDA cores
   alignas(16) float dseg[64];  // CLUSTER: this segment's log2 decay per key channel (read by the cluster)
@@ -906,6 +907,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ms->tmem_base;
   // every global access of this grid comes after the previous grid in the stream has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (segm && tid == 0) {  // failure injection marks of the workspace (zero: off)
+    ms->dbg_skip = *(volatile unsigned int*)&hdr->dbg_skip_seg;
+    ms->dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
+  }
   // CLUSTER: a CTA's shared memory is written by the others only once every CTA of the
   // cluster has started (the matching wait comes before the first remote access)
   if (clus) cluster_arrive_relaxed();
@@ -1222,20 +1227,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int slot = 0;
     bool alive = true;
     float sq = 1.f, sk = 1.f, sv = 1.f;  // this CTA's input scale factors (set at the first chunk)
-    if (hh == 0 && (lowrank || gated)) {
-      // warpgroup 0: this head's gate-producer columns and bias (zero past d_k) and the output
-      // norm weight into shared memory; the other roles read them after the scale barrier
-      // (warpgroup 1, WG_B, WG_C) or a CTA barrier
-      if (lowrank) {
-        const int ld = p.heads * kDK;
-        for (int i = wtid; i < 16 * 64; i += kWG) {
-          const int j = i >> 6, c = i & 63;
-          ms->w2s[j][c] = (j < p.grank && c < kDK) ? __ldg(p.gw2 + (long long)j * ld + h * kDK + c) : 0.f;
-        }
-        if (wtid < 64) ms->bs[wtid] = wtid < kDK ? __ldg(p.gb + h * kDK + wtid) : 0.f;
+    if (lowrank) {
+      // both warpgroups: this head's gate-producer columns and bias (zero past d_k) into
+      // shared memory, then a barrier of the two (named barrier 5, 256 threads)
+      const int ld = p.heads * kDK, t2 = tid;  // tid < 256 here
+      for (int i = t2; i < 16 * 64; i += 2 * kWG) {
+        const int j = i >> 6, c = i & 63;
+        ms->w2s[j][c] = (j < p.grank && c < kDK) ? __ldg(p.gw2 + (long long)j * ld + h * kDK + c) : 0.f;
       }
-      if (gated && wtid < 64) ms->nw[wtid] = __ldg(p.onorm_w + wtid);
-      wg_sync(wg);
+      if (t2 < 64) ms->bs[t2] = t2 < kDK ? __ldg(p.gb + h * kDK + t2) : 0.f;
+      asm volatile("bar.sync 5, 256;" ::: "memory");
     }
     for (int n = hh; n < cnt; n += 2) {
       const int st = n % kStages;
@@ -1600,7 +1601,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mine[4096 + r0] = a2r0;
         mine[4096 + r1] = a2r1;
       }
-      if (wtid == 0) mine[4096 + 64] = ms->sc_sin;
       __threadfence();
       wg_sync(wg);
       if (wtid == 0) mbar_arrive(&ms->agg_pub);
@@ -1615,6 +1615,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     uint8_t* wstage = smem + kOffStg + wq * 32 * 128;  // this warp's output staging tile
     int slot = 0;
+    // the output gate's norm weight (read by this warpgroup's epilogues, and by the others'
+    // after barriers that follow this warpgroup's)
+    if (gated && wtid < 64) ms->nw[wtid] = __ldg(p.onorm_w + wtid);
     // ---- the CTA's input scale, from its first chunk's raw q, k, v tiles (WG_A waits for it
     // before it overwrites them with its operands): powers of two that bring a tiny tile
     // maximum into [1, 2), so that scaling and undoing it are exact
@@ -1704,13 +1707,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s_lo = bi * bs, s_hi = min(ns, s_lo + bs);
       unsigned int* ctr = fp.counters + (size_t)seq * 2;
       const float* aggs = fp.agg + (size_t)seq * ns * kAggStride;
-      uint16_t* sst = fp.sstart + (size_t)seq * ns * 4096;
+      float* sst = fp.sstart + (size_t)seq * ns * 4096;
       float* xD = reinterpret_cast<float*>(smem + kOffSst);              // [128] block decays
       float4* xU = reinterpret_cast<float4*>(smem + kOffSst + 4 * kWG);  // [128] block summaries
-      float* segfac = reinterpret_cast<float*>(smem + kOffSst + 4096);   // [ns] start-state factors
       const unsigned int target = (unsigned int)ns;
       // failure injection: a segment withholds its arrival, and the waits give up early
-      const unsigned int dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
+      const unsigned int dbg_us = ms->dbg_us;
       const uint64_t limit = dbg_us ? 1000ull * dbg_us : 1000000000ull;
       const int loads = partial ? min(4, (cnt + 1) / 2) : 0;
       bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
@@ -1722,14 +1724,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // tiles are written and fenced)
           for (int q = 0; q < loads; ++q) p2_load(fp, ms, smem, seq, sp, q, q);
           issued = loads;
-          if (*(volatile unsigned int*)&hdr->dbg_skip_seg != (unsigned int)seg + 1u) red_release_add(ctr, 1u);
+          if (ms->dbg_skip != (unsigned int)seg + 1u) red_release_add(ctr, 1u);
           ok0 = wait_counter(ctr, target, ms, hdr, 0x601, limit);
         }
         ok0 = wg_agree(wg, wtid, ok0, ms, slot);
       }
       if (ok0) {
-        for (int sg = wtid; sg < ns; sg += kWG) segfac[sg] = __ldcg(aggs + (size_t)sg * kAggStride + 4096 + 64);
-        wg_sync(wg);
         for (int base = f0; base < f1; base += FP) {
           const int f = base + fi;
           const bool act = bi < nB && f < f1;
@@ -1768,15 +1768,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (act) {
-            const int v0 = 4 * (f & 15);
-            const uint32_t soff = (uint32_t)kk * 128u + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) + (v0 & 7) * 2;
 #pragma unroll
             for (int j = 0; j < kScanBlock; ++j) {
               const int sg = s_lo + j;
-              if (sg < s_hi) {
-                const float fs = segfac[sg];  // into segment sg's CTA scale
-                const uint2 w = make_uint2(pack_h2(X.x * fs, X.y * fs), pack_h2(X.z * fs, X.w * fs));
-                __stcg(reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(sst + (size_t)sg * 4096) + soff), w);
+              if (sg < s_hi) {  // segment sg's start state, fp32 in the inputs' scale
+                __stcg(reinterpret_cast<float4*>(sst + (size_t)sg * 4096) + f, X);
                 X = make_float4(fmaf(dd[j], X.x, u[j].x), fmaf(dd[j], X.y, u[j].y), fmaf(dd[j], X.z, u[j].z),
                                 fmaf(dd[j], X.w, u[j].w));
               }
@@ -1793,11 +1789,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok0 = wg_agree(wg, wtid, ok0, ms, slot);
       }
       if (ok0 && partial) {
-        // this segment's start state -> shared memory (already in the MMA layout), then
-        // the second phase on all four warpgroups
-        const uint4* src = reinterpret_cast<const uint4*>(sst + (size_t)seg * 4096);
-        uint4* dst = reinterpret_cast<uint4*>(smem + kOffSst);
-        for (int i = wtid; i < kTile / 16; i += kWG) dst[i] = __ldcg(src + i);
+        // this segment's start state -> shared memory: into this CTA's scale, fp16, the MMA
+        // layout (128-byte swizzle), then the second phase on all four warpgroups
+        const float4* src = reinterpret_cast<const float4*>(sst + (size_t)seg * 4096);
+        const float fs = ms->sc_sin;
+        for (int i = wtid; i < 1024; i += kWG) {
+          const float4 x = __ldcg(src + i);
+          const int kk = i >> 4, v0 = 4 * (i & 15);
+          *reinterpret_cast<uint2*>(smem + kOffSst + kk * 128 + ((((uint32_t)v0 >> 3) ^ ((uint32_t)kk & 7u)) << 4) +
+                                    (v0 & 7) * 2) = make_uint2(pack_h2(x.x * fs, x.y * fs), pack_h2(x.z * fs, x.w * fs));
+        }
         fence_proxy_async_smem();
         wg_sync(wg);
         if (wtid == 0) mbar_arrive(&ms->p2_go);
