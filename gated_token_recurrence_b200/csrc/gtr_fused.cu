@@ -14,7 +14,7 @@ size_t segmented_tile_bytes(const Problem& p) {
 
 size_t fused_workspace_bytes(const Problem& p) {
   const size_t segs = seg_capacity(p);
-  size_t b = sizeof(WsHeader) + kCounterBytes + segs * kAggStride * sizeof(float) + segs * 4096 * sizeof(float);
+  size_t b = sizeof(WsHeader) + kCounterBytes + segs * kAggStride * sizeof(float) + segs * 4096 * sizeof(uint16_t);
   b = (b + 1023) & ~size_t(1023);  // 1 KB-aligned tiles for the bulk copies
   return b + 2 * segmented_tile_bytes(p);
 }
@@ -29,8 +29,8 @@ FusedWorkspace fused_workspace_carve(void* ws, const Problem& p) {
   base += kCounterBytes;
   w.agg = reinterpret_cast<float*>(base);
   base += segs * kAggStride * sizeof(float);
-  w.sstart = reinterpret_cast<float*>(base);
-  base += segs * 4096 * sizeof(float);
+  w.sstart = reinterpret_cast<uint16_t*>(base);
+  base += segs * 4096 * sizeof(uint16_t);
   const size_t used = (size_t)(base - reinterpret_cast<uint8_t*>(ws));
   base = reinterpret_cast<uint8_t*>(ws) + ((used + 1023) & ~size_t(1023));
   const size_t tiles = segmented_tile_bytes(p);

@@ -22,7 +22,7 @@ struct FusedWorkspace {
   WsHeader* hdr;
   unsigned int* counters;  // per-sequence arrival counters (zero between calls)
   float* agg;              // per-segment summaries
-  float* sstart;           // per-segment start states (fp32, row-major, in the inputs' scale)
+  uint16_t* sstart;        // per-segment start states (fp16, MMA layout, their CTA's scale)
   uint16_t* qhp;           // segmented mode: per-chunk Qh' tiles (fp16, MMA layout)
   uint16_t* olc;           // segmented mode: per-chunk outputs from a zero segment start (fp16)
 };
