@@ -1269,6 +1269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* G = reinterpret_cast<float*>(sb + 3 * kTile);
       uint8_t* qr = kDK == 64 ? sb : sb + 3 * kTile + kRawQ;  // raw q, k
       uint8_t* kr = kDK == 64 ? sb + kTile : sb + 3 * kTile + kRawK;
+      if (n == 0) {
+        // the CTA's first chunk: its largest |q|, |k|, |v| per warp (published by the
+        // barrier after the gate sums, before any tile is overwritten)
+        const uint32_t m0 = absmax_bits(qr, 128 * kDK, wtid), m1 = absmax_bits(kr, 128 * kDK, wtid);
+        const uint32_t m2 = absmax_bits(sb + 2 * kTile, kTile, wtid);
+        if (lane == 0) ms->smax[w4][0] = m0, ms->smax[w4][1] = m1, ms->smax[w4][2] = m2;
+      }
       // ---- in-chunk cumulative log2-gates in scan order: my 4 rows (written back over
       // the gates, still without the offset of the rows before them), a scan over the
       // warp's 4 row blocks, then over the 4 warps through shared memory (staged rows run
@@ -1329,9 +1336,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_float4(incl[ps][0], incl[ps][1], incl[ps][2], incl[ps][3]);
       }
       wg_sync(wg);
-      if (n == hh) {
-        // this warpgroup's first chunk: the CTA's input scale, which WG_C derives from the
-        // first chunk's raw tiles while the gates are summed (they are overwritten below)
+      if (n == 0) {
+        // the CTA's input scale: powers of two that bring a tiny first-chunk maximum into
+        // [1, 2), so that scaling and undoing it are exact; every thread derives it from the
+        // four warps' maxima, thread 0 publishes it for the other warpgroups
+        int e[3];
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
+          e[t] = input_scale_exp<Tin>(bits16_to_float<Tin>(m));
+        }
+        sq = pow2f(e[0]);
+        sk = pow2f(e[1]);
+        sv = pow2f(e[2]);
+        if (wtid == 0) {
+          ms->sc_in[0] = sq;
+          ms->sc_in[1] = sk;
+          ms->sc_in[2] = sv;
+          ms->sc_out = pow2f(-(e[0] + e[1] + e[2])) * (kDK == 64 ? 1.f : 0.70710678118654752f);
+          ms->sc_spub = pow2f(-(e[1] + e[2]));
+          ms->sc_sin = pow2f(e[1] + e[2]);
+          mbar_arrive(&ms->scale_ready);
+        }
+      } else if (n == hh) {
+        // the other operand warpgroup's first chunk: the scale WG_A0 derived
         const float4 f = take_input_scale(wg, wtid, ms, hdr, slot);
         slot ^= 1;
         if (f.w == 0.f) {
@@ -1642,36 +1670,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the output gate's norm weight (read by this warpgroup's epilogues, and by the others'
     // after barriers that follow this warpgroup's)
     if (gated && wtid < 64) ms->nw[wtid] = __ldg(p.onorm_w + wtid);
-    // ---- the CTA's input scale, from its first chunk's raw q, k, v tiles (WG_A waits for it
-    // before it overwrites them with its operands): powers of two that bring a tiny tile
-    // maximum into [1, 2), so that scaling and undoing it are exact
-    bool alive = wg_wait(wg, wtid, &ms->full[0], 0u, ms, hdr, 0x506, slot, true);
-    if (alive) {
-      const uint8_t* sb0 = smem + kOffStage;
-      const uint32_t m0 = absmax_bits(kDK == 64 ? sb0 : sb0 + 3 * kTile + kRawQ, 128 * kDK, wtid);
-      const uint32_t m1 = absmax_bits(kDK == 64 ? sb0 + kTile : sb0 + 3 * kTile + kRawK, 128 * kDK, wtid);
-      const uint32_t m2 = absmax_bits(sb0 + 2 * kTile, kTile, wtid);
-      if (lane == 0) ms->smax[wq][0] = m0, ms->smax[wq][1] = m1, ms->smax[wq][2] = m2;
-      wg_sync(wg);
-      if (wtid == 0) {
-        int e[3];
-#pragma unroll
-        for (int t = 0; t < 3; ++t) {
-          const unsigned int m = max(max(ms->smax[0][t], ms->smax[1][t]), max(ms->smax[2][t], ms->smax[3][t]));
-          e[t] = input_scale_exp<Tin>(bits16_to_float<Tin>(m));
-          ms->sc_in[t] = pow2f(e[t]);
-        }
-        ms->sc_out = pow2f(-(e[0] + e[1] + e[2])) * (kDK == 64 ? 1.f : 0.70710678118654752f);
-        ms->sc_spub = pow2f(-(e[1] + e[2]));
-        ms->sc_sin = pow2f(e[1] + e[2]);
-        mbar_arrive(&ms->scale_ready);
-        if (segm) {  // failure injection marks of the workspace (zero: off), read by this warpgroup
-          ms->dbg_skip = *(volatile unsigned int*)&hdr->dbg_skip_seg;
-          ms->dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
-        }
-      }
-      wg_sync(wg);  // (the factors are read by this warpgroup's epilogues)
+    if (segm && wtid == 0) {  // failure injection marks of the workspace (zero: off), read by this warpgroup
+      ms->dbg_skip = *(volatile unsigned int*)&hdr->dbg_skip_seg;
+      ms->dbg_us = *(volatile unsigned int*)&hdr->dbg_wait_us;
     }
+    // the CTA's input scale (WG_A0 derives it from the first chunk; the outputs go back to
+    // the inputs' scale); the wait's barrier also publishes the marks above
+    bool alive = wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x506, slot);
     if (clus) {
       // the outputs stay in tensor memory until the start state is known: wait for their
       // last MMAs; then (segments s > 0) the chunks' Qh' tiles start loading into the idle
