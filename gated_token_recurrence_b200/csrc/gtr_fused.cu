@@ -9,7 +9,7 @@ namespace gtr {
 // Per-chunk tiles of the second phase (Qh' and O_local, fp16): only when sequences may
 // be split over CTAs.
 size_t segmented_tile_bytes(const Problem& p) {
-  return seg_capacity(p) ? (size_t)p.B * p.heads * p.n_chunks() * 4096 * sizeof(uint16_t) : 0;
+  return seg_capacity(p) ? (size_t)p.B * p.heads * max_fused_chunks(p) * 4096 * sizeof(uint16_t) : 0;
 }
 
 size_t fused_workspace_bytes(const Problem& p) {

@@ -156,7 +156,17 @@ struct alignas(64) FusedParams {
   int lowrank;             // 1: the log-gates come from the low-rank producer (z tiles, p.gw2, p.gb)
   float gtau_inv;          // 1 / tau of the gate producer
   int gated;               // 1: RMSNorm + SiLU output gate on the final outputs (p.ogate, p.onorm_w)
+  int lines, len;          // 1: line chunks of lines `len` cells long (0: contiguous chunks)
 };
+
+// Chunk c, offset r (0..63) of its scan positions -> scan position s.  Contiguous chunks
+// cover scan positions 64c .. 64c + 63; a line chunk covers grid line c (a row for the
+// row directions, a column for the column ones), len < 64 cells, zero-padded past the
+// line end.  False past the sequence or the line end.
+__device__ __forceinline__ bool chunk_scan_pos(const FusedParams& fp, int c, int r, long long L, long long& s) {
+  s = (long long)c * (fp.lines ? fp.len : kChunk) + r;
+  return fp.lines ? r < fp.len : s < L;
+}
 
 // Scan position s (< L < 2^31) -> token index y*W + x: the direction remap (rows top to
 // bottom, left to right or right to left; columns left to right, top to bottom or bottom
@@ -802,10 +812,10 @@ __device__ __forceinline__ void second_phase_body(const FusedParams& fp, Misc* m
     if (!wg_wait(q, wtid, &ms->p2_mma[q], (uint32_t)u & 1u, ms, hdr, 0x720u + q, slot)) return;
     tc_fence_after();
     const int ci = 2 * m2 + (wq >> 1), row = 32 * (wq & 1) + lane;
-    const long long s = (long long)(sp.c0 + ci) * kChunk + (fp.rev ? 63 - row : row);
+    long long s = 0;
+    const bool valid = ci < cnt && chunk_scan_pos(fp, sp.c0 + ci, fp.rev ? 63 - row : row, L, s);
     const uint8_t* olc_rows = sbuf + kP2Olc + (wq >> 1) * kTile + 32 * (wq & 1) * 128;
     // fp32 staging over the pair's Qh' (its MMA has completed)
-    const bool valid = ci < cnt && s < L;
     if (kBlock && fp.gated)
       gated_rows<Tout, Tin>(dq + ((uint32_t)(32 * wq) << 16), olc_rows + lane * 128, out_row<Tout>(fp, b, h, valid, s),
                             gate_row<Tin>(fp, b, h, valid, s), ms->nw, fp.p.oeps, sbuf + wq * 4096, lane, nf,
@@ -958,7 +968,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* kd = kDK == 64 ? sb + kTile : sb + 3 * kTile + kRawK;
           mbar_arrive_expect_tx(&ms->full[st], chunk_load_bytes<kDK>(fp, lowrank));
           const long long s0 = (long long)c * kChunk;
-          if (p.direction <= GTR_R2L) {
+          if (fp.lines) {
+            // line chunk: the 64 cells of grid line c from o0 (memory order along the line);
+            // cells past either end of the line read as zeros (k = v = 0 and log gamma = 0
+            // there: the state passes such rows unchanged)
+            const int o0 = kRev ? fp.len - kChunk : 0;
+            const int cx = p.direction <= GTR_R2L ? o0 : c, cy = p.direction <= GTR_R2L ? c : o0;
+            tma_load_5d(qd, &fp.tq, &ms->full[st], 0, h, cx, cy, b);
+            tma_load_5d(kd, &fp.tk, &ms->full[st], 0, h, cx, cy, b);
+            tma_load_5d(sb + 2 * kTile, &fp.tv, &ms->full[st], 0, h, cx, cy, b);
+            tma_load_5d(sb + 3 * kTile, &fp.tg, &ms->full[st], 0, h, cx, cy, b);
+          } else if (p.direction <= GTR_R2L) {
             // row view: 64 consecutive grid cells m (right-to-left: one image row)
             long long m0 = s0;
             if (p.direction == GTR_R2L) {
@@ -1700,8 +1720,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wg_wait(wg, wtid, &ms->o_full[pr % kOPairs], ph_use<kOPairs>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
         const int ci = 2 * pr + tsel;
-        const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
-        const bool valid = ci < cnt && s < L;
+        long long s = 0;
+        const bool valid = ci < cnt && chunk_scan_pos(fp, sp.c0 + ci, kRev ? 63 - trow : trow, L, s);
         const uint32_t src = tl + kColO + 64u * (uint32_t)(pr % kOPairs);
         if (partial) {
           uint8_t* od = valid ? reinterpret_cast<uint8_t*>(fp.olc + ((size_t)seq * fp.Nc + sp.c0 + ci) * 4096) + trow * 128
@@ -1959,8 +1979,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (seg > 0 && !wg_wait(q, wtid, &ms->corr_done[pr], 0u, ms, hdr, 0x531, slot)) break;
         tc_fence_after();
         const int ci = 2 * pr + tsel;
-        const long long s = (long long)(sp.c0 + ci) * kChunk + (kRev ? 63 - trow : trow);
-        const bool valid = ci < cnt && s < L;
+        long long s = 0;
+        const bool valid = ci < cnt && chunk_scan_pos(fp, sp.c0 + ci, kRev ? 63 - trow : trow, L, s);
         if (gated)
           gated_rows<Tout, Tin>(tl + kColO + 64u * (uint32_t)pr, nullptr, out_row<Tout>(fp, b, h, valid, s),
                                 gate_row<Tin>(fp, b, h, valid, s), ms->nw, fp.p.oeps, wstage, lane, nonfinite,
@@ -2009,15 +2029,24 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // is 64 consecutive scan positions of one (batch, head): the row view [B][L][nh][d] with a
 // box of 64 cells m, or the column view with a box of 64 rows y of one column x.  nh is the
 // heads dimension (1 for a per-token tensor), d the channels (d * esize a multiple of 16).
+// rowline: the row-line view [B][H][W][nh][d] with a box of 64 consecutive x of one row y
+// (line chunks of the row directions: cells past the row's ends read as zeros).
 bool make_chunk_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, const Problem& p,
-                    bool column, bool swizzle, int d, int nh) {
+                    bool column, bool swizzle, int d, int nh, bool rowline = false) {
   auto enc = get_encode();
   if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u)) return false;
   const cuuint64_t e = (cuuint64_t)esize, hd = (cuuint64_t)nh, dd = (cuuint64_t)d;
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle sw = swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   CUresult r;
-  if (!column) {
+  if (rowline) {
+    cuuint64_t dims[5] = {dd, hd, (cuuint64_t)p.W, (cuuint64_t)p.H, (cuuint64_t)p.B};
+    cuuint64_t strides[4] = {dd * e, hd * dd * e, (cuuint64_t)p.W * hd * dd * e,
+                             (cuuint64_t)p.H * p.W * hd * dd * e};
+    cuuint32_t box[5] = {(cuuint32_t)d, 1, 64, 1, 1};
+    r = enc(m, dt, 5, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else if (!column) {
     cuuint64_t dims[4] = {dd, hd, (cuuint64_t)p.L(), (cuuint64_t)p.B};
     cuuint64_t strides[3] = {dd * e, hd * dd * e, (cuuint64_t)p.L() * hd * dd * e};
     cuuint32_t box[4] = {(cuuint32_t)d, 1, 64, 1};
@@ -2054,12 +2083,46 @@ struct Plan {
   int mode, n_seq, n_s, grid;
 };
 
+// Line chunks for directions whose 64 consecutive scan positions are not one box (right-
+// to-left rows, or columns, not a multiple of 64 long): one grid line a chunk, zero-padded
+// past the line end, each one TMA box per tensor, instead of contiguous chunks staged by 64
+// single-row gathers.  Taken for lines of 39 to 63 cells (the padding keeps at least 60%
+// of the staged rows) and at most 64 lines, where a sequence's few chunks leave the
+// gathers' issue time on the critical path (a 40 x 40 grid: 40 line chunks beat 25
+// gathered ones).  More chunks were measured slower than the gathers, which then overlap
+// with the work of the chunks before them (the 48-cell columns of a 48 x 80 grid: 80
+// chunks instead of 60; its 80-cell rows, two chunks a line: 96).  Not with the low-rank
+// gate producer: a zero z row would not give a gate of 1.
+bool use_lines(const Problem& p) {
+  if (p.gz != nullptr || p.direction == GTR_L2R) return false;
+  const bool column = p.direction >= GTR_T2B;
+  const int len = column ? p.H : p.W, lines = column ? p.W : p.H;
+  return len >= 39 && len < 64 && lines <= 64;
+}
+// Chunks of one sequence on the fused path, for the problem's direction.
+int fused_chunks(const Problem& p) {
+  if (!use_lines(p)) return p.n_chunks();
+  return p.direction >= GTR_T2B ? p.W : p.H;
+}
+// The most chunks of one sequence over the four directions (the workspace query takes no
+// direction).
+int max_fused_chunks(const Problem& p) {
+  int m = p.n_chunks();
+  for (int d = GTR_L2R; d <= GTR_B2T; ++d) {
+    Problem q = p;
+    q.direction = d;
+    q.gz = nullptr;
+    const int c = fused_chunks(q);
+    if (c > m) m = c;
+  }
+  return m;
+}
+
 // Length-aware plan: many sequences -> one CTA each (STREAM); few sequences -> each is
 // split into n_s segments, one CTA each, so that the launch fills the SMs (SEGMENTED).
-Plan make_plan(const Problem& p, int sms) {
+Plan make_plan(const Problem& p, int Nc, int sms) {
   Plan pl;
   pl.n_seq = p.B * p.heads;
-  const int Nc = p.n_chunks();
   const int cap = sms < (int)kMaxSegCtas ? sms : (int)kMaxSegCtas;
   if (pl.n_seq * 2 > cap || Nc <= 1) {
     pl.mode = 0;
@@ -2150,8 +2213,12 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   // (top-to-bottom / bottom-to-top when columns hold whole chunks)
   fp.rev = (p.direction == GTR_R2L || p.direction == GTR_B2T) ? 1 : 0;
   const bool column = p.direction >= GTR_T2B;
-  const bool one_box = p.direction == GTR_L2R || (p.direction == GTR_R2L && p.W % 64 == 0) ||
+  const bool lines = use_lines(p);
+  fp.lines = lines ? 1 : 0;
+  fp.len = column ? p.H : p.W;
+  const bool one_box = lines || p.direction == GTR_L2R || (p.direction == GTR_R2L && p.W % 64 == 0) ||
                        (column && p.H % 64 == 0);
+  const bool rowline = lines && !column;  // (line chunks of the column directions use the column view)
   const CUtensorMapDataType dt16 =
       std::is_same<Tin, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   // optional pieces of the GTR block: the low-rank gate producer (z tiles instead of the
@@ -2162,13 +2229,15 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   // q, k: 128-byte swizzle (d_k = 64; built in place), or dense rows (d_k = 32)
   const bool swqk = kDK == 64;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  fp.tma = one_box && make_chunk_map(&fp.tq, p.q, dt16, 2, p, column, swqk, kDK, p.heads) &&
-                   make_chunk_map(&fp.tk, p.k, dt16, 2, p, column, swqk, kDK, p.heads) &&
-                   make_chunk_map(&fp.tv, p.v, dt16, 2, p, column, true, 64, p.heads) &&
+  fp.tma = one_box && make_chunk_map(&fp.tq, p.q, dt16, 2, p, column, swqk, kDK, p.heads, rowline) &&
+                   make_chunk_map(&fp.tk, p.k, dt16, 2, p, column, swqk, kDK, p.heads, rowline) &&
+                   make_chunk_map(&fp.tv, p.v, dt16, 2, p, column, true, 64, p.heads, rowline) &&
                    (fp.lowrank ? make_chunk_map(&fp.tz, p.gz, f32, 4, p, column, false, p.grank, 1)
-                               : make_chunk_map(&fp.tg, p.log_gamma, f32, 4, p, column, false, kDK, p.heads))
+                               : make_chunk_map(&fp.tg, p.log_gamma, f32, 4, p, column, false, kDK, p.heads, rowline))
                ? 1
                : 0;
+  if (!fp.tma) fp.lines = 0;  // (no box view: contiguous chunks by gathers)
+  const int Nc = fp.lines ? fused_chunks(p) : p.n_chunks();
   fp.divW = make_fastdiv((uint32_t)p.W);
   fp.divH = make_fastdiv((uint32_t)p.H);
   if (!fp.tma) {  // other chunks: 4-row gathers from [B*L*heads][d] row views
@@ -2203,12 +2272,11 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
         return GTR_ERR_CUDA;
     configured[ckind].fetch_or(1ull << dev);
   }
-  Plan pl = make_plan(p, device_sms());
+  Plan pl = make_plan(p, Nc, device_sms());
   if (pl.mode == 1 && force_mode < 0) {
     // short sequences: one cluster per sequence (the largest size the device holds for
     // every sequence at once), at most kClusterChunks chunks per CTA; then the fewest
     // CTAs that keep the longest run
-    const int Nc = p.n_chunks();
     int best_k = kClusterChunks + 1;
     for (int cs = kMaxCluster; cs >= 2; --cs) {
       if (max_active_clusters(kerns[2], dev, kind, cs) < pl.n_seq) continue;
@@ -2238,7 +2306,7 @@ gtr_status_t launch_fused_typed(const Problem& p, void* ws, cudaStream_t stream,
   fp.olc = w.olc;
   fp.n_seq = pl.n_seq;
   fp.n_s = pl.n_s;
-  fp.Nc = p.n_chunks();
+  fp.Nc = Nc;
   fp.mode = pl.mode;
   fp.grid = pl.grid;
   // the score factor 2^-A of a chunk stays below 2^11.5 (about e^8): Kh and the

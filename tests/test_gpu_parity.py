@@ -364,6 +364,30 @@ def test_short_sequences_over_clusters_of_every_size(shape, dtype):
         check(w, d, seed=31 + d, path="fused")
 
 
+# Lines of 39 to 63 cells in a direction whose chunks are not one box (right-to-left rows,
+# columns) are staged one line a chunk, zero-padded past the line end: every line length
+# at the edges of that range and between, reversed and forward, in each plan (one cluster
+# a sequence, segments over many CTAs, one CTA a sequence), both input dtypes.
+LINE_SHAPES = [
+    (2, 3, 39, 63),    # rows of 63 (right-to-left), columns of 39
+    (1, 2, 63, 45),    # columns of 63, rows of 45
+    (3, 1, 47, 52),    # three sequences of a batch
+    (8, 6, 40, 52),    # 48 sequences: segments over many CTAs
+    (5, 6, 45, 39),    # 30 sequences: segments over many CTAs, other line lengths
+    (1, 2, 200, 40),   # 200 rows of 40: contiguous chunks by gathers (too many lines)
+]
+
+
+@pytest.mark.parametrize("path", ["fused", "fused_sequential"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("shape", LINE_SHAPES)
+def test_line_chunks_match_the_oracle(shape, dtype, path):
+    B, heads, H, W = shape
+    w = Workload("lines", B=B, heads=heads, H=H, W=W, dtype=dtype, scale=0.5, index=9)
+    for d in range(4):
+        check(w, d, 7000 + 10 * H + W + d, path)
+
+
 # ------------------------------------------------------------------ launches back to back
 def test_graph_of_calls_in_every_plan_matches_the_oracle():
     """One CUDA graph holding calls of every plan back to back -- cluster, segmented
