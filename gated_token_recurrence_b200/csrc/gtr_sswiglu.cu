@@ -11,9 +11,12 @@
 // 16-bit data, 32 of fp32).  The xv tile with a one-token halo and the xg tile come in by
 // TMA; the halo box starts one row and one column before the tile, and the rows and
 // columns outside the grid arrive as zeros -- the convolution's zero padding.  Each
-// thread then produces 16-byte pieces of the output (8 channels of 16-bit data, 4 of
-// fp32): nine shared-memory neighbours times the fp32 weights, plus the bias, times
-// SiLU(xg), stored with coalesced 16-byte stores.  The path is bound by HBM bandwidth.
+// thread then produces one 16-byte channel piece (8 channels of 16-bit data, 4 of fp32)
+// of a strip of four output tokens down one column: its nine taps in registers, the six
+// halo rows the strip needs read once (each neighbour feeds every output of the strip it
+// touches), plus the bias, times SiLU(xg), stored with coalesced 16-byte stores.  The
+// path is bound by HBM bandwidth; the instruction count per output (shared-memory loads
+// and conversions) is what keeps it below that bound.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -106,13 +109,15 @@ __global__ void __launch_bounds__(kThreadsSw) sswiglu_dwconv_kernel(const __grid
   constexpr int kCh = kCB / (int)sizeof(T);  // channels per block
   constexpr int kN = Vec8<T>::N;             // channels per 16-byte piece
 
+  // channel blocks vary fastest: the CTAs running at once read whole token rows
+  // (C channels contiguous in memory) instead of one 128-byte piece of each token
   int t = blockIdx.x;
+  const int cb = t % sp.cblocks;
+  t /= sp.cblocks;
   const int tx = t % sp.tiles_x;
   t /= sp.tiles_x;
   const int ty = t % sp.tiles_y;
-  t /= sp.tiles_y;
-  const int cb = t % sp.cblocks;
-  const int b = t / sp.cblocks;
+  const int b = t / sp.tiles_y;
   const int x0 = tx * kTW, y0 = ty * kTH, c0 = cb * kCh;
   const int tid = threadIdx.x;
 
@@ -137,31 +142,49 @@ __global__ void __launch_bounds__(kThreadsSw) sswiglu_dwconv_kernel(const __grid
   for (int it = 0; !ok && it < 1000; ++it) ok = mbar_wait_sleep(&full, 0, 1000000u);
   if (!ok) return;
 
-  // work item w: token (row r, column c) of the tile, 16-byte piece j of its channels
+  // Thread t: 16-byte channel piece j = t % 8 of column c = (t / 8) % 16 of the tile, output
+  // rows 4q .. 4q + 3 (q = t / 128).  Its nine taps and bias live in registers; it walks the
+  // six halo rows those outputs need once, each neighbour feeding every output it touches,
+  // so a halo element is loaded and converted twice on average instead of nine times.
   constexpr int kPieces = kCB / 16;  // 8
-  for (int w = tid; w < kTH * kTW * kPieces; w += kThreadsSw) {
-    const int j = w % kPieces, tok = w / kPieces;
-    const int r = tok / kTW, c = tok % kTW;
-    const int y = y0 + r, x = x0 + c;
-    if (y >= sp.H || x >= sp.W) continue;
-    float acc[kN];
+  constexpr int kRows = kTH * kTW * kPieces / kThreadsSw;  // 4 output rows a thread
+  static_assert(kTW * kPieces * (kTH / kRows) == kThreadsSw, "one column strip of kRows rows per thread");
+  const int j = tid % kPieces, c = (tid / kPieces) % kTW, q = tid / (kPieces * kTW);
+  float wr[9][kN], acc[kRows][kN];
 #pragma unroll
-    for (int e = 0; e < kN; ++e) acc[e] = bsm[j * kN + e];
+  for (int e = 0; e < kN; ++e) {
 #pragma unroll
-    for (int dy = 0; dy < 3; ++dy)
+    for (int tap = 0; tap < 9; ++tap) wr[tap][e] = wsm[j * kN + e][tap];
 #pragma unroll
-      for (int dx = 0; dx < 3; ++dx) {
-        float f[kN];
-        Vec8<T>::load(*reinterpret_cast<const uint4*>(halo + ((r + dy) * (kTW + 2) + (c + dx)) * kCB + 16 * j), f);
+    for (int k = 0; k < kRows; ++k) acc[k][e] = bsm[j * kN + e];
+  }
 #pragma unroll
-        for (int e = 0; e < kN; ++e) acc[e] = fmaf(wsm[j * kN + e][3 * dy + dx], f[e], acc[e]);
+  for (int hr = 0; hr < kRows + 2; ++hr) {  // halo row kRows q + hr
+#pragma unroll
+    for (int dx = 0; dx < 3; ++dx) {
+      float f[kN];
+      Vec8<T>::load(*reinterpret_cast<const uint4*>(halo + ((kRows * q + hr) * (kTW + 2) + (c + dx)) * kCB + 16 * j), f);
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        const int dy = hr - k;  // output row kRows q + k takes halo rows k .. k + 2
+        if (dy >= 0 && dy < 3) {
+#pragma unroll
+          for (int e = 0; e < kN; ++e) acc[k][e] = fmaf(wr[3 * dy + dx][e], f[e], acc[k][e]);
+        }
       }
+    }
+  }
+  const int x = x0 + c;
+#pragma unroll
+  for (int k = 0; k < kRows; ++k) {
+    const int r = kRows * q + k, y = y0 + r;
+    if (y >= sp.H || x >= sp.W) continue;
     float g[kN];
     Vec8<T>::load(*reinterpret_cast<const uint4*>(xgt + (r * kTW + c) * kCB + 16 * j), g);
 #pragma unroll
-    for (int e = 0; e < kN; ++e) acc[e] *= g[e] / (1.f + __expf(-g[e]));  // SiLU(xg)
+    for (int e = 0; e < kN; ++e) acc[k][e] *= __fdividef(g[e], 1.f + __expf(-g[e]));  // SiLU(xg)
     T* o = reinterpret_cast<T*>(sp.out) + (((size_t)b * sp.H + y) * sp.W + x) * sp.C + c0 + j * kN;
-    __stcs(reinterpret_cast<uint4*>(o), Vec8<T>::store(acc));
+    __stcs(reinterpret_cast<uint4*>(o), Vec8<T>::store(acc[k]));
   }
 }
 
