@@ -535,9 +535,22 @@ def run_ours(args):
 
 
 def run_profile(args):
-    """Eager calls only (no graph, sweep, e2e or CPU leg): the command ncu captures."""
+    """Eager calls only (no graph, sweep, e2e or CPU leg): the command ncu captures.  A
+    stencil workload name (sw640, sw1024, sw2048) profiles the Spatial SwiGLU stencil."""
     import gated_token_recurrence_b200 as gtr
     device = torch.device("cuda", 0)
+    if args.workload in STENCILS:
+        st = STENCILS[args.workload]
+        ssets = []
+        for i in range(4):
+            xg, xv, cw, cb = (t.to(device) for t in make_stencil_inputs(st, 9000 + i))
+            ssets.append((xg, xv, cw, cb, torch.empty_like(xv)))
+        for i in range(args.warmup + args.steps):
+            xg, xv, cw, cb, out = ssets[i % len(ssets)]
+            gtr.sswiglu_dwconv(xg, xv, cw, cb, grid=(st.H, st.W), out=out)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": args.workload, "calls": args.warmup + args.steps}))
+        return 0
     w = WORKLOADS[args.workload]
     sets = make_sets(w, min(n_sets_for(w), 8), device, 0)
     ws = gtr.new_workspace(w.B, w.heads, w.H, w.W, w.d_k, w.d_v,
@@ -556,7 +569,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="640", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="640", choices=sorted(WORKLOADS) + sorted(STENCILS),
+                    help="GLA workload (stencil names: --profile only)")
     ap.add_argument("--path", default="auto", choices=["auto", "split", "fused", "fused_sequential"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -566,6 +580,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload in STENCILS and not args.profile:
+        ap.error("stencil workloads run under --profile only (the bench line reports them as sweep lines)")
     if args.impl == "reference":
         return run_reference(args)
     if args.profile:
