@@ -493,10 +493,23 @@ __device__ __forceinline__ void epilogue_rows(uint32_t taddr, uint8_t* rowdst, u
 // [+ the row's partial output olc, fp16, SEGMENTED second phase]),
 //   y_j = o_j / sqrt(mean_i o_i^2 + eps) * nw_j * SiLU(gate_j),
 // the lane's gate row `grow` (Tin, 64 values; nullptr for rows that are not stored).  Two
-// passes over tensor memory: the row's sum of squares, then the values.  Out of line.
+// passes over tensor memory: the row's sum of squares, then the values.  The gate row (128
+// bytes) is requested first, in 16-byte loads that stay ahead of the tensor-memory loads, so
+// its latency overlaps the norm pass instead of following each use; the partial output is
+// read 16 bytes at a time.  Out of line.
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
 template <typename Tout, typename Tin>
 __device__ __noinline__ void gated_rows(uint32_t taddr, const uint8_t* olc, uint8_t* rowdst, const Tin* grow,
                                         const float* nw, float eps, uint8_t* wstage, int lane, float& nf, float osc) {
+  uint4 gq[8];  // the gate row, 8 x 16 bytes (values 8c .. 8c + 7 in gq[c])
+#pragma unroll
+  for (int c = 0; c < 8; ++c) gq[c] = grow ? ld_nc_v4(reinterpret_cast<const uint4*>(grow) + c) : make_uint4(0, 0, 0, 0);
   float ss = 0.f;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
@@ -504,11 +517,16 @@ __device__ __noinline__ void gated_rows(uint32_t taddr, const uint8_t* olc, uint
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-      float2 o = make_float2(0.f, 0.f);
-      if (olc) o = __half22float2(bits_h2(*reinterpret_cast<const uint32_t*>(olc + 2 * (32 * half + j))));
-      const float x0 = (v[j] + o.x) * osc, x1 = (v[j + 1] + o.y) * osc;
-      ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+    for (int c = 0; c < 4; ++c) {
+      uint4 o4 = make_uint4(0, 0, 0, 0);
+      if (olc) o4 = *reinterpret_cast<const uint4*>(olc + 64 * half + 16 * c);
+      const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 o = __half22float2(bits_h2(ow[u]));
+        const float x0 = (v[8 * c + 2 * u] + o.x) * osc, x1 = (v[8 * c + 2 * u + 1] + o.y) * osc;
+        ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+      }
     }
   }
   const float rinv = rsqrtf(ss * (1.f / 64.f) + eps);
@@ -518,12 +536,20 @@ __device__ __noinline__ void gated_rows(uint32_t taddr, const uint8_t* olc, uint
     tmem_ld32(taddr + 32u * half, v);
     tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-      float2 o = make_float2(0.f, 0.f), g = make_float2(0.f, 0.f);
-      if (olc) o = __half22float2(bits_h2(*reinterpret_cast<const uint32_t*>(olc + 2 * (32 * half + j))));
-      if (grow) g = In2<Tin>::unpack(__ldg(reinterpret_cast<const unsigned int*>(grow + 32 * half + j)));
-      v[j] = (v[j] + o.x) * osc * rinv * nw[32 * half + j] * silu_fast(g.x);
-      v[j + 1] = (v[j + 1] + o.y) * osc * rinv * nw[32 * half + j + 1] * silu_fast(g.y);
+    for (int c = 0; c < 4; ++c) {
+      uint4 o4 = make_uint4(0, 0, 0, 0);
+      if (olc) o4 = *reinterpret_cast<const uint4*>(olc + 64 * half + 16 * c);
+      const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+      const uint4 g4 = gq[4 * half + c];
+      const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = 8 * c + 2 * u;  // value 32 half + j of the row
+        const float2 o = __half22float2(bits_h2(ow[u]));
+        const float2 g = In2<Tin>::unpack(gw[u]);
+        v[j] = (v[j] + o.x) * osc * rinv * nw[32 * half + j] * silu_fast(g.x);
+        v[j + 1] = (v[j + 1] + o.y) * osc * rinv * nw[32 * half + j + 1] * silu_fast(g.y);
+      }
     }
     stage_store_half<Tout>(v, rowdst, wstage, lane, half, nf);
   }
