@@ -264,8 +264,10 @@ __device__ __forceinline__ float log_sigmoid_fast(float x) {
 }
 
 // SiLU(x) = x * sigmoid(x) = x / (1 + e^-x).
+// (the approximate divide: a few ulp, and 0 once 1 + e^-x passes 2^126, the limit of
+// x / (1 + e^-x) for very negative x)
 __device__ __forceinline__ float silu_fast(float x) {
-  return x * __frcp_rn(1.f + ex2(-x * 1.4426950408889634f));
+  return __fdividef(x, 1.f + ex2(-x * 1.4426950408889634f));
 }
 
 // Bounded mbarrier wait: the thread sleeps in hardware until the phase completes; only
@@ -780,10 +782,75 @@ __device__ __noinline__ float4 take_input_scale(int wg, int wtid, Misc* ms, WsHe
 // plus the offsets o0 / o1 of its two passes) into the gate tile, then, once the score
 // region is free, the CUDA-core scores straight into tensor memory.  False: the wait gave
 // up.  The caller flips its slot.
+// Scores of a chunk whose gates allow the factorisation, in fp32 on the CUDA cores:
+// d_k^-1/2 sum_k (q_ik 2^A_ik)(k_jk 2^-A_jk) over scan(j) <= scan(i) -- the tensor-core
+// factorisation without its fp16 rounding.  The operand warpgroup first writes
+// Kf = k 2^-A (times sk) transposed ([k][j], fp32) into `kft` (16 KB), then each thread
+// forms its 32 scores (the 16x256b tensor-memory layout of cuda_core_scores: rows r0 and
+// r0 + 8 of warp w4, 16 columns a pass) from its rows' q 2^A and the shared Kf.  Used for
+// a sequence's first chunk under the output gate, whose first rows sum few terms.
+template <typename Tin, bool kRev, int kDK>
+__device__ __noinline__ void factored_scores(const uint8_t* sb, const float* G, float* kft, uint32_t taddr, int w4,
+                                             int lane, int wg, int row0, int cc, float ssc, float sq, float sk) {
+  const uint8_t* qraw = kDK == 64 ? sb : reinterpret_cast<const uint8_t*>(G) + kRawQ;
+  const uint8_t* kraw = kDK == 64 ? sb + kTile : reinterpret_cast<const uint8_t*>(G) + kRawK;
+  // Kf, transposed: this thread's rows row0 .. row0+3, channels 32p + 4cc .. +3
+  for (int ps = 0; ps < kDK / 32; ++ps)
+    for (int i = 0; i < 4; ++i) {
+      const int j = row0 + i, k0 = 32 * ps + 4 * cc;
+      for (int e = 0; e < 4; e += 2) {
+        const uint32_t oj = kDK == 64 ? sw128_offset(j, k0 + e) : (uint32_t)(j * 64 + 2 * (k0 + e));
+        const float2 kv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(kraw + oj));
+        kft[(k0 + e) * 64 + j] = kv.x * sk * ex2(-G[j * kDK + k0 + e]);
+        kft[(k0 + e + 1) * 64 + j] = kv.y * sk * ex2(-G[j * kDK + k0 + e + 1]);
+      }
+    }
+  wg_sync(wg);
+  const int r0 = 16 * w4 + (lane >> 2), cq = 2 * (lane & 3);
+  for (int ps = 0; ps < 2; ++ps) {
+    float acc[2][8];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[r][t] = 0.f;
+    for (int k = 0; k < kDK; k += 2) {
+      float2 qf[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = r0 + 8 * r;
+        const uint32_t oi = kDK == 64 ? sw128_offset(i, k) : (uint32_t)(i * 64 + 2 * k);
+        const float2 qv = In2<Tin>::unpack(*reinterpret_cast<const uint32_t*>(qraw + oi));
+        qf[r] = make_float2(qv.x * sq * ex2(G[i * kDK + k]), qv.y * sq * ex2(G[i * kDK + k + 1]));
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float2 kf = *reinterpret_cast<const float2*>(kft + (k + kk) * 64 + 32 * ps + 8 * c + cq);
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float q1 = kk ? qf[r].y : qf[r].x;
+            acc[r][2 * c] = fmaf(q1, kf.x, acc[r][2 * c]);
+            acc[r][2 * c + 1] = fmaf(q1, kf.y, acc[r][2 * c + 1]);
+          }
+        }
+    }
+    float sv[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int r = (x & 3) >> 1, c = x >> 2, b = x & 1;
+      const int i = r0 + 8 * r, j = 32 * ps + 8 * c + cq + b;
+      sv[x] = (kRev ? j >= i : j <= i) ? acc[r][2 * c + b] * ssc : 0.f;  // scan(j) <= scan(i)
+    }
+    tmem_st16x256_x4(taddr + 32u * ps, sv);
+  }
+}
+
 template <typename Tin, bool kRev, int kDK>
 __device__ __noinline__ bool cuda_core_chunk(float* G, float4 o0, float4 o1, int row0, int cc, Misc* ms,
                                              WsHeader* hdr, int wg, int wtid, int slot, int n, const uint8_t* sb,
-                                             uint32_t taddr, int w4, int lane, float ssc, float sq, float sk) {
+                                             uint32_t taddr, int w4, int lane, float ssc, float sq, float sk,
+                                             float* kft) {
   for (int ps = 0; ps < kDK / 32; ++ps) {
     const float4 o = ps ? o1 : o0;
     for (int i = 0; i < 4; ++i) {
@@ -794,7 +861,10 @@ __device__ __noinline__ bool cuda_core_chunk(float* G, float4 o0, float4 o1, int
   }
   if (!wg_wait(wg, wtid, &ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x302, slot)) return false;
   tc_fence_after();  // (the wait's barrier also publishes the full A)
-  cuda_core_scores<Tin, kRev, kDK>(sb, G, taddr, w4, lane, ssc, sq, sk);
+  if (kft)  // gates that allow the factorisation: fp32 factored scores
+    factored_scores<Tin, kRev, kDK>(sb, G, kft, taddr, w4, lane, wg, row0, cc, ssc, sq, sk);
+  else
+    cuda_core_scores<Tin, kRev, kDK>(sb, G, taddr, w4, lane, ssc, sq, sk);
   tmem_wait_st();
   tc_fence_before();
   wg_sync(wg);  // raw q / k reads done before the overwrite
@@ -909,7 +979,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool clus = kMode < 0 ? fp.mode == 2 : kMode == 2;  // ... through distributed shared memory
   const int seq = (segm || clus) ? (int)blockIdx.x / fp.n_s : (int)blockIdx.x;
   const int seg = (segm || clus) ? (int)blockIdx.x % fp.n_s : 0;
-  const bool partial = segm && seg > 0;    // outputs completed in the second phase
+  // outputs completed in the second phase: segments s > 0, and with the output gate segment 0
+  // too (its start state is zero), so that its gated epilogues run on all four warpgroups in
+  // the second phase instead of holding up every segment at the summary barrier
+  const bool partial = segm && (seg > 0 || gated);
   const int b = seq / p.heads, h = seq % p.heads;
   const long long L = p.L();
   const Span sp = seg_span(fp, seg);
@@ -917,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CLUSTER with at most kStages chunks a CTA: the staging buffers are never refilled, so
   // each chunk's Qh stays in its own and becomes Qh' in place at the end
   const bool inplace = clus && cnt <= kStages;
-  const bool qhw = (segm || clus) && seg > 0 && !inplace;  // Qh' tiles go to the workspace (the Qh' warp)
+  const bool qhw = partial || (clus && seg > 0 && !inplace);  // Qh' tiles go to the workspace (the Qh' warp)
   float nonfinite = 0.f;
   bool cwaited = false;                    // CLUSTER: this thread has passed the start barrier
 
@@ -1450,7 +1523,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the output gate, the sequence's first chunk also takes the exact CUDA-core scores: its
       // first tokens' outputs sum few terms, and the RMSNorm scales each row to unit size, so
       // the fp16 rounding of the factorised operands would no longer be averaged away.
-      const bool fbx = __any_sync(0xffffffffu, exp_unsafe) || (gated && sp.c0 + n == 0);
+      const bool unsafe = __any_sync(0xffffffffu, exp_unsafe);
+      const bool fbx = unsafe || (gated && sp.c0 + n == 0);
       if (fbx) {
         // ---- CUDA-core scores, straight into tensor memory (lane tile 0 of the chunk's
         // score region): d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk) over scan(j) <= scan(i),
@@ -1460,7 +1534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             G, make_float4(off[0][0], off[0][1], off[0][2], off[0][3]),
             make_float4(off[kPasses - 1][0], off[kPasses - 1][1], off[kPasses - 1][2], off[kPasses - 1][3]), row0, cc,
             ms, hdr, wg, wtid, slot, n, sb, tmem + ((uint32_t)(32 * w4) << 16) + kColSU + 64u * (uint32_t)(n % kSU), w4,
-            lane, kHalfIn ? kKf * sv : kKf, sq, sk);
+            lane, kHalfIn ? kKf * sv : kKf, sq, sk,
+            unsafe ? nullptr : reinterpret_cast<float*>(smem + kOffStg));  // (the staging area is idle until the first epilogue)
         slot ^= 1;
         if (!ok) {
           alive = false;
