@@ -128,7 +128,9 @@ gtr_status_t gtr_gla_fwd_f32(const void *q, const void *k, const void *v,
                              gtr_stream_t stream);
 
 /* Bytes of device workspace a gtr_gla_fwd_ex call with these arguments needs
- * (for every path the dispatcher may choose).  0 for invalid arguments. */
+ * (for every path the dispatcher may choose, and for every direction: the fused
+ * path stages some directions one grid line a chunk, which can take more chunks
+ * than ceil(L / 64)).  0 for invalid arguments. */
 size_t gtr_gla_workspace_bytes(int B, int heads, int grid_H, int grid_W, int d_k, int d_v,
                                int in_dtype, int path);
 
