@@ -103,6 +103,7 @@ struct DeviceCache {
   std::mutex mu;
   DeviceBuffer ws;                  // workspace for gtr_gla_fwd / typed forms
   DeviceBuffer io[5];               // q, k, v, log_gamma, out for the host-buffer entry
+  unsigned int* err_host = nullptr;  // pinned word: the error word read back with the output
 };
 
 DeviceCache g_cache[kMaxDevices];
@@ -347,11 +348,16 @@ gtr_status_t gtr_gla_fwd_host(const void* q, const void* k, const void* v, const
   if (st != GTR_OK) return st;
   st = run(p, path, c.ws.ptr, c.ws.bytes, stream);
   if (st != GTR_OK) return st;
-  if (cudaMemcpyAsync(out, c.io[4].ptr, bytes[4], cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+  // the output and the device error word come back in the same stream, then one synchronisation
+  if (!c.err_host && cudaMallocHost(reinterpret_cast<void**>(&c.err_host), sizeof(unsigned int)) != cudaSuccess) {
+    c.err_host = nullptr;
+    return GTR_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(out, c.io[4].ptr, bytes[4], cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemcpyAsync(c.err_host, c.ws.ptr, sizeof(unsigned int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
     return GTR_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return GTR_ERR_CUDA;
-  unsigned int err = 0;
-  if (cudaMemcpy(&err, c.ws.ptr, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return GTR_ERR_CUDA;
+  const unsigned int err = *c.err_host;
   if (err) {
     const unsigned int zero[2] = {0u, 0u};
     if (cudaMemcpy(c.ws.ptr, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return GTR_ERR_CUDA;
