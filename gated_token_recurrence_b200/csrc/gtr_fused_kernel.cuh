@@ -272,8 +272,13 @@ __device__ __forceinline__ float silu_fast(float x) {
 
 // Bounded mbarrier wait: the thread sleeps in hardware until the phase completes; only
 // after about a second without completion does the CTA record a timeout and abort.
-__device__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+// kOut: the loop after the first attempt is a call (out of line), so that a chunk loop full
+// of waits keeps only their fast paths (the segmented kernel, measured faster so).
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where);
+template <bool kOut = false>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
   if (mbar_wait_sleep(bar, parity, 1000000u)) return true;
+  if constexpr (kOut) return wait_bar_slow(bar, parity, ms, hdr, where);
   const uint64_t t0 = globaltimer();
   while (true) {
     if (*(volatile int*)&ms->abort) return false;
@@ -288,9 +293,12 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr
 
 // Bounded wait by polling (no suspension), for the MMA-issuing threads: they react to a
 // completed phase at once.
-__device__ bool wait_spin(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+__device__ __noinline__ bool wait_spin_slow(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where);
+template <bool kOut = false>
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
   for (int i = 0; i < 64; ++i)
     if (mbar_test(bar, parity)) return true;
+  if constexpr (kOut) return wait_spin_slow(bar, parity, ms, hdr, where);
   const uint64_t t0 = globaltimer();
   while (true) {
     for (int i = 0; i < 64; ++i)
@@ -302,6 +310,13 @@ __device__ bool wait_spin(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hd
       return false;
     }
   }
+}
+
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+  return wait_bar<false>(bar, parity, ms, hdr, where);
+}
+__device__ __noinline__ bool wait_spin_slow(uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr, uint32_t where) {
+  return wait_spin<false>(bar, parity, ms, hdr, where);
 }
 
 // Bounded wait until a global counter reaches `target` (`limit_ns`: about a second, or the
@@ -338,10 +353,11 @@ __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128
 // Warpgroup wait: its first thread does the bounded wait, then every thread of the
 // group takes the same decision (no thread is left alone at a named barrier) and
 // observes the completed phase itself.
-__device__ bool wg_wait(int wg, int wtid, uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr,
-                        uint32_t where, int& slot, bool spin = false) {
+template <bool kOut = false>
+__device__ __forceinline__ bool wg_wait(int wg, int wtid, uint64_t* bar, uint32_t parity, Misc* ms, WsHeader* hdr,
+                                        uint32_t where, int& slot, bool spin = false) {
   if (wtid == 0) {
-    const bool ok = spin ? wait_spin(bar, parity, ms, hdr, where) : wait_bar(bar, parity, ms, hdr, where);
+    const bool ok = spin ? wait_spin<kOut>(bar, parity, ms, hdr, where) : wait_bar<kOut>(bar, parity, ms, hdr, where);
     ms->go[wg][slot] = ok && !*(volatile int*)&ms->abort;
   }
   wg_sync(wg);
@@ -958,6 +974,7 @@ __device__ __forceinline__ void second_phase(const FusedParams& fp, Misc* ms, Ws
 template <typename Tin, typename Tout, bool kRev, bool kBox, int kMode, int kDK, bool kBlock>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_gla_kernel(const __grid_constant__ FusedParams fp) {
+  constexpr bool kOL = kMode == 1;  // out-of-line slow paths of the waits
   const bool lowrank = kBlock && fp.lowrank != 0;
   const bool gated = kBlock && fp.gated != 0;
   static_assert(kDK == 64 || kDK == 32, "key widths 64 and 32");
@@ -1053,8 +1070,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // A staging buffer is refilled once the P V of its previous chunk has completed and,
     // in a segment s > 0, that chunk's Qh' has been copied out.
     auto stage_free = [&](int n, int st) -> bool {
-      if (!wait_bar(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) return false;
-      return !qhw || wait_bar(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
+      if (!wait_bar<kOL>(&ms->empty[st], ph_rel<kStages>(n), ms, hdr, 0x100)) return false;
+      return !qhw || wait_bar<kOL>(&ms->qdone[st], ph_rel<kStages>(n), ms, hdr, 0x101);
     };
     if constexpr (kBox) {
       // One thread issues four TMA boxes per chunk (Q, K, V with the 128-byte swizzle, G
@@ -1252,7 +1269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* eseg = ms->eseg;
       for (int c = sp.c0, n = 0; c < sp.c1; ++c, ++n) {
         const int st = n % kStages;
-        if (!wait_bar(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x110)) { ok = false; break; }
+        if (!wait_bar<kOL>(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x110)) { ok = false; break; }
         const uint8_t* qt = smem + kOffStage + st * kStageBytes;  // Qh, built in place
         {
           *reinterpret_cast<float2*>(&ms->eseg[2 * lane]) = make_float2(ex2(a2s0), ex2(a2s1));
@@ -1292,8 +1309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_base = smem_u32(smem);
       for (int n = 0; n < cnt; ++n) {
         const int st = n % kStages;
-        if (!wait_spin(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x200)) break;
-        if (!wait_spin(&ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x201)) break;
+        if (!wait_spin<kOL>(&ms->opready[st], ph_use<kStages>(n), ms, hdr, 0x200)) break;
+        if (!wait_spin<kOL>(&ms->su_free[n % kSU], ph_rel<kSU>(n), ms, hdr, 0x201)) break;
         const uint32_t a_q = s_base + kOffStage + st * kStageBytes;  // Qh (built in place)
         const uint32_t a_k = a_q + kTile;                            // Kh
         const uint32_t a_v = a_q + 2 * kTile;
@@ -1328,15 +1345,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_o = tmem + kColO + 64u * (uint32_t)((m >> 1) % kOPairs) + ((m & 1) ? kLaneTile1 : 0u);
         // Qh built (the stage-1 issuer waits on the same phase; neither can lap it, as the
         // stage is refilled only after this chunk's P V), chunk-start state written
-        if (!wait_spin(&ms->opready[st], ph_use<kStages>(m), ms, hdr, 0x205)) break;
-        if (!wait_spin(&ms->sready[m % kNS], ph_use<kNS>(m), ms, hdr, 0x202)) break;
-        if (!(m & 1) && !wait_spin(&ms->o_free[(m >> 1) % kOPairs], ph_rel<kOPairs>(m >> 1), ms, hdr, 0x203)) break;
+        if (!wait_spin<kOL>(&ms->opready[st], ph_use<kStages>(m), ms, hdr, 0x205)) break;
+        if (!wait_spin<kOL>(&ms->sready[m % kNS], ph_use<kNS>(m), ms, hdr, 0x202)) break;
+        if (!(m & 1) && !wait_spin<kOL>(&ms->o_free[(m >> 1) % kOPairs], ph_rel<kOPairs>(m >> 1), ms, hdr, 0x203)) break;
         const uint32_t a_q = s_base + kOffStage + st * kStageBytes;
         const uint32_t a_s = s_base + kOffS + (m % kNS) * kTile;
         tc_fence_after();
         for (int k = 0; k < kDK / 16; ++k)
           mma_f16(d_o, sw128_desc(a_q + 32 * k), sw128_desc(a_s + 2048 * k), id_qs, k > 0);
-        if (!wait_spin(&ms->pready[su], ph_use<kSU>(m), ms, hdr, 0x204)) break;
+        if (!wait_spin<kOL>(&ms->pready[su], ph_use<kSU>(m), ms, hdr, 0x204)) break;
         // P sits in the lane tile of the chunk's output (A and D rows share lanes)
         const uint32_t a_v = a_q + 2 * kTile;
         const uint32_t a_p = tmem + kColSU + 64u * su + ((m & 1) ? kLaneTile1 : 0u);
@@ -1381,7 +1398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int n = hh; n < cnt; n += 2) {
       const int st = n % kStages;
-      if (!wg_wait(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
+      if (!wg_wait<kOL>(wg, wtid, &ms->full[st], ph_use<kStages>(n), ms, hdr, 0x301, slot)) {
         alive = false;
         break;
       }
@@ -1658,7 +1675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int n = 0; n < cnt; ++n) {
       const int st = n % kStages, su = n % kSU;
-      if (!wait_bar(&ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400)) { alive = false; break; }
+      if (!wait_bar<kOL>(&ms->su_full[su], ph_use<kSU>(n), ms, hdr, 0x400)) { alive = false; break; }
       tc_fence_after();
       const bool fbk = ms->fb[st] != 0;
       const float* alast = reinterpret_cast<const float*>(smem + kOffStage + st * kStageBytes + 3 * kTile);
@@ -1739,7 +1756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every thread leaves the loop (the waits are bounded): agree on the outcome, and that
     // the input scale is known (the summaries go back to the inputs' scale; the scale was
     // set before chunk 0's operands, so this spin finds it complete)
-    if ((segm || clus) && alive) alive = wait_spin(&ms->scale_ready, 0u, ms, hdr, 0x405);
+    if ((segm || clus) && alive) alive = wait_spin<kOL>(&ms->scale_ready, 0u, ms, hdr, 0x405);
     alive = wg_all(wg, alive);
     if (clus && alive) {
       // segment summary for the cluster's scan, read by the other CTAs after the cluster
@@ -1798,14 +1815,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // the CTA's input scale (WG_A0 derives it from the first chunk; the outputs go back to
     // the inputs' scale); the wait's barrier also publishes the marks above
-    bool alive = wg_wait(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x506, slot);
+    bool alive = wg_wait<kOL>(wg, wtid, &ms->scale_ready, 0u, ms, hdr, 0x506, slot);
     if (clus) {
       // the outputs stay in tensor memory until the start state is known: wait for their
       // last MMAs; then (segments s > 0) the chunks' Qh' tiles start loading into the idle
       // staging buffers
       for (int pr = 0; pr < (cnt + 1) / 2 && alive; ++pr)
-        alive = wg_wait(wg, wtid, &ms->o_full[pr], 0u, ms, hdr, 0x520, slot);
-      if (alive && qhw && wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x521, slot) && wtid == 0) {
+        alive = wg_wait<kOL>(wg, wtid, &ms->o_full[pr], 0u, ms, hdr, 0x520, slot);
+      if (alive && qhw && wg_wait<kOL>(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x521, slot) && wtid == 0) {
         mbar_arrive_expect_tx(&ms->p2_full[0], (uint32_t)(cnt * kTile));
         for (int g = 0; g < cnt; g += 2) {
           const int nb = min(2, cnt - g);
@@ -1819,7 +1836,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pairs = alive ? (cnt + 1) / 2 : 0;
       const float osc = ms->sc_out;
       for (int pr = 0; pr < pairs; ++pr) {
-        if (!wg_wait(wg, wtid, &ms->o_full[pr % kOPairs], ph_use<kOPairs>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
+        if (!wg_wait<kOL>(wg, wtid, &ms->o_full[pr % kOPairs], ph_use<kOPairs>(pr), ms, hdr, 0x500, slot)) { alive = false; break; }
         tc_fence_after();
         const int ci = 2 * pr + tsel;
         long long s = 0;
@@ -1875,7 +1892,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const unsigned int dbg_us = ms->dbg_us;
       const uint64_t limit = dbg_us ? 1000ull * dbg_us : 1000000000ull;
       const int loads = partial ? min(4, (cnt + 1) / 2) : 0;
-      bool ok0 = wg_wait(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
+      bool ok0 = wg_wait<kOL>(wg, wtid, &ms->agg_pub, 0u, ms, hdr, 0x600, slot);
       int issued = 0;
       if (ok0) {
         if (wtid == 0) {
@@ -2065,7 +2082,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wq * 32 * 128;
       const int npairs = (cnt + 1) / 2;
       int slot = 0;
-      if (seg > 0 && q == 3 && wtid == 0 && (inplace || wait_bar(&ms->p2_full[0], 0u, ms, hdr, 0x530))) {
+      if (seg > 0 && q == 3 && wtid == 0 && (inplace || wait_bar<kOL>(&ms->p2_full[0], 0u, ms, hdr, 0x530))) {
         const uint32_t id_qs = idesc_f16(0, 64, 64, 0, 1);
         const uint32_t s_base = smem_u32(smem);
         tc_fence_after();
@@ -2078,7 +2095,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int pr = q; pr < npairs; pr += 4) {
-        if (seg > 0 && !wg_wait(q, wtid, &ms->corr_done[pr], 0u, ms, hdr, 0x531, slot)) break;
+        if (seg > 0 && !wg_wait<kOL>(q, wtid, &ms->corr_done[pr], 0u, ms, hdr, 0x531, slot)) break;
         tc_fence_after();
         const int ci = 2 * pr + tsel;
         long long s = 0;
