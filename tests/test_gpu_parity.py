@@ -275,6 +275,25 @@ def test_fused_range_guard_reports_and_split_path_handles_it():
     assert rel_err(out, ref) <= 1e-2
 
 
+def test_host_entry_returns_the_device_error_and_recovers():
+    """The host-buffer entry reads the device error word back with the output: the range
+    case above returns GTR_ERR_RANGE from the call itself, and the next call on the same
+    library-owned buffers runs clean and matches the oracle."""
+    w = Workload("range", B=1, heads=1, H=8, W=16, dtype="bf16", index=9)
+    q, k, v, lg = make_inputs(w, 91)
+    out = torch.empty((w.B, w.L, w.heads, w.d_v), dtype=torch.float32).pin_memory()
+    bad = v.clone()
+    bad[0, 5, 0, 3] = 1.0e6
+    pin = [t.contiguous().pin_memory() for t in (q, k, bad, lg)]
+    with pytest.raises(gtr.GTRError) as e:
+        gtr.gla_fwd_host(*pin, out, grid=(w.H, w.W))
+    assert e.value.status == 6
+    pin[2] = v.contiguous().pin_memory()
+    gtr.gla_fwd_host(*pin, out, grid=(w.H, w.W))
+    ref = oracle.gla_fwd(q, k, v, lg, w.H, w.W, 0)
+    assert rel_err(out, ref) <= TOL[w.dtype]
+
+
 @pytest.mark.parametrize("name", ["640", "1024", "2048", "stack"])
 def test_paths_agree_on_workloads(name):
     """The fused plan, the one-CTA-per-sequence walk and the split path agree (1e-2 * rms)."""
