@@ -11,33 +11,38 @@
 //   P  = mask_{j<=i}(Qh Kh^T)   = d_k^-1/2 sum_k q_ik k_jk 2^(A_ik - A_jk)
 //   O  = Qh S + P V             (S = state at the chunk start, kept scaled by d_k^-1/2)
 //   U' = Kh^T V,  S <- 2^a * (S + U')     (= Diag(d) S + K~^T V with K~ = K * 2^(a - A))
-// The power-of-two factor d_k^-1/2 = 1/8 rides on Kh, so every product below
-// already carries it and the outputs leave tensor memory final.  All MMA operands
-// are fp16 (bf16 inputs convert exactly inside the fp16 range); accumulation and
-// the state are fp32.  Qh and Kh overwrite the Q and K tiles they are built from.
-// A chunk whose gates decay too fast for the factorisation to stay inside fp16
-// gets its scores from the CUDA cores (2^(A_i - A_j) per pair), written straight
-// into tensor memory.  Outputs that come out non-finite (an operand beyond the
-// fp16 range) are reported as GTR_ERR_RANGE.
+// The power of two in d_k^-1/2 (1/8 for d_k = 64; 1/4 for d_k = 32, whose remaining
+// 2^-1/2 is applied to the outputs) rides on Kh, so every product below already carries
+// it.  All MMA operands are fp16 (bf16 inputs convert inside the fp16 range); a CTA whose
+// first chunk holds tiny inputs scales q, k, v by powers of two into that range and
+// undoes it in fp32.  Accumulation and the state are fp32.  Qh and Kh overwrite the Q
+// and K tiles they are built from.  A chunk whose gates decay too fast for the
+// factorisation to stay inside fp16 gets its scores from the CUDA cores (2^(A_i - A_j)
+// per pair), written straight into tensor memory.  Outputs that come out non-finite (an
+// operand beyond the fp16 range) are reported as GTR_ERR_RANGE.
 //
-// Two modes.  STREAM: one CTA walks a whole sequence, carrying the exact fp32
-// state.  SEGMENTED: the n_s CTAs of a sequence each walk one contiguous run of
-// its chunks (a segment) from a zero start state.  Segment 0's outputs are final;
-// the others write their partial outputs O_local and Qh' = Qh * 2^(A from the
-// segment start) to the workspace and publish the segment summary (end state,
-// log2 decay).  The n_s CTAs then scan the summaries (each owns a slice of the
-// 64x64 state entries), and in a second phase every CTA of a segment s > 0 adds
-// Qh' S_start(s) to O_local, one M = 128 MMA per chunk pair, spread over all four
-// of its warpgroups.
+// Three plans.  STREAM: one CTA walks a whole sequence, carrying the exact fp32 state.
+// CLUSTER: the CTAs of one thread-block cluster split a short sequence, hold their
+// outputs in tensor memory and scan the segment summaries through distributed shared
+// memory.  SEGMENTED: the n_s CTAs of a sequence each walk one contiguous run of its
+// chunks (a segment) from a zero start state, write their partial outputs O_local and
+// Qh' = Qh * 2^(A from the segment start) to the workspace and publish the segment
+// summary (end state, log2 decay); segment 0's outputs are final unless the output gate
+// is on.  The n_s CTAs then scan the summaries (each owns a slice of the 64x64 state
+// entries), and in a second phase every CTA with partial outputs adds Qh' S_start(s) to
+// O_local, one M = 128 MMA per chunk pair, spread over all four of its warpgroups.
 //
 // Warp roles (640 threads):
-//   warps 0-7   WG_A  two warpgroups, one per half of the key channels: cumulative
-//               gates, Qh / Kh in place, CUDA-core scores
-//   warps 8-11  WG_B  score masking, fp32 state update, Qh' (16-lane tensor-memory
-//               loads, so every lane of a warp does the same work)
-//   warps 12-15 WG_C  epilogue; SEGMENTED: summary scan
-//   warps 16-17 producer: TMA boxes, or cp.async row copies (direction remap,
-//               128-byte-swizzled placement, zero fill past the sequence end)
+//   warps 0-7   WG_A  two warpgroups on alternating chunks: cumulative gates (from the
+//               low-rank producer's z rows when given), the input scale (first chunk),
+//               Qh / Kh in place, CUDA-core scores
+//   warps 8-11  WG_B  score masking, fp32 state update, the next chunk-start state
+//               (16-lane tensor-memory loads, so every lane of a warp does the same work)
+//   warps 12-15 WG_C  epilogue (the output gate when given); SEGMENTED: summary scan
+//   warp 16     producer: TMA boxes (row or column views, line chunks), or 4-row TMA
+//               gathers resolving the direction remap (cp.async row copies for views of
+//               2^31 rows or more); zero fill past the sequence or line end
+//   warp 17     Qh' tiles of segments s > 0 (and of segment 0 under the output gate)
 //   warp 18     tcgen05 MMA issuer of the scores and U' (in chunk order), tensor-memory owner
 //   warp 19     tcgen05 MMA issuer of the outputs O = Qh S, O += P V (in chunk order)
 //   SEGMENTED second phase: warpgroups 0-3 (warps 0-15) each take every fourth pair
@@ -205,7 +210,7 @@ struct Misc {
   uint64_t o_full[kOPairs], o_free[kOPairs];         // per output pair
   uint64_t agg_pub, p2_go, mma_final[2], corr_done[kOPairs];
   uint64_t p2_full[4], p2_mma[4];  // second phase, per warpgroup: tiles landed, correction done
-  uint64_t scale_ready;            // the input scale factors below are set (WG_A, first chunk)
+  uint64_t scale_ready;            // the input scale factors below are set (WG_A0, first chunk)
   uint32_t tmem_base;
   // Power-of-two input scale of this CTA, taken from its first chunk (1 unless that chunk's
   // largest |q|, |k| or |v| is tiny): q, k, v enter the fp16 operands multiplied by
@@ -221,13 +226,13 @@ struct Misc {
   alignas(16) float nw[64];       // output gate: RMSNorm weight
   int zrow[2][64];                // producer: z row b*L + m of each chunk row (gathers; -1 past the end)
   int abort;
-  unsigned int dbg_skip, dbg_us;  // failure injection (workspace header), read once at the start
+  unsigned int dbg_skip, dbg_us;  // failure injection (workspace header), read once by WG_C
   int go[4][3];          // per-warpgroup wait decisions, alternating slots; [3][2]: scaled segments seen
   int fb[kStages];       // stage -> scores from the CUDA cores
   alignas(16) float dseg[64];  // CLUSTER: this segment's log2 decay per key channel (read by the cluster)
   alignas(16) float red[2][2][4][32];  // WG_A cumsum: per warpgroup, channel half and warp, channel totals
   alignas(16) float eseg[64];          // Qh' warp: 2^(decay from the segment start) per channel
-  int rowoff[2][64];              // producer: grid cell b*L + m of each chunk row (-1 past the end)
+  int rowoff[2][64];              // producer, per chunk row: the row of the gather view (past the end: a row past the view) or, for row copies, grid cell b*L + m (-1 past the end)
 };
 // The in-chunk log2 decay per channel (a) of a staged chunk is kept in row 0 of its
 // gate tile once the gates are consumed, the factor 2^(decay from the segment start)
@@ -1041,7 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->p2_mma[i], 1);
       ms->go[i][0] = ms->go[i][1] = 0;
     }
-    if (i == 8) mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp (segments s > 0)
+    if (i == 8) mbar_init(&ms->agg_pub, qhw ? 2 : 1);  // WG_B (summary); the Qh' warp when it runs
     if (i == 10) mbar_init(&ms->mma_final[0], 1);
     if (i == 11) mbar_init(&ms->mma_final[1], 1);
     if (i == 9) mbar_init(&ms->p2_go, 1);
